@@ -1,0 +1,410 @@
+"""Pins for the CPU oracle: facts that do not come from the oracle's own code.
+
+Each test states what fixes the expected value: a hand-worked fixture (with its
+source under tests/golden/), a closed form, an invariant of optimal prefix codes,
+brute force on tiny alphabets, a textbook Huffman built here with heapq, or a
+library routine (torch's fp32->bf16 conversion, NumPy's float64 matrix product).
+"""
+import heapq
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+
+def _golden_rows(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line
+
+
+# ---------------------------------------------------------------- canonical codes
+
+def test_canonical_codes_rfc1951_example(golden_dir):
+    rows = [r.split() for r in _golden_rows(golden_dir, "canonical_rfc1951.txt")]
+    lengths = np.zeros(256, np.uint8)
+    for sym, ln, _ in rows:
+        lengths[int(sym)] = int(ln)
+    codes = oracle.canonical_codes(lengths)
+    for sym, ln, bits in rows:
+        assert format(int(codes[int(sym)]), f"0{int(ln)}b") == bits
+
+
+def test_canonical_codes_prefix_free_and_ordered():
+    rng = np.random.default_rng(7)
+    for _ in range(50):
+        hist = rng.integers(0, 50, size=256)
+        hist[rng.integers(0, 256)] += 1
+        lengths = oracle.code_lengths(hist, 16)
+        codes = oracle.canonical_codes(lengths)
+        words = sorted((format(int(codes[s]), f"0{int(lengths[s])}b"), int(lengths[s]), s)
+                       for s in range(256) if lengths[s])
+        # prefix-free: in lexicographic order a prefix would sit right before its extension
+        for (a, _, _), (b, _, _) in zip(words, words[1:]):
+            assert not b.startswith(a)
+        # canonical: lexicographic order == (length, symbol) order
+        assert [s for _, _, s in words] == [s for _, _, s in sorted(words, key=lambda t: (t[1], t[2]))]
+
+
+# ---------------------------------------------------------------- code lengths
+
+def _cost(hist, lengths):
+    return int(sum(int(h) * int(l) for h, l in zip(hist, lengths)))
+
+
+def _kraft_scaled(lengths, lmax):
+    return sum(1 << (lmax - int(l)) for l in lengths if l)
+
+
+def test_code_lengths_handworked(golden_dir):
+    for row in _golden_rows(golden_dir, "lengths_handworked.txt"):
+        lmax, counts, expect, cost = [p.split() for p in row.split("|")]
+        hist = np.array([int(c) for c in counts], np.int64)
+        got = oracle.code_lengths(hist, int(lmax[0]))
+        assert [int(v) for v in got] == [int(v) for v in expect], row
+        assert _cost(hist, got) == int(cost[0]), row
+
+
+def _brute_force_cost(counts, lmax):
+    """Minimum cost over all length vectors with Kraft <= 1 and lengths <= lmax."""
+    active = sorted((c for c in counts if c > 0), reverse=True)
+    m = len(active)
+    if m == 1:
+        return active[0]
+    best = None
+    for lens in itertools.combinations_with_replacement(range(1, lmax + 1), m):
+        if sum(2.0 ** -l for l in lens) <= 1.0 + 1e-12:
+            c = sum(a * l for a, l in zip(active, lens))
+            best = c if best is None else min(best, c)
+    return best
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_code_lengths_match_brute_force(seed):
+    rng = np.random.default_rng(1000 + seed)
+    m = int(rng.integers(2, 9))
+    hist = np.zeros(16, np.int64)
+    syms = rng.choice(16, size=m, replace=False)
+    hist[syms] = rng.integers(1, 60, size=m) ** int(rng.integers(1, 3))
+    lo = max(1, math.ceil(math.log2(m)))
+    for lmax in range(lo, 8):
+        got = oracle.code_lengths(hist, lmax)
+        assert int(got.max()) <= lmax
+        assert _kraft_scaled(got, lmax) == (1 << lmax)          # complete code
+        assert _cost(hist, got) == _brute_force_cost(hist, lmax), (hist, lmax, got)
+
+
+def _textbook_huffman_lengths(hist):
+    """Unlimited Huffman code lengths with a heap (Huffman 1952)."""
+    items = [(int(h), i, (i,)) for i, h in enumerate(hist) if h > 0]
+    lengths = np.zeros(len(hist), np.int64)
+    if len(items) == 1:
+        lengths[items[0][2][0]] = 1
+        return lengths
+    heapq.heapify(items)
+    tick = len(hist)
+    while len(items) > 1:
+        w1, _, s1 = heapq.heappop(items)
+        w2, _, s2 = heapq.heappop(items)
+        for s in s1 + s2:
+            lengths[s] += 1
+        heapq.heappush(items, (w1 + w2, tick, s1 + s2))
+        tick += 1
+    return lengths
+
+
+def _entropy_np(hist):
+    p = hist[hist > 0] / hist.sum()
+    return float(-(p * np.log2(p)).sum())
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_code_lengths_vs_textbook_huffman(seed):
+    rng = np.random.default_rng(2000 + seed)
+    kind = seed % 3
+    if kind == 0:
+        hist = rng.integers(0, 1000, size=256)
+    elif kind == 1:
+        hist = np.floor(1e6 * np.exp(-0.5 * ((np.arange(256) - 128) / rng.uniform(2, 30)) ** 2))
+    else:
+        hist = np.floor(1e6 * np.exp(-np.abs(np.arange(16) - 8) / rng.uniform(0.3, 3)))
+    hist = hist.astype(np.int64)
+    if hist.sum() == 0:
+        hist[0] = 1
+    huff = _textbook_huffman_lengths(hist)
+    for lmax in (12, 16, 24):
+        if (hist > 0).sum() > (1 << lmax):
+            continue
+        got = oracle.code_lengths(hist, lmax)
+        assert int(got.max()) <= lmax
+        if (hist > 0).sum() >= 2:
+            assert _kraft_scaled(got, lmax) == (1 << lmax)
+        H = _entropy_np(hist)
+        avg = _cost(hist, got) / hist.sum()
+        assert avg >= H - 1e-12
+        if huff.max() <= lmax:
+            assert _cost(hist, got) == _cost(hist, huff)        # unlimited optimum reached
+            assert avg < H + 1.0
+        else:
+            assert _cost(hist, got) >= _cost(hist, huff)
+
+
+def test_code_lengths_limit_errors():
+    with pytest.raises(oracle.OracleError):
+        oracle.code_lengths(np.ones(256, np.int64), 7)          # 256 symbols need >= 8 bits
+    got = oracle.code_lengths(np.ones(256, np.int64), 8)
+    assert (got == 8).all()                                      # uniform over 2^k -> all k
+
+
+# ---------------------------------------------------------------- quantization
+
+def test_quantize_handworked(golden_dir):
+    for row in _golden_rows(golden_dir, "quant_handworked.txt"):
+        head, ws, scale, zero, codes = [p.split() for p in row.split("|")]
+        bits, mode = int(head[0]), int(head[1])
+        w = np.array([float(v) for v in ws], np.float32)
+        q, s, z, _ = oracle.quantize(w, bits, mode)
+        assert s == float(scale[0]), row
+        assert z == int(zero[0]), row
+        assert [int(v) for v in q] == [int(v) for v in codes], row
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("kind", ["t4", "laplace", "uniform", "skew"])
+def test_asymmetric_quantization_properties(bits, kind):
+    w = workloads.small_tensor(kind, 64, 96, seed=bits).reshape(-1)
+    q, s, z, scheme = oracle.quantize(w, bits, oracle.MODE_ASYM)
+    qmax = (1 << bits) - 1
+    assert scheme == oracle.SCHEME_ASYM
+    assert q[np.argmin(w)] == 0                                  # round(x) + round(-x) = 0
+    assert q[np.argmax(w)] >= qmax - 1
+    order = np.argsort(w, kind="stable")
+    assert (np.diff(q[order].astype(int)) >= 0).all()            # monotone
+    rec = (q.astype(np.float64) - z) * s
+    inside = (w >= (0 - z) * s) & (w <= (qmax - z) * s)
+    assert np.all(np.abs(rec - w)[inside] <= 0.5 * s * (1 + 1e-6) + 1e-7 * np.abs(w[inside]))
+    assert abs(s - (float(w.max()) - float(w.min())) / qmax) <= 1e-7 * s
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_unsigned_quantization_properties(bits):
+    w = workloads.small_tensor("shifted", 50, 70, seed=3).reshape(-1)
+    q, s, z, scheme = oracle.quantize(w, bits, oracle.MODE_UNSIGNED)
+    qmax = (1 << bits) - 1
+    assert scheme == oracle.SCHEME_UNSIGNED and z == 0
+    assert q[np.argmax(w)] == qmax and q[np.argmin(w)] == 0      # min is exactly 0 here
+    assert np.all(np.abs(q * np.float64(s) - w) <= 0.5 * s * (1 + 1e-6))
+    with pytest.raises(oracle.OracleError):
+        oracle.quantize(np.array([-1.0, 1.0], np.float32), bits, oracle.MODE_UNSIGNED)
+
+
+def test_auto_picks_lower_entropy():
+    # negative values: unsigned is not eligible, AUTO == asymmetric
+    w = workloads.small_tensor("t4", 40, 40, seed=1)
+    assert oracle.quantize(w, 8, oracle.MODE_AUTO)[3] == oracle.SCHEME_ASYM
+    # min > 0 and two close values: unsigned's coarser grid merges them (2 codes vs 3)
+    w = np.array([0.51, 0.511, 1.0, 0.51, 0.511, 1.0], np.float32)
+    qa = oracle.quantize(w, 8, oracle.MODE_ASYM)[0]
+    qu = oracle.quantize(w, 8, oracle.MODE_UNSIGNED)[0]
+    ha, hu = _entropy_np(np.bincount(qa, minlength=256)), _entropy_np(np.bincount(qu, minlength=256))
+    assert hu < ha
+    q, s, z, scheme = oracle.quantize(w, 8, oracle.MODE_AUTO)
+    assert scheme == oracle.SCHEME_UNSIGNED and (q == qu).all()
+    # shifted tensors (min == 0): both schemes coincide, the tie goes to unsigned
+    w = workloads.small_tensor("shifted", 30, 30, seed=2)
+    assert oracle.quantize(w, 8, oracle.MODE_AUTO)[3] == oracle.SCHEME_UNSIGNED
+    # in every case AUTO's entropy is the lower of the two candidates
+    for kind in ("positive", "shifted", "t4"):
+        w = workloads.small_tensor(kind, 33, 65, seed=9)
+        qauto = oracle.quantize(w, 8, oracle.MODE_AUTO)[0]
+        cands = [oracle.quantize(w, 8, oracle.MODE_ASYM)[0]]
+        if w.min() >= 0:
+            cands.append(oracle.quantize(w, 8, oracle.MODE_UNSIGNED)[0])
+        ents = [_entropy_np(np.bincount(c, minlength=256)) for c in cands]
+        assert _entropy_np(np.bincount(qauto, minlength=256)) <= min(ents) + 1e-12
+
+
+def test_quantize_special_cases():
+    q, s, z, _ = oracle.quantize(np.full(10, -0.375, np.float32), 8, oracle.MODE_AUTO)
+    assert (q == 1).all() and s == -0.375 and z == 0
+    q, s, z, _ = oracle.quantize(np.zeros(10, np.float32), 4, oracle.MODE_AUTO)
+    assert (q == 0).all() and s == 1.0 and z == 0
+    q, s, z, _ = oracle.quantize(np.zeros(0, np.float32), 8, oracle.MODE_ASYM)
+    assert q.size == 0
+    for bad in (np.nan, np.inf, -np.inf):
+        with pytest.raises(oracle.OracleError):
+            oracle.quantize(np.array([0.0, bad], np.float32), 8, oracle.MODE_ASYM)
+
+
+# ---------------------------------------------------------------- dequant (bf16 RNE)
+
+def _torch_bf16_bits(f32):
+    return torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_dequant_matches_torch_bf16_rounding():
+    rng = np.random.default_rng(11)
+    for bits in (4, 8):
+        q = rng.integers(0, 1 << bits, size=20000).astype(np.uint8)
+        for s, z in ((0.0303817, 8), (1e-3, 128), (-0.375, 0), (3.7e-5, -200), (1.0, 0)):
+            s = float(np.float32(s))
+            got = oracle.dequant_bf16(q, s, z)
+            prod = (q.astype(np.int64) - z).astype(np.float32) * np.float32(s)   # IEEE fp32 multiply
+            assert (got == _torch_bf16_bits(prod)).all()
+
+
+def test_dequant_ties_to_even():
+    # (q - z) * 1.0 with q - z chosen so that the fp32 value sits exactly halfway between
+    # two bf16 values: 257 = 0x43808000 (tie, even below), 259 = 0x43818000 (tie, odd below)
+    got = oracle.dequant_bf16(np.array([1, 3], np.uint8), 1.0, -256)
+    assert list(got) == [0x4380, 0x4382]
+    assert list(got) == list(_torch_bf16_bits(np.array([257.0, 259.0], np.float32)))
+
+
+# ---------------------------------------------------------------- GEMV
+
+def test_gemv_matches_numpy_float64():
+    rng = np.random.default_rng(5)
+    w = torch.from_numpy(rng.standard_normal((37, 300)).astype(np.float32)).to(torch.bfloat16)
+    x = torch.from_numpy(rng.standard_normal((3, 300)).astype(np.float32)).to(torch.bfloat16)
+    wb, xb = workloads.bf16_bits(w), workloads.bf16_bits(x)
+    y, mag = oracle.gemv(wb, xb)
+    ref = x.double().numpy() @ w.double().numpy().T
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    assert np.allclose(mag, np.abs(x.double().numpy()) @ np.abs(w.double().numpy()).T, rtol=1e-14)
+
+
+# ---------------------------------------------------------------- bit layout (closed forms)
+
+def _two_code_tensor(bits01):
+    """0 -> -1.0 and 1 -> 0.875: 4-bit asymmetric gives scale 0.125, zero 8, codes 0 and 15,
+    each with a 1-bit canonical code (0 -> '0', 15 -> '1')."""
+    return np.where(np.asarray(bits01) == 1, 0.875, -1.0).astype(np.float32)
+
+
+def test_lane_layout_closed_form():
+    n = 2 * 256 + 40                                     # two full lane steps + a ragged tail
+    p = np.arange(n)
+    b = ((p * 7) % 5 == 1).astype(np.uint8)
+    blob = oracle.encode(_two_code_tensor(b).reshape(1, n), 4, oracle.MODE_ASYM, 12,
+                         oracle.FMT_LANES, 1024)
+    prm = oracle.params(blob)
+    assert prm["lengths"][0] == 1 and prm["lengths"][15] == 1 and prm["lengths"].sum() == 2
+    assert prm["n_chunks"] == 1 and prm["payload_words"] == 32
+    idx = np.frombuffer(blob, np.uint64, 4, 384)
+    assert list(idx) == [0, 0, 32, n]
+    words = np.frombuffer(blob, np.uint32, 32, 384 + 32)
+    for lane in range(32):
+        seq = [int(b[q]) for t in range(3) for q in range(256 * t + 8 * lane, 256 * t + 8 * lane + 8)
+               if q < n]
+        expect = 0
+        for i, bit in enumerate(seq):
+            expect |= bit << (31 - i)
+        assert int(words[lane]) == expect, lane
+
+
+def test_single_stream_layout_closed_form():
+    n = 100
+    b = ((np.arange(n) * 3) % 7 < 3).astype(np.uint8)
+    blob = oracle.encode(_two_code_tensor(b).reshape(10, 10), 4, oracle.MODE_ASYM, 12,
+                         oracle.FMT_SINGLE, 30)
+    prm = oracle.params(blob)
+    assert prm["n_chunks"] == 4 and prm["payload_words"] == 4
+    idx = np.frombuffer(blob, np.uint64, 10, 384).reshape(5, 2)
+    assert idx[:, 0].tolist() == [0, 30, 60, 90, 100]       # bit offsets: one bit per symbol
+    assert idx[:, 1].tolist() == [0, 30, 60, 90, 100]
+    words = np.frombuffer(blob, np.uint32, 4, 384 + 80)
+    for k in range(4):
+        expect = 0
+        for i in range(32):
+            if 32 * k + i < n:
+                expect |= int(b[32 * k + i]) << (31 - i)
+        assert int(words[k]) == expect
+
+
+# ---------------------------------------------------------------- encode -> decode identity
+
+CASES = [
+    ("t4", 8, oracle.MODE_ASYM, 16, oracle.FMT_SINGLE, 4096, 64, 64),
+    ("t4", 8, oracle.MODE_ASYM, 16, oracle.FMT_SINGLE, 1000, 33, 65),
+    ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, 8192, 128, 96),
+    ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, 512, 7, 131),
+    ("t4", 8, oracle.MODE_AUTO, 16, oracle.FMT_LANES, 768, 50, 51),
+    ("shifted", 8, oracle.MODE_AUTO, 16, oracle.FMT_LANES, 256, 3, 300),
+    ("skew", 8, oracle.MODE_ASYM, 16, oracle.FMT_LANES, 16384, 200, 100),
+    ("skew", 8, oracle.MODE_ASYM, 9, oracle.FMT_LANES, 1024, 20, 100),
+    ("uniform", 8, oracle.MODE_ASYM, 16, oracle.FMT_LANES, 2048, 40, 64),
+    ("constant", 8, oracle.MODE_AUTO, 16, oracle.FMT_LANES, 256, 5, 77),
+    ("zeros", 4, oracle.MODE_AUTO, 12, oracle.FMT_SINGLE, 50, 3, 33),
+    ("two_values", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, 256, 1, 1),
+    ("t4", 4, oracle.MODE_ASYM, 4, oracle.FMT_LANES, 512, 9, 100),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}-b{c[1]}-f{c[4]}-c{c[5]}-{c[6]}x{c[7]}" for c in CASES])
+def test_encode_decode_identity(case):
+    kind, bits, mode, lmax, fmt, chunk, rows, cols = case
+    w = workloads.small_tensor(kind, rows, cols, seed=rows + cols)
+    blob = oracle.encode(w, bits, mode, lmax, fmt, chunk)
+    q, s, z, scheme = oracle.quantize(w, bits, mode)
+    assert (oracle.decode(blob) == q).all()
+    prm = oracle.params(blob)
+    assert (prm["scale"], prm["zero"], prm["scheme"]) == (s, z, scheme)
+    lengths = prm["lengths"][: 1 << bits]
+    hist = np.bincount(q, minlength=1 << bits)
+    assert int(lengths.max()) <= lmax and ((lengths > 0) == (hist > 0)).all()
+    if (hist > 0).sum() >= 2:
+        assert _kraft_scaled(lengths, lmax) == (1 << lmax)
+    # chunk-range decode agrees with the whole decode
+    if prm["n_chunks"] > 1:
+        c0, c1 = 1, prm["n_chunks"]
+        part = oracle.decode_chunks(blob, c0, c1)
+        assert (part == q[c0 * prm["chunk_symbols"]:]).all()
+
+
+def test_empty_tensor_blob():
+    blob = oracle.encode(np.zeros((0, 16), np.float32), 8, oracle.MODE_ASYM, 16, oracle.FMT_LANES, 256)
+    prm = oracle.params(blob)
+    assert prm["n"] == 0 and prm["n_chunks"] == 0 and prm["payload_words"] == 0
+    assert oracle.decode(blob).size == 0
+
+
+def test_workload_codes_statistics():
+    """The 4-bit Laplace workload: the 12-bit limit binds, Kraft stays exactly 1."""
+    W = workloads.get("laplace_4096x4096_u4")
+    w = workloads.weights(W, W.tensors[0]).numpy()[:1024]
+    q, s, z, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
+    hist = np.bincount(q, minlength=16).astype(np.int64)
+    lengths = oracle.code_lengths(hist, 12)
+    assert _kraft_scaled(lengths, 12) == 1 << 12
+    H = _entropy_np(hist)
+    avg = _cost(hist, lengths) / hist.sum()
+    assert H <= avg < H + 1
+    assert avg >= _cost(hist, _textbook_huffman_lengths(hist)) / hist.sum()
+
+
+def test_corrupted_blobs_are_rejected_or_detected():
+    w = workloads.small_tensor("laplace", 64, 128, seed=4)
+    blob = bytearray(oracle.encode(w, 4, oracle.MODE_ASYM, 12, oracle.FMT_SINGLE, 1024))
+    q = oracle.quantize(w, 4, oracle.MODE_ASYM)[0]
+    with pytest.raises(oracle.OracleError):
+        oracle.decode(bytes(blob[:-8]))                        # truncated payload
+    bad = bytearray(blob)
+    bad[0] ^= 1
+    with pytest.raises(oracle.OracleError):
+        oracle.decode(bytes(bad))                              # bad magic
+    bad = bytearray(blob)
+    bad[384 + 16] = (bad[384 + 16] + 1) % 256                  # chunk 1 starts one bit late
+    try:
+        got = oracle.decode(bytes(bad))
+        assert not (got == q).all()
+    except oracle.OracleError:
+        pass
