@@ -1,0 +1,412 @@
+"""Benchmark of the Huffman weight-decoding hot path on B200.
+
+One step = one pass of the whole hot path over the 4096x4096 4-bit Laplace
+tensor (32 word-interleaved lanes per 8192-symbol chunk):
+    decode -> packed uint4 codes, decode -> dequantize -> bf16, and the fused
+    decode -> dequantize -> GEMV (batch 1),
+each through the C ABI of libentro.  Inputs are resident in HBM; L2 is flushed
+(a 256 MiB write) before every kernel, since the whole working set would fit in
+L2.  Kernel times come from CUDA events on the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+With N > 1 (torchrun) every rank decodes its own replica of the workload (the
+chunks are independent problems; no data-path collective), and the line
+reports the whole-job rate from the slowest rank ("weak" scaling).
+--impl reference times the CPU oracle doing the same step on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "decoded Gsym/s and % HBM roofline (Huffman decode+dequant); fused GEMV tok/s"
+WORKLOAD = "laplace_4096x4096_u4"
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return dist, dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
+    return None, 0, 1, 0
+
+
+def _max_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(dist, device):
+    if dist is not None:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while running."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.bus = ""
+        if device.type == "cuda":
+            pr = torch.cuda.get_device_properties(device)
+            self.bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 10 and (not self.bus or parts[0].lower().endswith(self.bus[-10:])):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+        rows = self.rows
+        if not rows:
+            return {"samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        util = [num(r[4]) for r in rows]
+        loaded = [num(r[1]) for r in rows if num(r[4]) and num(r[4]) > 0 and num(r[1]) is not None] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": sorted(reasons), "samples": len(rows),
+                "util_max": max(u for u in util if u is not None) if any(u is not None for u in util) else None}
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+def _oracle_step(blob: bytes, chunks, threads: int, x_bits: np.ndarray):
+    """The oracle on host cores: decode the sample's chunks to codes, to bf16 weights,
+    and through the fp64 GEMV, chunk ranges split over threads (the EntroLLM
+    multi-threaded chunk decoder).  Returns symbols processed."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    p = oracle.params(blob)
+    C, K = p["chunk_symbols"], p["cols"]
+    c0, c1 = chunks
+    bounds = np.linspace(c0, c1, threads + 1).astype(int)
+
+    def work(i):
+        a, b = int(bounds[i]), int(bounds[i + 1])
+        if a >= b:
+            return 0
+        q = oracle.decode_chunks(blob, a, b)                     # pass 1: codes
+        q2 = oracle.decode_chunks(blob, a, b)                    # pass 2: codes -> bf16
+        wb = oracle.dequant_bf16(q2, p["scale"], p["zero"])
+        q3 = oracle.decode_chunks(blob, a, b)                    # pass 3: -> GEMV over the rows
+        wg = oracle.dequant_bf16(q3, p["scale"], p["zero"]).reshape(-1, K)
+        oracle.gemv(wg, x_bits)
+        return q.size + wb.size + wg.size
+
+    with ThreadPoolExecutor(threads) as ex:
+        return sum(ex.map(work, range(threads)))
+
+
+def cpu_baseline(seconds: float = 12.0):
+    import oracle
+    W = workloads.get(WORKLOAD)
+    spec = W.tensors[0]
+    w = workloads.weights(W, spec).numpy()
+    blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols))
+    p = oracle.params(blob)
+    x_bits = workloads.bf16_bits(workloads.activations(0, 1, spec.cols))
+    threads = max(1, min(os.cpu_count() or 1, 64))
+    n_chunks = p["n_chunks"]
+    total, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        total += _oracle_step(blob, (0, n_chunks), threads, x_bits)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds or reps >= 8:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": total / dt / 1e9, "unit": "Gsym/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} pass(es) of the whole {spec.rows}x{spec.cols} tensor "
+                      f"({n_chunks} chunks; codes, bf16 and GEMV passes), chunk ranges over {threads} threads, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    W = workloads.get(WORKLOAD)
+    spec = W.tensors[0]
+    w = workloads.weights(W, spec).numpy()
+    blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols))
+    p = oracle.params(blob)
+    x_bits = workloads.bf16_bits(workloads.activations(0, 1, spec.cols))
+    threads = max(1, min(os.cpu_count() or 1, 64))
+    sample = (0, min(p["n_chunks"], 256))                         # 1/8 of the tensor per step
+    for _ in range(args.warmup):
+        _oracle_step(blob, sample, threads, x_bits)
+    t0 = time.perf_counter()
+    syms = 0
+    for _ in range(args.steps):
+        syms += _oracle_step(blob, sample, threads, x_bits)
+    dt = time.perf_counter() - t0
+    value = syms / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Gsym/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u4->bf16/fp64",
+            "data": "synthetic", "config": _config(W, spec, p["chunk_symbols"]),
+            "cpu_baseline": {"value": value, "unit": "Gsym/s", "cores": threads, "kind": "oracle",
+                             "sample": f"chunks {sample[0]}..{sample[1]} of {p['n_chunks']} per step "
+                                       f"(codes, bf16 and GEMV passes) over {threads} threads"},
+            "e2e": {"value": value, "unit": "Gsym/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(W, spec, chunk):
+    return {"workload": W.name, "shape": [spec.rows, spec.cols], "bits": W.bits, "quant": "asymmetric",
+            "max_code_len": W.max_len, "chunk_symbols": chunk, "lanes": 32, "gemv_batch": 1,
+            "l2": "flushed before every kernel (256 MiB write, not timed)"}
+
+
+# ------------------------------------------------------------------ native arm
+
+def run_native(args, dist, rank, world, local_rank):
+    import huffman_decode_canonical_b200 as entro
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    W = workloads.get(WORKLOAD)
+    spec = W.tensors[0]
+    chunk = W.chunk_symbols(spec.cols)
+    w = workloads.weights(W, spec).numpy()
+    blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
+                             chunk_symbols=chunk)
+    info = blob.info()
+    dt = entro.upload(blob, device=device)
+    n = info["n"]
+    codes = dt.empty_codes()
+    bf = dt.empty_bf16()
+    x = workloads.activations(0, 1, spec.cols).to(device)
+    y = torch.empty((1, spec.rows), dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    kernels = [("codes", lambda: dt.decode_codes(out=codes, status=status)),
+               ("bf16", lambda: dt.decode_dequant_bf16(out=bf, status=status)),
+               ("gemv", lambda: dt.decode_gemv(x, y=y, status=status))]
+
+    def step(evs=None):
+        for i, (_, fn) in enumerate(kernels):
+            flush.fill_(i + 1)
+            if evs is not None:
+                evs[2 * i].record(stream)
+            fn()
+            if evs is not None:
+                evs[2 * i + 1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    clocks.start()
+    # untimed burn-in so that clock samples cover a loaded GPU even for short runs
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        step()
+        torch.cuda.synchronize(device)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    _barrier(dist, device)
+    torch.cuda.synchronize(device)
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        step(events[s])
+    torch.cuda.synchronize(device)
+    wall = time.perf_counter() - wall0
+    _barrier(dist, device)
+    clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    per = {name: [events[s][2 * i].elapsed_time(events[s][2 * i + 1]) for s in range(args.steps)]
+           for i, (name, _) in enumerate(kernels)}
+    mean_ms = {k: sum(v) / len(v) for k, v in per.items()}
+    step_ms = sum(mean_ms.values())
+    step_ms_max = _max_over_ranks(dist, step_ms, device)
+    bf16_ms_max = _max_over_ranks(dist, mean_ms["bf16"], device)
+
+    # algorithmic bytes per launch: coded bits (no lane padding) + chunk index + output
+    coded = info["coded_bits"] / 8.0
+    index = info["index_bytes"]
+    alg = {"codes": coded + index + dt.codes_nbytes(), "bf16": coded + index + 2.0 * n,
+           "gemv": coded + index + 2.0 * spec.cols + 4.0 * spec.rows}
+    peak, peak_kind = _peaks()
+    kern = {}
+    for k in mean_ms:
+        us = 1e3 * mean_ms[k]
+        gbs = alg[k] / (mean_ms[k] * 1e-3) / 1e9
+        kern[k] = {"us": round(us, 3), "gsym_s": round(n / (mean_ms[k] * 1e-3) / 1e9, 2),
+                   "alg_bytes": int(alg[k]), "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4)}
+    kern["gemv"]["tok_s"] = round(1.0 / (mean_ms["gemv"] * 1e-3), 1)
+    achieved = alg["bf16"] / (bf16_ms_max * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "lanes_kernel<4, bf16> (decode + dequant to bf16)",
+                "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": _traffic("bf16")}
+
+    e2e = _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status)
+    e2e["value"] = _max_over_ranks(dist, -e2e["value"], device) * -1 if dist is not None else e2e["value"]
+    if rank != 0:
+        return 0
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline()
+    value = world * 3 * n / (step_ms_max * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "Gsym/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes -> bf16 / fp32 accumulate",
+            "data": "synthetic", "config": _config(W, spec, chunk),
+            "value_definition": "symbols decoded per second over the step (3 passes of n = 16.8M symbols)",
+            "kernels": kern,
+            "bits_per_weight": {"coded": round(info["coded_bits"] / n, 4),
+                                "payload": round(8.0 * info["payload_bytes"] / n, 4),
+                                "all_in": round(8.0 * (info["payload_bytes"] + info["index_bytes"] + 16384) / n, 4)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps,
+            "clocks": clk, "wall_s_timed": round(wall, 4)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary of the current kernels, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f).get(kernel)
+    except Exception:
+        return None
+
+
+def _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status):
+    """The same step through the public API with host buffers: upload the blob's device
+    image from host memory, decode the three ways, read every result back."""
+    import ctypes
+    host_codes = torch.empty(codes.numel(), dtype=torch.uint8, pin_memory=True)
+    host_bf = torch.empty(bf.shape, dtype=torch.bfloat16, pin_memory=True)
+    host_y = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
+    nbytes = blob.device_bytes()
+    mem = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    lib = entro.lib()
+
+    def one():
+        h = ctypes.c_void_p()
+        r = lib.entro_upload(blob._h, ctypes.c_void_p(mem.data_ptr()), nbytes, ctypes.c_void_p(stream.cuda_stream),
+                             ctypes.byref(h))
+        assert r == 0
+        st = ctypes.c_void_p(status.data_ptr())
+        s = ctypes.c_void_p(stream.cuda_stream)
+        assert lib.entro_decode_codes(h, ctypes.c_void_p(codes.data_ptr()), st, s) == 0
+        assert lib.entro_decode_dequant_bf16(h, ctypes.c_void_p(bf.data_ptr()), st, s) == 0
+        assert lib.entro_decode_gemv(h, ctypes.c_void_p(x.data_ptr()), 1, ctypes.c_void_p(y.data_ptr()), st, s) == 0
+        host_codes.copy_(codes, non_blocking=True)
+        host_bf.copy_(bf, non_blocking=True)
+        host_y.copy_(y, non_blocking=True)
+        lib.entro_tensor_free(h)
+
+    reps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        one()
+    torch.cuda.synchronize(device)
+    dt_s = (time.perf_counter() - t0) / reps
+    d2h = host_codes.numel() + 2 * host_bf.numel() + 4 * host_y.numel()
+    return {"value": round(3 * n / dt_s / 1e9, 3), "unit": "Gsym/s", "h2d_bytes_per_step": int(nbytes),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(1e3 * dt_s, 4),
+            "note": "entro_upload from the blob's pageable host bytes (decode tables built on the host), "
+                    "three decodes, results copied to pinned host memory; wall clock per step"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    dist, rank, world, local_rank = _dist()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        return run_native(args, dist, rank, world, local_rank)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

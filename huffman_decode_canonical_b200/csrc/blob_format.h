@@ -1,0 +1,65 @@
+// blob_format.h -- layout of a serialized entro blob and of its device image.
+//
+// Blob (little-endian, version 1):
+//   [0, 128)    header (BlobHeader below)
+//   [128, 384)  code length of each of the 256 symbols, 0 = symbol absent
+//   index       (n_chunks + 1) entries of {u64 start, u64 first_symbol};
+//               start = bit offset of the chunk (single stream) or word offset
+//               of the chunk (lanes); the last entry holds the totals
+//   payload     payload_words x u32, codes MSB-first within each word
+//
+// Lanes format: a chunk of n_c symbols is split over 32 lanes; lane l codes
+// the runs of 8 consecutive symbols at chunk positions 256*t + 8*l + (0..7),
+// t = 0, 1, ...  Every lane of a chunk is padded with zero bits to the
+// chunk's longest lane (W_c words), and word j of lane l sits at
+// payload[chunk_start + 32*j + l], so one 128-byte row holds word j of all
+// lanes (the interleaved lanes of the LazyWeights abstract; the run of 8
+// makes each lane's output 8 adjacent weights).
+#pragma once
+#include <stdint.h>
+
+namespace entro {
+
+constexpr uint32_t kMagic = 0x52544E45u;  // "ENTR"
+constexpr uint32_t kVersion = 1;
+constexpr int kHeaderBytes = 128;
+constexpr int kLengthsBytes = 256;
+constexpr int kLanes = 32;
+constexpr int kRun = 8;
+constexpr int kStepSymbols = kLanes * kRun;  // 256 symbols per lane step
+constexpr int kMaxLutBits = 12;
+constexpr int kMaxLenLimit = 24;
+constexpr int64_t kMaxLanesChunk = 16384;
+constexpr int64_t kMaxSingleChunk = int64_t(1) << 20;
+constexpr double kMaxZero = 16777216.0;  // |zero| <= 2^24
+
+#pragma pack(push, 1)
+struct BlobHeader {
+    uint32_t magic, version, bits, scheme, max_len, format, lanes, run;
+    uint64_t rows, cols, n, chunk_symbols, n_chunks;
+    uint32_t scale_bits;
+    int32_t zero;
+    uint64_t payload_words;
+    uint8_t reserved[40];
+};
+#pragma pack(pop)
+static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
+
+inline uint64_t index_offset() { return kHeaderBytes + kLengthsBytes; }
+inline uint64_t payload_offset(uint64_t n_chunks) { return index_offset() + 16 * (n_chunks + 1); }
+
+// Device image of one tensor, all sections 256-byte aligned inside the
+// caller's allocation.
+//   lut      u32[2^lut_bits]: bits 0..4 code length (0 = longer than
+//            lut_bits or no code), bits 8..15 symbol; bits 16..31 are filled
+//            in shared memory by the kernels with the bf16 dequantized value
+//   slow     u32 limit[32] (left-justified to max_len bits), i32 offs[32],
+//            u8 sorted_symbols[256]
+//   index    copied verbatim from the blob
+//   payload  copied verbatim, followed by kPadWords zero words
+constexpr int kPadWords = 64;
+constexpr int kSlowBytes = 32 * 4 + 32 * 4 + 256;
+
+inline uint64_t align256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+}  // namespace entro

@@ -1,0 +1,1089 @@
+// decode.cu -- sm_100a kernels and the device half of the libentro C ABI.
+//
+// What runs here (EntroLLM, arXiv 2505.02380v4, abstract and "parallel
+// decoding" in the technical summary; LazyWeights, arXiv 2611.17108v1,
+// abstract: interleaved lanes, decode on demand so memory moves only coded
+// bytes):
+//   * lanes kernel: one warp per chunk of the 32-lane format.  The chunk's
+//     words are staged into shared memory with cp.async.bulk (one elected
+//     lane, mbarrier completion, double buffered per warp, no cluster
+//     multicast).  Each lane keeps a 64-bit MSB-first bit window, peeks 12
+//     bits into a shared-memory table of (length, symbol), and falls back to
+//     canonical length tables for longer codes.  Lane l emits runs of 8
+//     adjacent weights, so a warp writes 128/256/512 contiguous bytes per run
+//     (uint4 codes / uint8 codes / bf16) with one vector store per lane.
+//   * the same kernel dequantizes, w = bf16_rne(float(q - zero) * scale), with
+//     the value of every code computed once per CTA in fp32 and carried in the
+//     high half of the table entry, or feeds the bf16 weights straight into an
+//     fp32 GEMV with a warp-shuffle reduction per row (weights never touch
+//     memory).
+//   * single kernel: the one-bitstream-per-chunk format, one thread per chunk.
+// No tensor cores: the work is bit manipulation and streaming, not a dense
+// contraction.  Errors are reported through a status word, never by trapping;
+// every wait on a copy is bounded.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "blob_format.h"
+#include "entro.h"
+#include "entro_internal.h"
+
+namespace entro {
+
+constexpr int kLutSize = 1 << kMaxLutBits;  // 4096 entries, 16 KB of shared memory
+constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
+constexpr int kMaxWarps = 8;
+constexpr int kMaxBatch = 16;
+
+enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
+
+struct DevTensor {
+    const uint32_t *lut;         // [4096] length | symbol << 8
+    const uint32_t *slow_limit;  // [32]  (first[l] + count[l]) << (max_len - l)
+    const int32_t *slow_offs;    // [32]  rank of the first code of length l minus first[l]
+    const uint8_t *slow_syms;    // [256] symbols sorted by (length, symbol)
+    const uint64_t *index;       // (n_chunks + 1) x {start, first_symbol}
+    const uint32_t *payload;
+    long long n, rows, cols, chunk_symbols, n_chunks, payload_words;
+    float scale;
+    int zero, bits, max_len, format, max_chunk_words, n_codes;
+};
+
+struct GroupEntry {
+    DevTensor d;
+    void *out;               // codes or bf16 output
+    const __nv_bfloat16 *x;  // GEMV input [batch, cols]
+    float *y;                // GEMV output [batch, rows]
+    long long chunk_begin;   // prefix over entries, in chunks
+    long long sym_begin;     // prefix over entries, in symbols
+};
+
+struct LaunchArgs {
+    const GroupEntry *table;  // device array, or nullptr: use `one`
+    GroupEntry one;
+    int count;
+    int batch;
+    int x_in_smem;
+    int max_words;   // staging words per lane row (max over entries of max_chunk_words)
+    long long x_floats;  // floats reserved for x in shared memory
+    long long total_syms;
+    int32_t *status;
+};
+
+struct TensorHandle {
+    DevTensor d;
+    int device;
+    bool slow;
+    uint64_t device_bytes;
+};
+
+// ------------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ void set_status(int32_t *st, int code) {
+    if (st) atomicCAS(st, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk global -> shared copy completing on an mbarrier (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after ~1 s instead of hanging the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
+// Canonical decode of a code longer than the table's 12 bits: the code length
+// is the first l with (top max_len bits) < limit[l].  Returns a table-style
+// entry (length | symbol << 8 | value bits << 16) or a 1-bit entry after
+// flagging corruption.
+__device__ __noinline__ uint32_t slow_entry(uint64_t win, int max_len, const uint32_t *limit,
+                                            const int32_t *offs, const uint8_t *syms,
+                                            const uint32_t *vtab, int32_t *status) {
+    const uint32_t v = static_cast<uint32_t>(win >> (64 - max_len));
+    int l = kMaxLutBits + 1;
+    while (l <= max_len && v >= limit[l]) l++;
+    if (l > max_len) {
+        set_status(status, ENTRO_E_CORRUPT);
+        return 1u;
+    }
+    const uint32_t sym = syms[(offs[l] + static_cast<int>(v >> (max_len - l))) & 255];
+    return static_cast<uint32_t>(l) | (sym << 8) | vtab[sym];
+}
+
+struct Smem {
+    uint32_t *lut;
+    uint32_t *vtab;
+    uint32_t *slim;
+    int32_t *soffs;
+    uint8_t *ssyms;
+    float *xs;
+    uint64_t *bars;
+    uint32_t *stage;
+};
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// shared-memory carve-up; identical on host (sizing) and device
+__host__ __device__ inline size_t smem_layout(int warps, long long x_floats, int max_words, size_t *off_x,
+                                              size_t *off_bars, size_t *off_stage) {
+    size_t o = 0;
+    o += kLutSize * 4;  // lut
+    o += 256 * 4;       // vtab
+    o += 32 * 4 + 32 * 4 + 256;
+    o = align_up(o, 16);
+    *off_x = o;
+    o += (size_t)x_floats * 4;
+    o = align_up(o, 16);
+    *off_bars = o;
+    o += (size_t)warps * 2 * 8;
+    o = align_up(o, 128);
+    *off_stage = o;
+    o += (size_t)warps * 2 * (size_t)max_words * kLanes * 4;
+    return o;
+}
+
+__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_floats, int max_words) {
+    size_t ox, ob, os;
+    smem_layout(warps, x_floats, max_words, &ox, &ob, &os);
+    Smem s;
+    s.lut = reinterpret_cast<uint32_t *>(base);
+    s.vtab = s.lut + kLutSize;
+    s.slim = s.vtab + 256;
+    s.soffs = reinterpret_cast<int32_t *>(s.slim + 32);
+    s.ssyms = reinterpret_cast<uint8_t *>(s.soffs + 32);
+    s.xs = reinterpret_cast<float *>(base + ox);
+    s.bars = reinterpret_cast<uint64_t *>(base + ob);
+    s.stage = reinterpret_cast<uint32_t *>(base + os);
+    return s;
+}
+
+// Per-tensor tables into shared memory.  The value of code q is the
+// dequantized weight bf16_rne(float(q - zero) * scale), carried in the high
+// 16 bits of the table entry (EntroLLM: weights are stored as quantized codes
+// and dequantized for inference).
+template <int OUT, bool SLOW>
+__device__ void load_tables(const GroupEntry &g, const Smem &s, int batch, int x_in_smem, long long x_floats) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const DevTensor &d = g.d;
+    for (int q = tid; q < 256; q += nthr) {
+        uint32_t v = 0;
+        if (OUT != OUT_CODES && q < (1 << d.bits)) {
+            const float f = __fmul_rn(__int2float_rn(q - d.zero), d.scale);
+            v = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f))) << 16;
+        }
+        s.vtab[q] = v;
+    }
+    if (SLOW) {
+        for (int i = tid; i < 32; i += nthr) {
+            s.slim[i] = d.slow_limit[i];
+            s.soffs[i] = d.slow_offs[i];
+        }
+        for (int i = tid; i < 256; i += nthr) s.ssyms[i] = d.slow_syms[i];
+    }
+    if (OUT == OUT_GEMV && x_in_smem) {
+        const long long kb = (long long)d.cols * batch;
+        const long long lim = x_floats < kb ? x_floats : kb;
+        for (long long i = tid; i < lim; i += nthr) s.xs[i] = __bfloat162float(g.x[i]);
+    }
+    __syncthreads();  // vtab ready
+    const uint4 *src = reinterpret_cast<const uint4 *>(d.lut);
+    uint4 *dst = reinterpret_cast<uint4 *>(s.lut);
+    for (int i = tid; i < kLutSize / 4; i += nthr) {
+        uint4 e = __ldg(src + i);
+        if (OUT != OUT_CODES) {
+            e.x = (e.x & 0xFFFFu) | s.vtab[(e.x >> 8) & 0xFF];
+            e.y = (e.y & 0xFFFFu) | s.vtab[(e.y >> 8) & 0xFF];
+            e.z = (e.z & 0xFFFFu) | s.vtab[(e.z >> 8) & 0xFF];
+            e.w = (e.w & 0xFFFFu) | s.vtab[(e.w >> 8) & 0xFF];
+        }
+        dst[i] = e;
+    }
+    __syncthreads();
+}
+
+// Lane bit reader over a staged chunk: word j of this lane at buf[32 * j].
+struct LaneReader {
+    const uint32_t *buf;
+    int words;  // W_c
+    int j;      // next word
+    int nb;     // valid bits in win
+    uint64_t win;
+
+    __device__ __forceinline__ void refill() {
+        if (nb <= 32) {
+            const uint32_t w = (j < words) ? buf[kLanes * j] : 0u;
+            win |= static_cast<uint64_t>(w) << (32 - nb);
+            nb += 32;
+            j++;
+        }
+    }
+    __device__ __forceinline__ uint32_t next(const Smem &s, int max_len, int32_t *status, bool slow) {
+        const uint32_t idx = static_cast<uint32_t>(win >> (64 - kMaxLutBits));
+        uint32_t e = s.lut[idx];
+        if (slow && (e & 31u) == 0)
+            e = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, s.vtab, status);
+        const uint32_t len = e & 31u;
+        win <<= len;
+        nb -= static_cast<int>(len);
+        return e;
+    }
+    __device__ __forceinline__ bool overran() const { return 32LL * j - nb > 32LL * words; }
+};
+
+// Decode one full run of 8 symbols.  With max_len <= 16 one refill (>= 33
+// bits) covers two symbols; longer limits refill before every symbol.
+template <bool SLOW>
+__device__ __forceinline__ void decode_run8(LaneReader &rd, const Smem &s, int max_len, bool refill_each,
+                                            int32_t *status, uint32_t (&e)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        rd.refill();
+        e[i] = rd.next(s, max_len, status, SLOW);
+        if (SLOW && refill_each) rd.refill();
+        e[i + 1] = rd.next(s, max_len, status, SLOW);
+    }
+}
+
+template <int BITS, int OUT>
+__device__ __forceinline__ void emit_run8(const uint32_t (&e)[8], void *out, long long pos) {
+    // pos: first symbol of the run (multiple of 8)
+    if (OUT == OUT_CODES && BITS == 4) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) w |= ((e[i] >> 8) & 0xFu) << (4 * i);
+        reinterpret_cast<uint32_t *>(out)[pos >> 3] = w;
+    } else if (OUT == OUT_CODES) {
+        const uint32_t p01 = __byte_perm(e[0], e[1], 0x0051), p23 = __byte_perm(e[2], e[3], 0x0051);
+        const uint32_t p45 = __byte_perm(e[4], e[5], 0x0051), p67 = __byte_perm(e[6], e[7], 0x0051);
+        uint2 v;
+        v.x = __byte_perm(p01, p23, 0x5410);
+        v.y = __byte_perm(p45, p67, 0x5410);
+        reinterpret_cast<uint2 *>(out)[pos >> 3] = v;
+    } else if (OUT == OUT_BF16) {
+        uint4 v;
+        v.x = __byte_perm(e[0], e[1], 0x7632);
+        v.y = __byte_perm(e[2], e[3], 0x7632);
+        v.z = __byte_perm(e[4], e[5], 0x7632);
+        v.w = __byte_perm(e[6], e[7], 0x7632);
+        reinterpret_cast<uint4 *>(out)[pos >> 3] = v;
+    }
+}
+
+template <int BITS, int OUT>
+__device__ __forceinline__ void emit_partial(const uint32_t (&e)[8], int cnt, void *out, long long pos) {
+    if (OUT == OUT_CODES && BITS == 4) {
+        uint8_t *o = reinterpret_cast<uint8_t *>(out) + (pos >> 1);
+        for (int k = 0; 2 * k < cnt; k++) {
+            uint32_t b = (e[2 * k] >> 8) & 0xFu;
+            if (2 * k + 1 < cnt) b |= ((e[2 * k + 1] >> 8) & 0xFu) << 4;
+            o[k] = static_cast<uint8_t>(b);
+        }
+    } else if (OUT == OUT_CODES) {
+        uint8_t *o = reinterpret_cast<uint8_t *>(out) + pos;
+        for (int i = 0; i < cnt; i++) o[i] = static_cast<uint8_t>(e[i] >> 8);
+    } else if (OUT == OUT_BF16) {
+        uint16_t *o = reinterpret_cast<uint16_t *>(out) + pos;
+        for (int i = 0; i < cnt; i++) o[i] = static_cast<uint16_t>(e[i] >> 16);
+    }
+}
+
+__device__ __forceinline__ void load_x8(const Smem &s, const __nv_bfloat16 *xg, int x_in_smem, long long off,
+                                        float (&xv)[8]) {
+    if (x_in_smem) {
+        const float4 a = *reinterpret_cast<const float4 *>(s.xs + off);
+        const float4 b = *reinterpret_cast<const float4 *>(s.xs + off + 4);
+        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
+        xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+    } else {
+        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(xg + off));
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            xv[2 * k] = __uint_as_float(w[k] << 16);
+            xv[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Decode chunk c of entry g from its staged words.
+template <int BITS, int OUT, bool SLOW, int BPAD>
+__device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const uint32_t *buf, long long c,
+                                             int batch, int x_in_smem, int32_t *status) {
+    const DevTensor &d = g.d;
+    const int lane = threadIdx.x & 31;
+    const long long st = static_cast<long long>(d.index[2 * c]);
+    const long long nx = static_cast<long long>(d.index[2 * c + 2]);
+    const int words = static_cast<int>((nx - st) / kLanes);
+    const long long first = c * d.chunk_symbols;
+    const long long remain = d.n - first;
+    const int nc = static_cast<int>(remain < d.chunk_symbols ? remain : d.chunk_symbols);
+    const bool refill_each = SLOW && d.max_len > 16;
+    LaneReader rd{buf + lane, words, 0, 0, 0ull};
+    rd.refill();
+    rd.refill();
+    if (OUT == OUT_GEMV) {
+        const int K = static_cast<int>(d.cols);
+        const int spr = K / kStepSymbols;
+        const int rows_c = nc / K;
+        const long long row0 = first / K;
+        for (int r = 0; r < rows_c; r++) {
+            float acc[BPAD];
+#pragma unroll
+            for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
+            for (int t = 0; t < spr; t++) {
+                uint32_t e[8];
+                decode_run8<SLOW>(rd, s, d.max_len, refill_each, status, e);
+                float w[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) w[i] = __uint_as_float(e[i] & 0xFFFF0000u);
+                const long long col = static_cast<long long>(t) * kStepSymbols + 8 * lane;
+#pragma unroll
+                for (int b = 0; b < BPAD; b++) {
+                    if (b < batch) {
+                        float xv[8];
+                        load_x8(s, g.x, x_in_smem, static_cast<long long>(b) * K + col, xv);
+#pragma unroll
+                        for (int i = 0; i < 8; i++) acc[b] = __fmaf_rn(w[i], xv[i], acc[b]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < BPAD; b++) {
+                if (b < batch) {
+                    const float v = warp_sum(acc[b]);
+                    if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row0 + r] = v;
+                }
+            }
+        }
+    } else if (nc == d.chunk_symbols) {
+        const int steps = nc / kStepSymbols;
+        for (int t = 0; t < steps; t++) {
+            uint32_t e[8];
+            decode_run8<SLOW>(rd, s, d.max_len, refill_each, status, e);
+            emit_run8<BITS, OUT>(e, g.out, first + static_cast<long long>(t) * kStepSymbols + 8 * lane);
+        }
+    } else {
+        const int steps = (nc + kStepSymbols - 1) / kStepSymbols;
+        for (int t = 0; t < steps; t++) {
+            const int p0 = t * kStepSymbols + 8 * lane;
+            const int cnt = max(0, min(8, nc - p0));
+            uint32_t e[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                e[i] = 0;
+                if (i < cnt) {
+                    rd.refill();
+                    e[i] = rd.next(s, d.max_len, status, SLOW);
+                }
+            }
+            if (cnt == 8) emit_run8<BITS, OUT>(e, g.out, first + p0);
+            else if (cnt > 0) emit_partial<BITS, OUT>(e, cnt, g.out, first + p0);
+        }
+    }
+    if (rd.overran()) set_status(status, ENTRO_E_OVERRUN);
+}
+
+__device__ __forceinline__ const GroupEntry &entry_at(const LaunchArgs &a, int i) {
+    return a.table ? a.table[i] : a.one;
+}
+
+// Issue the staging copy of chunk c of d into buf (one lane).  Returns false
+// (and arrives with no bytes) when the index is inconsistent.
+__device__ __forceinline__ bool issue_chunk(const DevTensor &d, long long c, uint32_t *buf, uint64_t *bar,
+                                            int max_words) {
+    const uint64_t st = d.index[2 * c], nx = d.index[2 * c + 2];
+    const uint64_t words = nx - st;
+    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && words % kLanes == 0 &&
+                    words / kLanes <= static_cast<uint64_t>(max_words);
+    const uint32_t bytes = ok ? static_cast<uint32_t>(words * 4) : 0u;
+    mbar_arrive_expect_tx(bar, bytes);
+    if (bytes) bulk_copy_g2s(buf, d.payload + st, bytes, bar);
+    return ok;
+}
+
+template <int BITS, int OUT, bool SLOW, int BPAD>
+__global__ void __launch_bounds__(kMaxWarps * 32) lanes_kernel(const __grid_constant__ LaunchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Smem s = carve(smem_raw, warps, a.x_floats, a.max_words);
+    uint64_t *bar = s.bars + 2 * warp;
+    uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * a.max_words * kLanes;
+    const size_t buf_words = static_cast<size_t>(a.max_words) * kLanes;
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
+    }
+    fence_mbar_init();
+    __syncthreads();
+
+    // this CTA's share: chunks that start inside its symbol range
+    const long long s0 = a.total_syms * blockIdx.x / gridDim.x;
+    const long long s1 = a.total_syms * (blockIdx.x + 1) / gridDim.x;
+    // locate the entry holding s0
+    int ei = 0;
+    {
+        int lo = 0, hi = a.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (entry_at(a, mid).sym_begin <= s0) lo = mid;
+            else hi = mid - 1;
+        }
+        ei = lo;
+    }
+    uint32_t use_count[2] = {0, 0};  // completed phases per buffer
+    bool dead = false;               // this warp gave up on a copy: it only keeps the CTA's barriers
+    for (; ei < a.count; ei++) {
+        const GroupEntry &g = entry_at(a, ei);
+        if (g.sym_begin >= s1) break;
+        const long long C = g.d.chunk_symbols;
+        // chunks of this entry whose first symbol lies in [s0, s1)
+        long long ca = s0 > g.sym_begin ? (s0 - g.sym_begin + C - 1) / C : 0;
+        long long cb = (s1 - g.sym_begin + C - 1) / C;
+        if (cb > g.d.n_chunks) cb = g.d.n_chunks;
+        if (ca >= cb) continue;
+        load_tables<OUT, SLOW>(g, s, a.batch, a.x_in_smem, a.x_floats);
+        if (!dead) {
+            // warp w takes chunks ca + w, ca + w + warps, ...  double buffered
+            long long c = ca + warp;
+            int k = 0;
+            bool pending[2] = {false, false};
+            if (lane == 0) {
+                if (c < cb) issue_chunk(g.d, c, stage, bar, a.max_words);
+                if (c + warps < cb) issue_chunk(g.d, c + warps, stage + buf_words, bar + 1, a.max_words);
+            }
+            pending[0] = c < cb;
+            pending[1] = c + warps < cb;
+            for (; c < cb; c += warps, k++) {
+                const int b = k & 1;
+                const bool ok_wait = __all_sync(0xffffffffu, mbar_wait(bar + b, use_count[b] & 1));
+                if (!ok_wait) {
+                    set_status(a.status, ENTRO_E_TIMEOUT);
+                    dead = true;
+                    break;
+                }
+                use_count[b]++;
+                pending[b] = false;
+                const uint64_t st = g.d.index[2 * c], nx = g.d.index[2 * c + 2];
+                const bool ok = nx >= st && nx <= static_cast<uint64_t>(g.d.payload_words) &&
+                                (nx - st) % kLanes == 0 &&
+                                (nx - st) / kLanes <= static_cast<uint64_t>(a.max_words);
+                if (ok)
+                    decode_chunk<BITS, OUT, SLOW, BPAD>(g, s, stage + b * buf_words, c, a.batch, a.x_in_smem,
+                                                        a.status);
+                else
+                    set_status(a.status, ENTRO_E_CORRUPT);
+                __syncwarp();
+                if (c + 2 * warps < cb) {
+                    if (lane == 0) {
+                        fence_proxy_async();
+                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.max_words);
+                    }
+                    pending[b] = true;
+                }
+            }
+            if (dead) {
+                // let copies still in flight land (bounded) before shared memory is reused
+                for (int b = 0; b < 2; b++)
+                    if (pending[b]) mbar_wait(bar + b, use_count[b] & 1);
+            }
+        }
+        __syncthreads();  // every warp done with this entry's tables
+    }
+}
+
+// ------------------------------------------------------------------ single-stream format
+
+template <int BITS, int OUT, bool SLOW>
+__global__ void __launch_bounds__(128) single_kernel(const __grid_constant__ LaunchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const Smem s = carve(smem_raw, 0, 0, 0);
+    const GroupEntry &g = a.one;
+    const DevTensor &d = g.d;
+    load_tables<OUT, SLOW>(g, s, 1, 0, 0);
+    const long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= d.n_chunks) return;
+    const uint64_t bit0 = d.index[2 * c], bit1 = d.index[2 * c + 2];
+    const long long first = static_cast<long long>(d.index[2 * c + 1]);
+    const long long last = static_cast<long long>(d.index[2 * c + 3]);
+    if (bit1 < bit0 || (bit1 + 31) / 32 > static_cast<uint64_t>(d.payload_words) || last < first) {
+        set_status(a.status, ENTRO_E_CORRUPT);
+        return;
+    }
+    const long long limit_words = d.payload_words + kPadWords;
+    long long wi = static_cast<long long>(bit0 >> 5);
+    const int sh = static_cast<int>(bit0 & 31);
+    uint64_t win = (static_cast<uint64_t>(d.payload[wi]) << 32) | d.payload[wi + 1];
+    win <<= sh;
+    int nb = 64 - sh;
+    wi += 2;
+    uint8_t *o8 = reinterpret_cast<uint8_t *>(g.out);
+    uint16_t *o16 = reinterpret_cast<uint16_t *>(g.out);
+    uint32_t pending = 0;
+    for (long long p = first; p < last; p++) {
+        if (nb <= 32) {
+            const uint32_t w = wi < limit_words ? d.payload[wi] : 0u;
+            win |= static_cast<uint64_t>(w) << (32 - nb);
+            nb += 32;
+            wi++;
+        }
+        const uint32_t idx = static_cast<uint32_t>(win >> (64 - kMaxLutBits));
+        uint32_t e = s.lut[idx];
+        if (SLOW && (e & 31u) == 0) e = slow_entry(win, d.max_len, s.slim, s.soffs, s.ssyms, s.vtab, a.status);
+        const uint32_t len = e & 31u;
+        win <<= len;
+        nb -= static_cast<int>(len);
+        if (OUT == OUT_BF16) {
+            o16[p] = static_cast<uint16_t>(e >> 16);
+        } else if (BITS == 8) {
+            o8[p] = static_cast<uint8_t>(e >> 8);
+        } else {  // chunks start on even symbols (checked on the host): bytes are private
+            const uint32_t q = (e >> 8) & 0xFu;
+            if ((p & 1) == 0) {
+                pending = q;
+                if (p + 1 == last) o8[p >> 1] = static_cast<uint8_t>(pending);
+            } else {
+                o8[p >> 1] = static_cast<uint8_t>(pending | (q << 4));
+            }
+        }
+    }
+    const uint64_t consumed = 32ull * static_cast<uint64_t>(wi - static_cast<long long>(bit0 >> 5)) -
+                              static_cast<uint64_t>(nb) - static_cast<uint64_t>(sh);
+    if (consumed != bit1 - bit0) set_status(a.status, ENTRO_E_CORRUPT);
+}
+
+// ------------------------------------------------------------------ host side
+
+// Message of the last CUDA runtime error the library saw on this host thread.
+static thread_local char g_cuda_msg[160] = "";
+
+static int cuda_fail(cudaError_t e, const char *where) {
+    snprintf(g_cuda_msg, sizeof(g_cuda_msg), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+    return ENTRO_E_CUDA;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+static std::mutex g_mu;
+static std::vector<DeviceInfo> g_dev;
+
+static int device_info(int dev, DeviceInfo *out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+    DeviceInfo &di = g_dev[dev];
+    if (di.sms == 0) {
+        cudaError_t e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) {
+            di.sms = 0;
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        }
+    }
+    *out = di;
+    return ENTRO_OK;
+}
+
+static void build_tables(const uint8_t *len, int max_len, uint32_t *lut, uint32_t *limit, int32_t *offs,
+                         uint8_t *syms, int *n_codes) {
+    uint32_t code[256];
+    canonical_codes(len, code);
+    std::memset(lut, 0, kLutSize * 4);
+    int count[33] = {0};
+    int nz = 0;
+    for (int s = 0; s < 256; s++) {
+        if (!len[s]) continue;
+        nz++;
+        count[len[s]]++;
+        if (len[s] <= kMaxLutBits) {
+            const uint32_t lo = code[s] << (kMaxLutBits - len[s]);
+            const uint32_t hi = (code[s] + 1) << (kMaxLutBits - len[s]);
+            for (uint32_t i = lo; i < hi; i++) lut[i] = static_cast<uint32_t>(len[s]) | (static_cast<uint32_t>(s) << 8);
+        }
+    }
+    *n_codes = nz;
+    uint32_t first[33] = {0};
+    int base[33] = {0};
+    uint32_t c = 0;
+    int rank = 0;
+    for (int l = 1; l <= 32; l++) {
+        c = (c + static_cast<uint32_t>(count[l - 1])) << 1;
+        first[l] = c;
+        base[l] = rank;
+        rank += count[l];
+    }
+    for (int l = 0; l < 32; l++) {
+        limit[l] = 0;
+        offs[l] = 0;
+        if (l >= 1 && l <= max_len) {
+            limit[l] = (first[l] + static_cast<uint32_t>(count[l])) << (max_len - l);
+            offs[l] = base[l] - static_cast<int32_t>(first[l]);
+        }
+    }
+    int k = 0;
+    std::memset(syms, 0, 256);
+    for (int l = 1; l <= max_len; l++)
+        for (int s = 0; s < 256; s++)
+            if (len[s] == l) syms[k++] = static_cast<uint8_t>(s);
+}
+
+struct ImageLayout {
+    uint64_t lut, slow, index, payload, total;
+};
+
+static ImageLayout image_layout(const Blob &b) {
+    ImageLayout L;
+    L.lut = 0;
+    L.slow = align256(L.lut + kLutSize * 4);
+    L.index = align256(L.slow + kSlowBytes);
+    L.payload = align256(L.index + 16 * (b.header.n_chunks + 1));
+    L.total = align256(L.payload + 4 * (b.header.payload_words + kPadWords));
+    return L;
+}
+
+}  // namespace entro
+
+using namespace entro;
+
+extern "C" int entro_device_bytes(const entro_blob *blob, uint64_t *bytes) {
+    if (!blob || !bytes) return ENTRO_E_INVAL;
+    *bytes = image_layout(*reinterpret_cast<const Blob *>(blob)).total;
+    return ENTRO_OK;
+}
+
+extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_bytes, void *stream,
+                            entro_tensor **out) {
+    if (!blob || !out || !d_mem) return ENTRO_E_INVAL;
+    *out = nullptr;
+    const Blob &b = *reinterpret_cast<const Blob *>(blob);
+    const ImageLayout L = image_layout(b);
+    if (d_bytes < L.total || (reinterpret_cast<uintptr_t>(d_mem) & 255)) return ENTRO_E_INVAL;
+    if (b.header.format == ENTRO_FORMAT_LANES && b.max_chunk_words > 16384) return ENTRO_E_LIMIT;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ENTRO_E_CUDA;
+    TensorHandle *t = new (std::nothrow) TensorHandle();
+    if (!t) return ENTRO_E_NOMEM;
+    std::vector<uint8_t> host(L.index - L.lut, 0);
+    uint32_t *lut = reinterpret_cast<uint32_t *>(host.data());
+    uint32_t *limit = reinterpret_cast<uint32_t *>(host.data() + L.slow);
+    int32_t *offs = reinterpret_cast<int32_t *>(host.data() + L.slow + 128);
+    uint8_t *syms = host.data() + L.slow + 256;
+    int n_codes = 0;
+    build_tables(b.lengths, (int)b.header.max_len, lut, limit, offs, syms, &n_codes);
+    uint8_t *base = static_cast<uint8_t *>(d_mem);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint8_t *src = b.bytes.data();
+    cudaError_t e = cudaMemcpyAsync(base, host.data(), host.size(), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(base + L.index, src + index_offset(), 16 * (b.header.n_chunks + 1),
+                            cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess && b.header.payload_words)
+        e = cudaMemcpyAsync(base + L.payload, src + payload_offset(b.header.n_chunks), 4 * b.header.payload_words,
+                            cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(base + L.payload + 4 * b.header.payload_words, 0, 4 * kPadWords, st);
+    // pageable sources: make sure the host staging above is consumed before `host` dies
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        delete t;
+        return ENTRO_E_CUDA;
+    }
+    DevTensor &d = t->d;
+    d.lut = reinterpret_cast<const uint32_t *>(base + L.lut);
+    d.slow_limit = reinterpret_cast<const uint32_t *>(base + L.slow);
+    d.slow_offs = reinterpret_cast<const int32_t *>(base + L.slow + 128);
+    d.slow_syms = base + L.slow + 256;
+    d.index = reinterpret_cast<const uint64_t *>(base + L.index);
+    d.payload = reinterpret_cast<const uint32_t *>(base + L.payload);
+    d.n = (long long)b.header.n;
+    d.rows = (long long)b.header.rows;
+    d.cols = (long long)b.header.cols;
+    d.chunk_symbols = (long long)b.header.chunk_symbols;
+    d.n_chunks = (long long)b.header.n_chunks;
+    d.payload_words = (long long)b.header.payload_words;
+    std::memcpy(&d.scale, &b.header.scale_bits, 4);
+    d.zero = b.header.zero;
+    d.bits = (int)b.header.bits;
+    d.max_len = (int)b.header.max_len;
+    d.format = (int)b.header.format;
+    d.max_chunk_words = (int)b.max_chunk_words;
+    d.n_codes = n_codes;
+    t->device = dev;
+    t->slow = d.max_len > kMaxLutBits || n_codes == 1;
+    t->device_bytes = L.total;
+    *out = reinterpret_cast<entro_tensor *>(t);
+    return ENTRO_OK;
+}
+
+extern "C" void entro_tensor_free(entro_tensor *t) { delete reinterpret_cast<TensorHandle *>(t); }
+
+namespace entro {
+
+using LanesFn = void (*)(LaunchArgs);
+
+template <int BITS, int OUT, bool SLOW>
+static LanesFn pick_bpad(int bpad) {
+    if (OUT != OUT_GEMV) return lanes_kernel<BITS, OUT, SLOW, 1>;
+    switch (bpad) {
+        case 1: return lanes_kernel<BITS, OUT, SLOW, 1>;
+        case 2: return lanes_kernel<BITS, OUT, SLOW, 2>;
+        case 4: return lanes_kernel<BITS, OUT, SLOW, 4>;
+        case 8: return lanes_kernel<BITS, OUT, SLOW, 8>;
+        default: return lanes_kernel<BITS, OUT, SLOW, 16>;
+    }
+}
+
+static LanesFn pick_lanes(int bits, int out, bool slow, int bpad) {
+    if (bits == 4) {
+        if (out == OUT_CODES) return slow ? pick_bpad<4, OUT_CODES, true>(1) : pick_bpad<4, OUT_CODES, false>(1);
+        if (out == OUT_BF16) return slow ? pick_bpad<4, OUT_BF16, true>(1) : pick_bpad<4, OUT_BF16, false>(1);
+        return slow ? pick_bpad<4, OUT_GEMV, true>(bpad) : pick_bpad<4, OUT_GEMV, false>(bpad);
+    }
+    if (out == OUT_CODES) return slow ? pick_bpad<8, OUT_CODES, true>(1) : pick_bpad<8, OUT_CODES, false>(1);
+    if (out == OUT_BF16) return slow ? pick_bpad<8, OUT_BF16, true>(1) : pick_bpad<8, OUT_BF16, false>(1);
+    return slow ? pick_bpad<8, OUT_GEMV, true>(bpad) : pick_bpad<8, OUT_GEMV, false>(bpad);
+}
+
+static LanesFn pick_single(int bits, int out, bool slow) {
+    if (bits == 4) {
+        if (out == OUT_CODES) return slow ? single_kernel<4, OUT_CODES, true> : single_kernel<4, OUT_CODES, false>;
+        return slow ? single_kernel<4, OUT_BF16, true> : single_kernel<4, OUT_BF16, false>;
+    }
+    if (out == OUT_CODES) return slow ? single_kernel<8, OUT_CODES, true> : single_kernel<8, OUT_CODES, false>;
+    return slow ? single_kernel<8, OUT_BF16, true> : single_kernel<8, OUT_BF16, false>;
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory and report how many CTAs
+// of `threads` fit on one SM.  The opt-in attribute only ever grows (it is a
+// per-kernel maximum, so a smaller later launch must not lower it below a
+// larger cached one); occupancy is cached per (kernel, device, threads, bytes).
+struct KernelConfig {
+    const void *fn;
+    int device, threads;
+    size_t bytes;
+    int per_sm;
+};
+struct KernelOptIn {
+    const void *fn;
+    int device;
+    size_t bytes;
+};
+static std::vector<KernelConfig> g_kcfg;
+static std::vector<KernelOptIn> g_optin;
+
+static int kernel_config(const void *fn, int device, int threads, size_t bytes, int *per_sm) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    KernelOptIn *opt = nullptr;
+    for (KernelOptIn &o : g_optin)
+        if (o.fn == fn && o.device == device) opt = &o;
+    if (!opt || opt->bytes < bytes) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        if (opt) opt->bytes = bytes;
+        else g_optin.push_back({fn, device, bytes});
+    }
+    for (const KernelConfig &k : g_kcfg)
+        if (k.fn == fn && k.device == device && k.threads == threads && k.bytes == bytes) {
+            *per_sm = k.per_sm;
+            return ENTRO_OK;
+        }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (n < 1) {
+        snprintf(g_cuda_msg, sizeof(g_cuda_msg), "no CTA of %d threads and %zu bytes fits an SM", threads, bytes);
+        return ENTRO_E_CUDA;
+    }
+    g_kcfg.push_back({fn, device, threads, bytes, n});
+    *per_sm = n;
+    return ENTRO_OK;
+}
+
+static int bpad_for(int batch) {
+    int b = 1;
+    while (b < batch) b <<= 1;
+    return b;
+}
+
+static constexpr long long kXSmemFloats = 24 * 1024;  // up to 96 KB of fp32 activations per CTA
+
+// Launch the lanes kernel over `count` entries (table on device, or `one`).
+static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
+                        const GroupEntry &one, int32_t *status, cudaStream_t st) {
+    bool slow = false;
+    int bits = ts[0]->d.bits, max_words = 1;
+    long long max_kb = 0, total = 0;
+    for (int i = 0; i < count; i++) {
+        const DevTensor &d = ts[i]->d;
+        if (d.bits != bits) return ENTRO_E_INVAL;
+        slow = slow || ts[i]->slow;
+        max_words = std::max(max_words, d.max_chunk_words);
+        max_kb = std::max(max_kb, d.cols * (long long)bpad_for(batch));
+        total += d.n;
+    }
+    if (total == 0) return ENTRO_OK;
+    DeviceInfo di;
+    if (device_info(ts[0]->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
+    const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
+    long long x_floats = (out_kind == OUT_GEMV && max_kb <= kXSmemFloats) ? max_kb : 0;
+    int warps = kMaxWarps;
+    size_t ox, ob, os, bytes = 0;
+    for (;;) {
+        bytes = smem_layout(warps, x_floats, max_words, &ox, &ob, &os);
+        if ((int)bytes <= di.smem_optin) break;
+        if (warps > 1) warps >>= 1;
+        else if (x_floats) { x_floats = 0; warps = kMaxWarps; }
+        else return ENTRO_E_LIMIT;
+    }
+    LanesFn fn = pick_lanes(bits, out_kind, slow, bpad);
+    int per_sm = 0;
+    if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, bytes, &per_sm) != ENTRO_OK)
+        return ENTRO_E_CUDA;
+    long long chunks = 0;
+    for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
+    long long grid = std::min<long long>((chunks + warps - 1) / warps, (long long)per_sm * di.sms);
+    grid = std::max<long long>(grid, 1);
+    LaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.table = d_table;
+    a.one = one;
+    a.count = count;
+    a.batch = batch;
+    a.x_in_smem = x_floats > 0;
+    a.max_words = max_words;
+    a.x_floats = x_floats;
+    a.total_syms = total;
+    a.status = status;
+    fn<<<(unsigned)grid, warps * 32, bytes, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
+}
+
+static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t *status, cudaStream_t st) {
+    const DevTensor &d = t->d;
+    if (d.n_chunks == 0) return ENTRO_OK;
+    LanesFn fn = pick_single(d.bits, out_kind, t->slow);
+    size_t ox, ob, os;
+    const size_t bytes = smem_layout(0, 0, 0, &ox, &ob, &os);
+    const int threads = 32;
+    int per_sm = 0;
+    if (kernel_config(reinterpret_cast<const void *>(fn), t->device, threads, bytes, &per_sm) != ENTRO_OK)
+        return ENTRO_E_CUDA;
+    LaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.one.d = d;
+    a.one.out = out;
+    a.count = 1;
+    a.batch = 1;
+    a.status = status;
+    const long long grid = (d.n_chunks + threads - 1) / threads;
+    fn<<<(unsigned)grid, threads, bytes, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "single kernel launch");
+}
+
+static int decode_one(const entro_tensor *tensor, int out_kind, void *out, int32_t *status, void *stream) {
+    if (!tensor) return ENTRO_E_INVAL;
+    const TensorHandle *t = reinterpret_cast<const TensorHandle *>(tensor);
+    if (t->d.n == 0) return ENTRO_OK;  // nothing to decode; `out` may be null
+    if (!out) return ENTRO_E_INVAL;
+    if (reinterpret_cast<uintptr_t>(out) & 15) return ENTRO_E_INVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (t->d.format == ENTRO_FORMAT_SINGLE) {
+        if (out_kind == OUT_CODES && t->d.bits == 4 && (t->d.chunk_symbols & 1)) return ENTRO_E_INVAL;
+        return launch_single(t, out_kind, out, status, st);
+    }
+    GroupEntry one;
+    std::memset(&one, 0, sizeof(one));
+    one.d = t->d;
+    one.out = out;
+    return launch_lanes(&t, 1, out_kind, 1, nullptr, one, status, st);
+}
+
+static int gemv_check(const TensorHandle *t, const void *x, int batch, const float *y) {
+    if (!t || !x || !y || batch < 1 || batch > kMaxBatch) return ENTRO_E_INVAL;
+    if (reinterpret_cast<uintptr_t>(x) & 15) return ENTRO_E_INVAL;
+    const DevTensor &d = t->d;
+    if (d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
+    if (d.cols <= 0 || d.cols % kStepSymbols || d.chunk_symbols % d.cols) return ENTRO_E_INVAL;
+    return ENTRO_OK;
+}
+
+}  // namespace entro
+
+extern "C" int entro_decode_codes(const entro_tensor *t, void *d_out, int32_t *d_status, void *stream) {
+    return decode_one(t, OUT_CODES, d_out, d_status, stream);
+}
+
+extern "C" int entro_decode_dequant_bf16(const entro_tensor *t, void *d_out, int32_t *d_status, void *stream) {
+    return decode_one(t, OUT_BF16, d_out, d_status, stream);
+}
+
+extern "C" int entro_decode_gemv(const entro_tensor *tensor, const void *d_x, int32_t batch, float *d_y,
+                                 int32_t *d_status, void *stream) {
+    const TensorHandle *t = reinterpret_cast<const TensorHandle *>(tensor);
+    int r = gemv_check(t, d_x, batch, d_y);
+    if (r != ENTRO_OK) return r;
+    GroupEntry one;
+    std::memset(&one, 0, sizeof(one));
+    one.d = t->d;
+    one.x = static_cast<const __nv_bfloat16 *>(d_x);
+    one.y = d_y;
+    return launch_lanes(&t, 1, OUT_GEMV, batch, nullptr, one, d_status, static_cast<cudaStream_t>(stream));
+}
+
+namespace entro {
+struct GroupHandle {
+    std::vector<const TensorHandle *> ts;
+    GroupEntry first;
+    const GroupEntry *d_table;
+    int kind;
+    int batch;
+};
+}  // namespace entro
+
+extern "C" uint64_t entro_group_table_bytes(int32_t count) {
+    return count > 0 ? align256(sizeof(GroupEntry) * (uint64_t)count) : 0;
+}
+
+extern "C" int entro_group_prepare(const entro_tensor *const *tensors, int32_t count, int32_t kind,
+                                   const void *const *xs, float *const *ys, void *const *outs, int32_t batch,
+                                   void *d_table, uint64_t table_bytes, void *stream, entro_group **out) {
+    if (!out) return ENTRO_E_INVAL;
+    *out = nullptr;
+    if (!tensors || count < 1 || !d_table || (reinterpret_cast<uintptr_t>(d_table) & 255)) return ENTRO_E_INVAL;
+    if (kind != ENTRO_GROUP_GEMV && kind != ENTRO_GROUP_BF16) return ENTRO_E_INVAL;
+    if (table_bytes < entro_group_table_bytes(count)) return ENTRO_E_INVAL;
+    const int out_kind = kind == ENTRO_GROUP_GEMV ? OUT_GEMV : OUT_BF16;
+    if (out_kind == OUT_GEMV && (!xs || !ys)) return ENTRO_E_INVAL;
+    if (out_kind == OUT_BF16 && !outs) return ENTRO_E_INVAL;
+    GroupHandle *h = new (std::nothrow) GroupHandle();
+    if (!h) return ENTRO_E_NOMEM;
+    std::vector<GroupEntry> host((size_t)count);
+    h->ts.resize((size_t)count);
+    long long chunks = 0, syms = 0;
+    for (int i = 0; i < count; i++) {
+        const TensorHandle *t = reinterpret_cast<const TensorHandle *>(tensors[i]);
+        int r = ENTRO_OK;
+        if (!t || t->d.format != ENTRO_FORMAT_LANES) r = ENTRO_E_INVAL;
+        else if (out_kind == OUT_GEMV) r = gemv_check(t, xs[i], batch, ys[i]);
+        else if (!outs[i] || (reinterpret_cast<uintptr_t>(outs[i]) & 15)) r = ENTRO_E_INVAL;
+        if (r == ENTRO_OK && i > 0 && (t->device != h->ts[0]->device || t->d.bits != h->ts[0]->d.bits))
+            r = ENTRO_E_INVAL;
+        if (r != ENTRO_OK) {
+            delete h;
+            return r;
+        }
+        h->ts[i] = t;
+        GroupEntry &g = host[i];
+        std::memset(&g, 0, sizeof(g));
+        g.d = t->d;
+        if (out_kind == OUT_GEMV) {
+            g.x = static_cast<const __nv_bfloat16 *>(xs[i]);
+            g.y = ys[i];
+        } else {
+            g.out = outs[i];
+        }
+        g.chunk_begin = chunks;
+        g.sym_begin = syms;
+        chunks += t->d.n_chunks;
+        syms += t->d.n;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(d_table, host.data(), sizeof(GroupEntry) * (size_t)count, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        delete h;
+        return ENTRO_E_CUDA;
+    }
+    h->first = host[0];
+    h->d_table = static_cast<const GroupEntry *>(d_table);
+    h->kind = out_kind;
+    h->batch = out_kind == OUT_GEMV ? batch : 1;
+    *out = reinterpret_cast<entro_group *>(h);
+    return ENTRO_OK;
+}
+
+extern "C" int entro_group_launch(const entro_group *group, int32_t *d_status, void *stream) {
+    if (!group) return ENTRO_E_INVAL;
+    const GroupHandle *h = reinterpret_cast<const GroupHandle *>(group);
+    return launch_lanes(h->ts.data(), (int)h->ts.size(), h->kind, h->batch, h->d_table, h->first, d_status,
+                        static_cast<cudaStream_t>(stream));
+}
+
+extern "C" void entro_group_free(entro_group *group) { delete reinterpret_cast<GroupHandle *>(group); }
+
+extern "C" const char *entro_strerror(int code) {
+    switch (code) {
+        case ENTRO_OK: return "ok";
+        case ENTRO_E_INVAL: return "invalid argument";
+        case ENTRO_E_LIMIT: return "outside a documented limit";
+        case ENTRO_E_FORMAT: return "malformed blob";
+        case ENTRO_E_CORRUPT: return "corrupt coded data (no code matches)";
+        case ENTRO_E_OVERRUN: return "coded stream ran past its chunk";
+        case ENTRO_E_NOMEM: return "out of host memory";
+        case ENTRO_E_CUDA: return "CUDA runtime error";
+        case ENTRO_E_TIMEOUT: return "bounded wait on a copy gave up";
+        default: return "unknown error";
+    }
+}
+
+extern "C" int entro_version(void) { return 100; }
+
+extern "C" const char *entro_last_cuda_error(void) { return g_cuda_msg; }
