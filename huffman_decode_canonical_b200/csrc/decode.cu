@@ -37,15 +37,17 @@
 
 namespace entro {
 
-constexpr int kLutSize = 1 << kMaxLutBits;  // 4096 entries, 16 KB of shared memory
+constexpr int kLutSize = 1 << kMaxLutBits;   // 4096 entries, 16 KB of shared memory
 constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
-constexpr int kMaxWarps = 8;
+constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
+constexpr int kSlackRows = 2;                 // staging rows past a chunk's longest lane (read-ahead)
 
 enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
 
 struct DevTensor {
-    const uint32_t *lut;         // [4096] length | symbol << 8
+    const uint32_t *lut;         // [4096] one code per entry: length | symbol << 8
+    const uint32_t *mlut;        // [4096] several codes per entry: bits | count << 4 | symbols << 8
     const uint32_t *slow_limit;  // [32]  (first[l] + count[l]) << (max_len - l)
     const int32_t *slow_offs;    // [32]  rank of the first code of length l minus first[l]
     const uint8_t *slow_syms;    // [256] symbols sorted by (length, symbol)
@@ -71,8 +73,9 @@ struct LaunchArgs {
     int count;
     int batch;
     int x_in_smem;
-    int max_words;   // staging words per lane row (max over entries of max_chunk_words)
-    long long x_floats;  // floats reserved for x in shared memory
+    int stage_rows;       // rows of 32 words per staging buffer (longest chunk + slack)
+    int out_words;        // per-warp code staging, 32-bit words
+    long long x_elems;    // bf16 activations held in shared memory
     long long total_syms;
     int32_t *status;
 };
@@ -141,13 +144,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// acc += lo(w2) * lo(x2), then acc += hi(w2) * hi(x2): bf16 operands, fp32
+// accumulation with one rounding per step (the same value as an fp32 FMA of
+// the widened operands).
+__device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w2), "r"(x2));
+    return acc;
+}
+
 // Canonical decode of a code longer than the table's 12 bits: the code length
-// is the first l with (top max_len bits) < limit[l].  Returns a table-style
-// entry (length | symbol << 8 | value bits << 16) or a 1-bit entry after
-// flagging corruption.
+// is the first l with (top max_len bits) < limit[l].  Returns length | symbol
+// << 8, or a 1-bit entry after flagging corruption.
 __device__ __noinline__ uint32_t slow_entry(uint64_t win, int max_len, const uint32_t *limit,
-                                            const int32_t *offs, const uint8_t *syms,
-                                            const uint32_t *vtab, int32_t *status) {
+                                            const int32_t *offs, const uint8_t *syms, int32_t *status) {
     const uint32_t v = static_cast<uint32_t>(win >> (64 - max_len));
     int l = kMaxLutBits + 1;
     while (l <= max_len && v >= limit[l]) l++;
@@ -156,202 +171,107 @@ __device__ __noinline__ uint32_t slow_entry(uint64_t win, int max_len, const uin
         return 1u;
     }
     const uint32_t sym = syms[(offs[l] + static_cast<int>(v >> (max_len - l))) & 255];
-    return static_cast<uint32_t>(l) | (sym << 8) | vtab[sym];
+    return static_cast<uint32_t>(l) | (sym << 8);
 }
 
 struct Smem {
-    uint32_t *lut;
-    uint32_t *vtab;
+    uint32_t *lut;    // decode table (multi-symbol for the lanes kernel)
+    uint32_t *vtab;   // bf16 value of each code, low half
+    uint32_t *vpair;  // 4-bit: bf16 values of the two codes of a byte
     uint32_t *slim;
     int32_t *soffs;
     uint8_t *ssyms;
-    float *xs;
+    __nv_bfloat16 *xs;
+    uint64_t *tbar;   // CTA barrier for the table copies
     uint64_t *bars;
     uint32_t *stage;
+    uint32_t *ostage;
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+struct SmemOffsets {
+    size_t x, bars, stage, ostage, total;
+};
+
 // shared-memory carve-up; identical on host (sizing) and device
-__host__ __device__ inline size_t smem_layout(int warps, long long x_floats, int max_words, size_t *off_x,
-                                              size_t *off_bars, size_t *off_stage) {
-    size_t o = 0;
-    o += kLutSize * 4;  // lut
-    o += 256 * 4;       // vtab
-    o += 32 * 4 + 32 * 4 + 256;
-    o = align_up(o, 16);
-    *off_x = o;
-    o += (size_t)x_floats * 4;
-    o = align_up(o, 16);
-    *off_bars = o;
-    o += (size_t)warps * 2 * 8;
-    o = align_up(o, 128);
-    *off_stage = o;
-    o += (size_t)warps * 2 * (size_t)max_words * kLanes * 4;
+__host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_rows, int out_words) {
+    SmemOffsets o;
+    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
+    p = align_up(p, 16);
+    o.x = p;
+    p += (size_t)x_elems * 2;
+    p = align_up(p, 16);
+    o.bars = p;
+    p += (size_t)(warps + 1) * 2 * 8;
+    p = align_up(p, 128);
+    o.stage = p;
+    p += (size_t)warps * 2 * (size_t)stage_rows * kLanes * 4;
+    p = align_up(p, 16);
+    o.ostage = p;
+    p += (size_t)warps * (size_t)out_words * 4;
+    o.total = p;
     return o;
 }
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_floats, int max_words) {
-    size_t ox, ob, os;
-    smem_layout(warps, x_floats, max_words, &ox, &ob, &os);
+__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_rows, int out_words) {
+    const SmemOffsets o = smem_layout(warps, x_elems, stage_rows, out_words);
     Smem s;
     s.lut = reinterpret_cast<uint32_t *>(base);
     s.vtab = s.lut + kLutSize;
-    s.slim = s.vtab + 256;
+    s.vpair = s.vtab + 256;
+    s.slim = s.vpair + 256;
     s.soffs = reinterpret_cast<int32_t *>(s.slim + 32);
     s.ssyms = reinterpret_cast<uint8_t *>(s.soffs + 32);
-    s.xs = reinterpret_cast<float *>(base + ox);
-    s.bars = reinterpret_cast<uint64_t *>(base + ob);
-    s.stage = reinterpret_cast<uint32_t *>(base + os);
+    s.xs = reinterpret_cast<__nv_bfloat16 *>(base + o.x);
+    s.tbar = reinterpret_cast<uint64_t *>(base + o.bars);
+    s.bars = s.tbar + 2;
+    s.stage = reinterpret_cast<uint32_t *>(base + o.stage);
+    s.ostage = reinterpret_cast<uint32_t *>(base + o.ostage);
     return s;
 }
 
-// Per-tensor tables into shared memory.  The value of code q is the
-// dequantized weight bf16_rne(float(q - zero) * scale), carried in the high
-// 16 bits of the table entry (EntroLLM: weights are stored as quantized codes
-// and dequantized for inference).
+__device__ __forceinline__ uint32_t dequant_bf16_bits(int q, int zero, float scale) {
+    const float f = __fmul_rn(__int2float_rn(q - zero), scale);
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+// Per-tensor tables into shared memory.  vtab[q] is the dequantized weight
+// bf16_rne(float(q - zero) * scale) (EntroLLM: weights are kept as quantized
+// codes and dequantized for inference), computed here in fp32 once per CTA;
+// vpair[b] holds the values of both 4-bit codes of byte b.  The decode table,
+// the canonical tables and (GEMV) the activations arrive by bulk copies on the
+// CTA barrier; thread 0 issues them at phase `tphase`.
 template <int OUT, bool SLOW>
-__device__ void load_tables(const GroupEntry &g, const Smem &s, int batch, int x_in_smem, long long x_floats) {
+__device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int batch, int x_in_smem) {
+    if (threadIdx.x != 0) return;
+    const DevTensor &d = g.d;
+    uint32_t bytes = kLutSize * 4;
+    if (SLOW) bytes += kSlowBytes;
+    const uint32_t xbytes = (OUT == OUT_GEMV && x_in_smem) ? static_cast<uint32_t>(d.cols * batch * 2) : 0u;
+    bytes += xbytes;
+    mbar_arrive_expect_tx(s.tbar, bytes);
+    bulk_copy_g2s(s.lut, multi ? d.mlut : d.lut, kLutSize * 4, s.tbar);
+    if (SLOW) bulk_copy_g2s(s.slim, d.slow_limit, kSlowBytes, s.tbar);
+    if (xbytes) bulk_copy_g2s(s.xs, g.x, xbytes, s.tbar);
+}
+
+template <int OUT, bool SLOW>
+__device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphase) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const DevTensor &d = g.d;
-    for (int q = tid; q < 256; q += nthr) {
-        uint32_t v = 0;
-        if (OUT != OUT_CODES && q < (1 << d.bits)) {
-            const float f = __fmul_rn(__int2float_rn(q - d.zero), d.scale);
-            v = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f))) << 16;
+    if (OUT != OUT_CODES) {
+        for (int q = tid; q < 256; q += nthr) {
+            const uint32_t v = q < (1 << d.bits) ? dequant_bf16_bits(q, d.zero, d.scale) : 0u;
+            s.vtab[q] = v;
+            if (d.bits == 4)
+                s.vpair[q] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
+                             (dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
         }
-        s.vtab[q] = v;
     }
-    if (SLOW) {
-        for (int i = tid; i < 32; i += nthr) {
-            s.slim[i] = d.slow_limit[i];
-            s.soffs[i] = d.slow_offs[i];
-        }
-        for (int i = tid; i < 256; i += nthr) s.ssyms[i] = d.slow_syms[i];
-    }
-    if (OUT == OUT_GEMV && x_in_smem) {
-        const long long kb = (long long)d.cols * batch;
-        const long long lim = x_floats < kb ? x_floats : kb;
-        for (long long i = tid; i < lim; i += nthr) s.xs[i] = __bfloat162float(g.x[i]);
-    }
-    __syncthreads();  // vtab ready
-    const uint4 *src = reinterpret_cast<const uint4 *>(d.lut);
-    uint4 *dst = reinterpret_cast<uint4 *>(s.lut);
-    for (int i = tid; i < kLutSize / 4; i += nthr) {
-        uint4 e = __ldg(src + i);
-        if (OUT != OUT_CODES) {
-            e.x = (e.x & 0xFFFFu) | s.vtab[(e.x >> 8) & 0xFF];
-            e.y = (e.y & 0xFFFFu) | s.vtab[(e.y >> 8) & 0xFF];
-            e.z = (e.z & 0xFFFFu) | s.vtab[(e.z >> 8) & 0xFF];
-            e.w = (e.w & 0xFFFFu) | s.vtab[(e.w >> 8) & 0xFF];
-        }
-        dst[i] = e;
-    }
+    const bool ok = mbar_wait(s.tbar, tphase & 1);
     __syncthreads();
-}
-
-// Lane bit reader over a staged chunk: word j of this lane at buf[32 * j].
-struct LaneReader {
-    const uint32_t *buf;
-    int words;  // W_c
-    int j;      // next word
-    int nb;     // valid bits in win
-    uint64_t win;
-
-    __device__ __forceinline__ void refill() {
-        if (nb <= 32) {
-            const uint32_t w = (j < words) ? buf[kLanes * j] : 0u;
-            win |= static_cast<uint64_t>(w) << (32 - nb);
-            nb += 32;
-            j++;
-        }
-    }
-    __device__ __forceinline__ uint32_t next(const Smem &s, int max_len, int32_t *status, bool slow) {
-        const uint32_t idx = static_cast<uint32_t>(win >> (64 - kMaxLutBits));
-        uint32_t e = s.lut[idx];
-        if (slow && (e & 31u) == 0)
-            e = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, s.vtab, status);
-        const uint32_t len = e & 31u;
-        win <<= len;
-        nb -= static_cast<int>(len);
-        return e;
-    }
-    __device__ __forceinline__ bool overran() const { return 32LL * j - nb > 32LL * words; }
-};
-
-// Decode one full run of 8 symbols.  With max_len <= 16 one refill (>= 33
-// bits) covers two symbols; longer limits refill before every symbol.
-template <bool SLOW>
-__device__ __forceinline__ void decode_run8(LaneReader &rd, const Smem &s, int max_len, bool refill_each,
-                                            int32_t *status, uint32_t (&e)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-        rd.refill();
-        e[i] = rd.next(s, max_len, status, SLOW);
-        if (SLOW && refill_each) rd.refill();
-        e[i + 1] = rd.next(s, max_len, status, SLOW);
-    }
-}
-
-template <int BITS, int OUT>
-__device__ __forceinline__ void emit_run8(const uint32_t (&e)[8], void *out, long long pos) {
-    // pos: first symbol of the run (multiple of 8)
-    if (OUT == OUT_CODES && BITS == 4) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int i = 0; i < 8; i++) w |= ((e[i] >> 8) & 0xFu) << (4 * i);
-        reinterpret_cast<uint32_t *>(out)[pos >> 3] = w;
-    } else if (OUT == OUT_CODES) {
-        const uint32_t p01 = __byte_perm(e[0], e[1], 0x0051), p23 = __byte_perm(e[2], e[3], 0x0051);
-        const uint32_t p45 = __byte_perm(e[4], e[5], 0x0051), p67 = __byte_perm(e[6], e[7], 0x0051);
-        uint2 v;
-        v.x = __byte_perm(p01, p23, 0x5410);
-        v.y = __byte_perm(p45, p67, 0x5410);
-        reinterpret_cast<uint2 *>(out)[pos >> 3] = v;
-    } else if (OUT == OUT_BF16) {
-        uint4 v;
-        v.x = __byte_perm(e[0], e[1], 0x7632);
-        v.y = __byte_perm(e[2], e[3], 0x7632);
-        v.z = __byte_perm(e[4], e[5], 0x7632);
-        v.w = __byte_perm(e[6], e[7], 0x7632);
-        reinterpret_cast<uint4 *>(out)[pos >> 3] = v;
-    }
-}
-
-template <int BITS, int OUT>
-__device__ __forceinline__ void emit_partial(const uint32_t (&e)[8], int cnt, void *out, long long pos) {
-    if (OUT == OUT_CODES && BITS == 4) {
-        uint8_t *o = reinterpret_cast<uint8_t *>(out) + (pos >> 1);
-        for (int k = 0; 2 * k < cnt; k++) {
-            uint32_t b = (e[2 * k] >> 8) & 0xFu;
-            if (2 * k + 1 < cnt) b |= ((e[2 * k + 1] >> 8) & 0xFu) << 4;
-            o[k] = static_cast<uint8_t>(b);
-        }
-    } else if (OUT == OUT_CODES) {
-        uint8_t *o = reinterpret_cast<uint8_t *>(out) + pos;
-        for (int i = 0; i < cnt; i++) o[i] = static_cast<uint8_t>(e[i] >> 8);
-    } else if (OUT == OUT_BF16) {
-        uint16_t *o = reinterpret_cast<uint16_t *>(out) + pos;
-        for (int i = 0; i < cnt; i++) o[i] = static_cast<uint16_t>(e[i] >> 16);
-    }
-}
-
-__device__ __forceinline__ void load_x8(const Smem &s, const __nv_bfloat16 *xg, int x_in_smem, long long off,
-                                        float (&xv)[8]) {
-    if (x_in_smem) {
-        const float4 a = *reinterpret_cast<const float4 *>(s.xs + off);
-        const float4 b = *reinterpret_cast<const float4 *>(s.xs + off + 4);
-        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
-        xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
-    } else {
-        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(xg + off));
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            xv[2 * k] = __uint_as_float(w[k] << 16);
-            xv[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-        }
-    }
+    return __syncthreads_and(ok);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -360,10 +280,202 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Decode chunk c of entry g from its staged words.
+// ------------------------------------------------------------------ phase 1: one lane's stream
+//
+// The lane keeps a 64-bit MSB-first window of its bitstream.  One 12-bit peek
+// into the multi-symbol table yields up to 6 (4-bit) or 3 (8-bit) symbols and
+// the bits they take; codes longer than 12 bits go through the canonical
+// slow path.  Symbols collect in a pending register; every 8 form one run,
+// written to the warp's code stage at word 32*t + lane (4-bit) or double-word
+// 32*t + lane (8-bit), i.e. in output order, without bank conflicts.
+
+template <int BITS, bool SLOW>
+struct LaneDecoder {
+    const uint32_t *buf;  // word j of this lane at buf[32 * j]
+    uint32_t *ost;        // this lane's first staged run; run t at ost[32 * t] (words or double-words)
+    uint32_t *sink;       // a private scratch slot that absorbs not-ready stores
+    int jcap, j, nb;
+    uint64_t win;
+    uint64_t pend;        // pending symbols, first at bit 0
+    uint32_t pend_hi;     // 8-bit: symbols 8.. of the pending set
+    int pc;               // pending count
+    int t;                // runs stored
+
+    __device__ __forceinline__ void refill() {
+        const uint32_t w = buf[kLanes * min(j, jcap)];
+        if (nb <= 32) {
+            win |= static_cast<uint64_t>(w) << (32 - nb);
+            nb += 32;
+            j++;
+        }
+    }
+
+    // one table lookup; appends its symbols to the pending set
+    __device__ __forceinline__ void lookup(const Smem &s, int max_len, int32_t *status) {
+        const uint32_t e = s.lut[static_cast<uint32_t>(win >> (64 - kMaxLutBits))];
+        uint32_t cnt = (e >> 4) & 15u, syms = e >> 8, bits = e & 15u;
+        if (SLOW && cnt == 0) {
+            const uint32_t se = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, status);
+            bits = se & 31u;
+            syms = (se >> 8) & 0xFFu;
+            cnt = 1;
+        }
+        win <<= bits;
+        nb -= static_cast<int>(bits);
+        if (BITS == 4) {
+            pend |= static_cast<uint64_t>(syms) << (4 * pc);
+        } else {
+            const int sh = 8 * pc;  // < 64: appends happen only while fewer than 8 are pending
+            pend |= static_cast<uint64_t>(syms) << sh;
+            if (sh > 40) pend_hi |= syms >> (64 - sh);
+        }
+        pc += static_cast<int>(cnt);
+    }
+
+    // After a lookup at most one run is complete (pending < 16).  The store is
+    // issued either way -- to the run's slot when ready, else to the sink --
+    // so the warp stays converged.
+    __device__ __forceinline__ void emit(int full_runs) {
+        const bool ready = pc >= 8 && t < full_runs;
+        if (BITS == 4) {
+            uint32_t *dst = ready ? ost + kLanes * t : sink;
+            *dst = static_cast<uint32_t>(pend);
+            if (ready) pend >>= 32;
+        } else {
+            uint64_t *dst = ready ? reinterpret_cast<uint64_t *>(ost) + kLanes * t : reinterpret_cast<uint64_t *>(sink);
+            *dst = pend;
+            if (ready) {
+                pend = pend_hi;
+                pend_hi = 0;
+            }
+        }
+        pc -= ready ? 8 : 0;
+        t += ready ? 1 : 0;
+    }
+};
+
+// ------------------------------------------------------------------ phase 2: stage -> output
+
+// 8 codes of run-word w -> 8 bf16 values (4 words, value of code 8w+i in half i)
+template <int BITS>
+__device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int w) {
+    uint4 v;
+    if (BITS == 4) {
+        const uint32_t c = ost[w];
+        v.x = s.vpair[c & 0xFFu];
+        v.y = s.vpair[(c >> 8) & 0xFFu];
+        v.z = s.vpair[(c >> 16) & 0xFFu];
+        v.w = s.vpair[c >> 24];
+    } else {
+        const uint2 c = reinterpret_cast<const uint2 *>(ost)[w];
+        v.x = __byte_perm(s.vtab[c.x & 0xFFu], s.vtab[(c.x >> 8) & 0xFFu], 0x5410);
+        v.y = __byte_perm(s.vtab[(c.x >> 16) & 0xFFu], s.vtab[c.x >> 24], 0x5410);
+        v.z = __byte_perm(s.vtab[c.y & 0xFFu], s.vtab[(c.y >> 8) & 0xFFu], 0x5410);
+        v.w = __byte_perm(s.vtab[(c.y >> 16) & 0xFFu], s.vtab[c.y >> 24], 0x5410);
+    }
+    return v;
+}
+
+// Emit runs [tb, te) of a whole chunk (every lane owns 8 codes per run).
+template <int BITS, int OUT, int BPAD>
+__device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
+                                          int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD]) {
+    const DevTensor &d = g.d;
+    const int lane = threadIdx.x & 31;
+    if (OUT == OUT_CODES) {
+        // staged codes are packed and in output order: 16-byte copies
+        constexpr int kU4PerRun = kLanes * BITS / 16;  // uint4 per run of the warp (8 or 16)
+        const uint4 *src = reinterpret_cast<const uint4 *>(ost) + tb * kU4PerRun;
+        uint4 *dst = reinterpret_cast<uint4 *>(g.out) + first * BITS / 128 + tb * kU4PerRun;
+        for (int i = lane; i < (te - tb) * kU4PerRun; i += kLanes) dst[i] = src[i];
+    } else if (OUT == OUT_BF16) {
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(g.out) + first);
+        for (int t = tb; t < te; t++) dst[kLanes * t + lane] = values8<BITS>(s, ost, kLanes * t + lane);
+    } else {
+        // fused GEMV: run t covers columns 256*(t % spr) + 8*lane .. +7 of row t / spr
+        const int K = static_cast<int>(d.cols);
+        const int spr = K / kStepSymbols;
+        const long long row0 = first / K;
+        const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
+        const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
+        for (int t = tb; t < te; t++) {
+            const int st = t % spr;
+            const uint4 wv = values8<BITS>(s, ost, kLanes * t + lane);
+            const int xo = st * kLanes + lane;  // uint4 index within one x row
+#pragma unroll
+            for (int b = 0; b < BPAD; b++) {
+                if (b < batch) {
+                    const int xi = b * (K >> 3) + xo;
+                    const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                    acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
+                    acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
+                    acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
+                    acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
+                }
+            }
+            if (st == spr - 1) {
+                const long long row = row0 + t / spr;
+#pragma unroll
+                for (int b = 0; b < BPAD; b++) {
+                    if (b < batch) {
+                        const float v = warp_sum(acc[b]);
+                        if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row] = v;
+                    }
+                    acc[b] = 0.f;
+                }
+            }
+        }
+    }
+}
+
+// Emit a ragged (last) chunk of nc codes after the whole chunk was staged.
+template <int BITS, int OUT>
+__device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
+                                            int nc) {
+    const int lane = threadIdx.x & 31;
+    const int words = (nc + 7) >> 3;
+    if (OUT == OUT_CODES) {
+        uint8_t *o = reinterpret_cast<uint8_t *>(g.out) + first * BITS / 8;
+        for (int w = lane; w < words; w += kLanes) {
+            const int cnt = min(8, nc - 8 * w);
+            if (BITS == 4) {
+                const uint32_t c = ost[w];
+                for (int k = 0; 2 * k < cnt; k++) {
+                    uint32_t b = (c >> (8 * k)) & 0xFFu;
+                    if (2 * k + 1 >= cnt) b &= 0xFu;
+                    o[4 * w + k] = static_cast<uint8_t>(b);
+                }
+            } else {
+                const uint8_t *c = reinterpret_cast<const uint8_t *>(ost) + 8 * w;
+                for (int k = 0; k < cnt; k++) o[8 * w + k] = c[k];
+            }
+        }
+    } else if (OUT == OUT_BF16) {
+        for (int w = lane; w < words; w += kLanes) {
+            const uint4 v = values8<BITS>(s, ost, w);
+            uint16_t *o = reinterpret_cast<uint16_t *>(g.out) + first + 8 * w;
+            const int cnt = min(8, nc - 8 * w);
+            if (cnt == 8) {
+                *reinterpret_cast<uint4 *>(o) = v;
+            } else {
+                for (int k = 0; k < cnt; k++) {
+                    const uint32_t pair = (k < 2) ? v.x : (k < 4) ? v.y : (k < 6) ? v.z : v.w;
+                    o[k] = static_cast<uint16_t>(pair >> (16 * (k & 1)));
+                }
+            }
+        }
+    }
+}
+
+constexpr int kEmitBlock = 8;  // runs decoded between two emission rounds
+
+// Decode chunk c of entry g from its staged words.  Whole chunks are emitted
+// every kEmitBlock runs, so the stores of one block drain while the lanes
+// decode the next.
 template <int BITS, int OUT, bool SLOW, int BPAD>
-__device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const uint32_t *buf, long long c,
-                                             int batch, int x_in_smem, int32_t *status) {
+__device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const uint32_t *buf,
+                                             uint32_t *ost, int stage_rows, long long c, int batch, int x_in_smem,
+                                             int32_t *status) {
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
     const long long st = static_cast<long long>(d.index[2 * c]);
@@ -373,108 +485,119 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
     const long long remain = d.n - first;
     const int nc = static_cast<int>(remain < d.chunk_symbols ? remain : d.chunk_symbols);
     const bool refill_each = SLOW && d.max_len > 16;
-    LaneReader rd{buf + lane, words, 0, 0, 0ull};
-    rd.refill();
-    rd.refill();
-    if (OUT == OUT_GEMV) {
-        const int K = static_cast<int>(d.cols);
-        const int spr = K / kStepSymbols;
-        const int rows_c = nc / K;
-        const long long row0 = first / K;
-        for (int r = 0; r < rows_c; r++) {
-            float acc[BPAD];
+    uint32_t *lost = ost + (BITS == 4 ? lane : 2 * lane);
+    uint32_t *sink = ost + (static_cast<size_t>(d.chunk_symbols) * BITS / 32) + (BITS == 4 ? lane : 2 * lane);
+    LaneDecoder<BITS, SLOW> ld;
+    ld.buf = buf + lane;
+    ld.ost = lost;
+    ld.sink = sink;
+    ld.jcap = stage_rows - 1;
+    ld.j = 0;
+    ld.nb = 0;
+    ld.win = 0;
+    ld.pend = 0;
+    ld.pend_hi = 0;
+    ld.pc = 0;
+    ld.t = 0;
+    ld.refill();
+    ld.refill();
+    bool ok = true;
+    if (nc == d.chunk_symbols) {
+        const int runs = nc / kStepSymbols;
+        float acc[BPAD];
 #pragma unroll
-            for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
-            for (int t = 0; t < spr; t++) {
-                uint32_t e[8];
-                decode_run8<SLOW>(rd, s, d.max_len, refill_each, status, e);
-                float w[8];
-#pragma unroll
-                for (int i = 0; i < 8; i++) w[i] = __uint_as_float(e[i] & 0xFFFF0000u);
-                const long long col = static_cast<long long>(t) * kStepSymbols + 8 * lane;
-#pragma unroll
-                for (int b = 0; b < BPAD; b++) {
-                    if (b < batch) {
-                        float xv[8];
-                        load_x8(s, g.x, x_in_smem, static_cast<long long>(b) * K + col, xv);
-#pragma unroll
-                        for (int i = 0; i < 8; i++) acc[b] = __fmaf_rn(w[i], xv[i], acc[b]);
-                    }
-                }
+        for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
+        for (int tb = 0; tb < runs; tb += kEmitBlock) {
+            const int te = min(tb + kEmitBlock, runs);
+            while (ld.t < te) {
+                ld.refill();
+                ld.lookup(s, d.max_len, status);
+                ld.emit(runs);
+                if (SLOW && refill_each) ld.refill();
+                ld.lookup(s, d.max_len, status);
+                ld.emit(runs);
             }
-#pragma unroll
-            for (int b = 0; b < BPAD; b++) {
-                if (b < batch) {
-                    const float v = warp_sum(acc[b]);
-                    if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row0 + r] = v;
-                }
-            }
+            __syncwarp();
+            emit_runs<BITS, OUT, BPAD>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
         }
-    } else if (nc == d.chunk_symbols) {
-        const int steps = nc / kStepSymbols;
-        for (int t = 0; t < steps; t++) {
-            uint32_t e[8];
-            decode_run8<SLOW>(rd, s, d.max_len, refill_each, status, e);
-            emit_run8<BITS, OUT>(e, g.out, first + static_cast<long long>(t) * kStepSymbols + 8 * lane);
-        }
+        ok = ld.j <= words + kSlackRows;
     } else {
-        const int steps = (nc + kStepSymbols - 1) / kStepSymbols;
-        for (int t = 0; t < steps; t++) {
-            const int p0 = t * kStepSymbols + 8 * lane;
-            const int cnt = max(0, min(8, nc - p0));
-            uint32_t e[8];
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                e[i] = 0;
-                if (i < cnt) {
-                    rd.refill();
-                    e[i] = rd.next(s, d.max_len, status, SLOW);
-                }
+        // symbols of this lane: positions 256*t + 8*lane + i < nc
+        const int full_steps = nc / kStepSymbols, rem = nc % kStepSymbols;
+        const int S = 8 * full_steps + max(0, min(8, rem - 8 * lane));
+        const int full_runs = S >> 3, tail = S & 7;
+        if (S > 0) {
+            while (ld.t < full_runs) {
+                ld.refill();
+                ld.lookup(s, d.max_len, status);
+                ld.emit(full_runs);
+                if (SLOW && refill_each) ld.refill();
+                ld.lookup(s, d.max_len, status);
+                ld.emit(full_runs);
             }
-            if (cnt == 8) emit_run8<BITS, OUT>(e, g.out, first + p0);
-            else if (cnt > 0) emit_partial<BITS, OUT>(e, cnt, g.out, first + p0);
+            if (tail) {
+                while (ld.pc < tail) {
+                    ld.refill();
+                    ld.lookup(s, d.max_len, status);
+                }
+                if (BITS == 4) lost[kLanes * ld.t] = static_cast<uint32_t>(ld.pend);
+                else reinterpret_cast<uint64_t *>(lost)[kLanes * ld.t] = ld.pend;
+            }
+            ok = ld.j <= words + kSlackRows;
         }
+        __syncwarp();
+        emit_ragged<BITS, OUT>(g, s, ost, first, nc);
     }
-    if (rd.overran()) set_status(status, ENTRO_E_OVERRUN);
+    if (!ok) set_status(status, ENTRO_E_OVERRUN);
+    __syncwarp();
 }
 
 __device__ __forceinline__ const GroupEntry &entry_at(const LaunchArgs &a, int i) {
     return a.table ? a.table[i] : a.one;
 }
 
-// Issue the staging copy of chunk c of d into buf (one lane).  Returns false
-// (and arrives with no bytes) when the index is inconsistent.
-__device__ __forceinline__ bool issue_chunk(const DevTensor &d, long long c, uint32_t *buf, uint64_t *bar,
-                                            int max_words) {
+__device__ __forceinline__ bool chunk_words_ok(const DevTensor &d, long long c, int stage_rows) {
     const uint64_t st = d.index[2 * c], nx = d.index[2 * c + 2];
-    const uint64_t words = nx - st;
-    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && words % kLanes == 0 &&
-                    words / kLanes <= static_cast<uint64_t>(max_words);
-    const uint32_t bytes = ok ? static_cast<uint32_t>(words * 4) : 0u;
+    return nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % kLanes == 0 &&
+           (nx - st) / kLanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
+}
+
+// Issue the staging copy of a chunk whose words are [st, nx) (one lane).  An
+// inconsistent index arrives with no bytes; the consumer re-checks and skips.
+__device__ __forceinline__ void issue_words(const DevTensor &d, uint64_t st, uint64_t nx, uint32_t *buf,
+                                            uint64_t *bar, int stage_rows) {
+    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % kLanes == 0 &&
+                    (nx - st) / kLanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
+    const uint32_t bytes = ok ? static_cast<uint32_t>((nx - st) * 4) : 0u;
     mbar_arrive_expect_tx(bar, bytes);
     if (bytes) bulk_copy_g2s(buf, d.payload + st, bytes, bar);
-    return ok;
+}
+
+__device__ __forceinline__ void issue_chunk(const DevTensor &d, long long c, uint32_t *buf, uint64_t *bar,
+                                            int stage_rows) {
+    issue_words(d, d.index[2 * c], d.index[2 * c + 2], buf, bar, stage_rows);
 }
 
 template <int BITS, int OUT, bool SLOW, int BPAD>
-__global__ void __launch_bounds__(kMaxWarps * 32) lanes_kernel(const __grid_constant__ LaunchArgs a) {
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Smem s = carve(smem_raw, warps, a.x_floats, a.max_words);
+    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows, a.out_words);
     uint64_t *bar = s.bars + 2 * warp;
-    uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * a.max_words * kLanes;
-    const size_t buf_words = static_cast<size_t>(a.max_words) * kLanes;
+    const size_t buf_words = static_cast<size_t>(a.stage_rows) * kLanes;
+    uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
+    uint32_t *ost = s.ostage + static_cast<size_t>(warp) * a.out_words;
     if (lane == 0) {
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
     }
+    if (threadIdx.x == 0) mbar_init(s.tbar, 1);
     fence_mbar_init();
     __syncthreads();
 
     // this CTA's share: chunks that start inside its symbol range
     const long long s0 = a.total_syms * blockIdx.x / gridDim.x;
     const long long s1 = a.total_syms * (blockIdx.x + 1) / gridDim.x;
-    // locate the entry holding s0
     int ei = 0;
     {
         int lo = 0, hi = a.count - 1;
@@ -485,62 +608,73 @@ __global__ void __launch_bounds__(kMaxWarps * 32) lanes_kernel(const __grid_cons
         }
         ei = lo;
     }
-    uint32_t use_count[2] = {0, 0};  // completed phases per buffer
-    bool dead = false;               // this warp gave up on a copy: it only keeps the CTA's barriers
+    uint32_t phase0 = 0, phase1 = 0;  // completed phases of the two staging buffers
+    uint32_t tphase = 0;              // completed phases of the table barrier
+    bool dead = false;                // this warp gave up on a copy: it only keeps the CTA's barriers
     for (; ei < a.count; ei++) {
         const GroupEntry &g = entry_at(a, ei);
         if (g.sym_begin >= s1) break;
         const long long C = g.d.chunk_symbols;
-        // chunks of this entry whose first symbol lies in [s0, s1)
         long long ca = s0 > g.sym_begin ? (s0 - g.sym_begin + C - 1) / C : 0;
         long long cb = (s1 - g.sym_begin + C - 1) / C;
         if (cb > g.d.n_chunks) cb = g.d.n_chunks;
         if (ca >= cb) continue;
-        load_tables<OUT, SLOW>(g, s, a.batch, a.x_in_smem, a.x_floats);
+        issue_tables<OUT, SLOW>(g, s, true, a.batch, a.x_in_smem);
+        // warp w takes chunks ca + w, ca + w + warps, ...  double buffered.  The
+        // index entries of the first two are read by four lanes at once, and
+        // both copies fly while the tables arrive.
+        long long c = ca + warp;
+        bool pend0 = false, pend1 = false;
         if (!dead) {
-            // warp w takes chunks ca + w, ca + w + warps, ...  double buffered
-            long long c = ca + warp;
-            int k = 0;
-            bool pending[2] = {false, false};
+            const long long cq = (lane < 2) ? c : c + warps;
+            uint64_t iv = 0;
+            if (lane < 4 && cq < cb) iv = g.d.index[2 * cq + 2 * (lane & 1)];
+            const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
+            const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
             if (lane == 0) {
-                if (c < cb) issue_chunk(g.d, c, stage, bar, a.max_words);
-                if (c + warps < cb) issue_chunk(g.d, c + warps, stage + buf_words, bar + 1, a.max_words);
+                if (c < cb) issue_words(g.d, st0, nx0, stage, bar, a.stage_rows);
+                if (c + warps < cb) issue_words(g.d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows);
             }
-            pending[0] = c < cb;
-            pending[1] = c + warps < cb;
-            for (; c < cb; c += warps, k++) {
+            pend0 = c < cb;
+            pend1 = c + warps < cb;
+        }
+        const bool tables_ok = finish_tables<OUT, SLOW>(g, s, tphase);
+        tphase++;
+        if (!tables_ok) {
+            set_status(a.status, ENTRO_E_TIMEOUT);
+            dead = true;
+        }
+        if (!dead) {
+            for (int k = 0; c < cb; c += warps, k++) {
                 const int b = k & 1;
-                const bool ok_wait = __all_sync(0xffffffffu, mbar_wait(bar + b, use_count[b] & 1));
+                const uint32_t phase = b ? phase1 : phase0;
+                const bool ok_wait = __all_sync(0xffffffffu, mbar_wait(bar + b, phase & 1));
                 if (!ok_wait) {
                     set_status(a.status, ENTRO_E_TIMEOUT);
                     dead = true;
                     break;
                 }
-                use_count[b]++;
-                pending[b] = false;
-                const uint64_t st = g.d.index[2 * c], nx = g.d.index[2 * c + 2];
-                const bool ok = nx >= st && nx <= static_cast<uint64_t>(g.d.payload_words) &&
-                                (nx - st) % kLanes == 0 &&
-                                (nx - st) / kLanes <= static_cast<uint64_t>(a.max_words);
-                if (ok)
-                    decode_chunk<BITS, OUT, SLOW, BPAD>(g, s, stage + b * buf_words, c, a.batch, a.x_in_smem,
-                                                        a.status);
+                if (b) { phase1++; pend1 = false; }
+                else { phase0++; pend0 = false; }
+                if (chunk_words_ok(g.d, c, a.stage_rows))
+                    decode_chunk<BITS, OUT, SLOW, BPAD>(g, s, stage + b * buf_words, ost, a.stage_rows, c, a.batch,
+                                                        a.x_in_smem, a.status);
                 else
                     set_status(a.status, ENTRO_E_CORRUPT);
-                __syncwarp();
                 if (c + 2 * warps < cb) {
                     if (lane == 0) {
                         fence_proxy_async();
-                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.max_words);
+                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows);
                     }
-                    pending[b] = true;
+                    if (b) pend1 = true;
+                    else pend0 = true;
                 }
             }
-            if (dead) {
-                // let copies still in flight land (bounded) before shared memory is reused
-                for (int b = 0; b < 2; b++)
-                    if (pending[b]) mbar_wait(bar + b, use_count[b] & 1);
-            }
+        }
+        if (dead) {
+            // let copies still in flight land (bounded) before shared memory is reused
+            if (pend0) mbar_wait(bar, phase0 & 1);
+            if (pend1) mbar_wait(bar + 1, phase1 & 1);
         }
         __syncthreads();  // every warp done with this entry's tables
     }
@@ -551,10 +685,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32) lanes_kernel(const __grid_cons
 template <int BITS, int OUT, bool SLOW>
 __global__ void __launch_bounds__(128) single_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    const Smem s = carve(smem_raw, 0, 0, 0);
+    const Smem s = carve(smem_raw, 0, 0, 0, 0);
     const GroupEntry &g = a.one;
     const DevTensor &d = g.d;
-    load_tables<OUT, SLOW>(g, s, 1, 0, 0);
+    if (threadIdx.x == 0) mbar_init(s.tbar, 1);
+    fence_mbar_init();
+    __syncthreads();
+    issue_tables<OUT, SLOW>(g, s, false, 1, 0);
+    if (!finish_tables<OUT, SLOW>(g, s, 0)) {
+        set_status(a.status, ENTRO_E_TIMEOUT);
+        return;
+    }
     const long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (c >= d.n_chunks) return;
     const uint64_t bit0 = d.index[2 * c], bit1 = d.index[2 * c + 2];
@@ -581,23 +722,22 @@ __global__ void __launch_bounds__(128) single_kernel(const __grid_constant__ Lau
             nb += 32;
             wi++;
         }
-        const uint32_t idx = static_cast<uint32_t>(win >> (64 - kMaxLutBits));
-        uint32_t e = s.lut[idx];
-        if (SLOW && (e & 31u) == 0) e = slow_entry(win, d.max_len, s.slim, s.soffs, s.ssyms, s.vtab, a.status);
+        uint32_t e = s.lut[static_cast<uint32_t>(win >> (64 - kMaxLutBits))];
+        if (SLOW && (e & 31u) == 0) e = slow_entry(win, d.max_len, s.slim, s.soffs, s.ssyms, a.status);
         const uint32_t len = e & 31u;
+        const uint32_t sym = (e >> 8) & 0xFFu;
         win <<= len;
         nb -= static_cast<int>(len);
         if (OUT == OUT_BF16) {
-            o16[p] = static_cast<uint16_t>(e >> 16);
+            o16[p] = static_cast<uint16_t>(s.vtab[sym]);
         } else if (BITS == 8) {
-            o8[p] = static_cast<uint8_t>(e >> 8);
+            o8[p] = static_cast<uint8_t>(sym);
         } else {  // chunks start on even symbols (checked on the host): bytes are private
-            const uint32_t q = (e >> 8) & 0xFu;
             if ((p & 1) == 0) {
-                pending = q;
+                pending = sym;
                 if (p + 1 == last) o8[p >> 1] = static_cast<uint8_t>(pending);
             } else {
-                o8[p >> 1] = static_cast<uint8_t>(pending | (q << 4));
+                o8[p >> 1] = static_cast<uint8_t>(pending | (sym << 4));
             }
         }
     }
@@ -640,8 +780,13 @@ static int device_info(int dev, DeviceInfo *out) {
     return ENTRO_OK;
 }
 
-static void build_tables(const uint8_t *len, int max_len, uint32_t *lut, uint32_t *limit, int32_t *offs,
-                         uint8_t *syms, int *n_codes) {
+// Host-built decode tables of one tensor (canonical codes, RFC 1951 order).
+//   lut:  12-bit peek -> (length, symbol) of the first code, 0 if longer than 12
+//   mlut: 12-bit peek -> every whole code inside the 12 bits, up to 6 (4-bit)
+//         or 3 (8-bit): bits used | count << 4 | symbols << 8
+//   limit / offs / syms: canonical description for codes longer than 12 bits
+static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lut, uint32_t *mlut,
+                         uint32_t *limit, int32_t *offs, uint8_t *syms, int *n_codes) {
     uint32_t code[256];
     canonical_codes(len, code);
     std::memset(lut, 0, kLutSize * 4);
@@ -658,6 +803,19 @@ static void build_tables(const uint8_t *len, int max_len, uint32_t *lut, uint32_
         }
     }
     *n_codes = nz;
+    const int per = bits == 4 ? 6 : 3;
+    for (uint32_t v = 0; v < (uint32_t)kLutSize; v++) {
+        uint32_t used = 0, k = 0, packed = 0;
+        while ((int)k < per) {
+            const uint32_t e = lut[(v << used) & (kLutSize - 1)];
+            const uint32_t l = e & 31u;
+            if (l == 0 || used + l > (uint32_t)kMaxLutBits) break;
+            packed |= ((e >> 8) & 0xFFu) << (bits * k);
+            used += l;
+            k++;
+        }
+        mlut[v] = used | (k << 4) | (packed << 8);
+    }
     uint32_t first[33] = {0};
     int base[33] = {0};
     uint32_t c = 0;
@@ -684,13 +842,14 @@ static void build_tables(const uint8_t *len, int max_len, uint32_t *lut, uint32_
 }
 
 struct ImageLayout {
-    uint64_t lut, slow, index, payload, total;
+    uint64_t lut, mlut, slow, index, payload, total;
 };
 
 static ImageLayout image_layout(const Blob &b) {
     ImageLayout L;
     L.lut = 0;
-    L.slow = align256(L.lut + kLutSize * 4);
+    L.mlut = align256(L.lut + kLutSize * 4);
+    L.slow = align256(L.mlut + kLutSize * 4);
     L.index = align256(L.slow + kSlowBytes);
     L.payload = align256(L.index + 16 * (b.header.n_chunks + 1));
     L.total = align256(L.payload + 4 * (b.header.payload_words + kPadWords));
@@ -721,11 +880,12 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     if (!t) return ENTRO_E_NOMEM;
     std::vector<uint8_t> host(L.index - L.lut, 0);
     uint32_t *lut = reinterpret_cast<uint32_t *>(host.data());
+    uint32_t *mlut = reinterpret_cast<uint32_t *>(host.data() + L.mlut);
     uint32_t *limit = reinterpret_cast<uint32_t *>(host.data() + L.slow);
     int32_t *offs = reinterpret_cast<int32_t *>(host.data() + L.slow + 128);
     uint8_t *syms = host.data() + L.slow + 256;
     int n_codes = 0;
-    build_tables(b.lengths, (int)b.header.max_len, lut, limit, offs, syms, &n_codes);
+    build_tables(b.lengths, (int)b.header.max_len, (int)b.header.bits, lut, mlut, limit, offs, syms, &n_codes);
     uint8_t *base = static_cast<uint8_t *>(d_mem);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint8_t *src = b.bytes.data();
@@ -746,6 +906,7 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     }
     DevTensor &d = t->d;
     d.lut = reinterpret_cast<const uint32_t *>(base + L.lut);
+    d.mlut = reinterpret_cast<const uint32_t *>(base + L.mlut);
     d.slow_limit = reinterpret_cast<const uint32_t *>(base + L.slow);
     d.slow_offs = reinterpret_cast<const int32_t *>(base + L.slow + 128);
     d.slow_syms = base + L.slow + 256;
@@ -861,19 +1022,21 @@ static int bpad_for(int batch) {
     return b;
 }
 
-static constexpr long long kXSmemFloats = 24 * 1024;  // up to 96 KB of fp32 activations per CTA
+static constexpr long long kXSmemElems = 48 * 1024;  // up to 96 KB of bf16 activations per CTA
 
 // Launch the lanes kernel over `count` entries (table on device, or `one`).
 static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
                         const GroupEntry &one, int32_t *status, cudaStream_t st) {
     bool slow = false;
-    int bits = ts[0]->d.bits, max_words = 1;
-    long long max_kb = 0, total = 0;
+    const int bits = ts[0]->d.bits;
+    int max_words = 0;
+    long long max_kb = 0, max_chunk = 0, total = 0;
     for (int i = 0; i < count; i++) {
         const DevTensor &d = ts[i]->d;
         if (d.bits != bits) return ENTRO_E_INVAL;
         slow = slow || ts[i]->slow;
         max_words = std::max(max_words, d.max_chunk_words);
+        max_chunk = std::max(max_chunk, d.chunk_symbols);
         max_kb = std::max(max_kb, d.cols * (long long)bpad_for(batch));
         total += d.n;
     }
@@ -881,22 +1044,27 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     DeviceInfo di;
     if (device_info(ts[0]->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
-    long long x_floats = (out_kind == OUT_GEMV && max_kb <= kXSmemFloats) ? max_kb : 0;
-    int warps = kMaxWarps;
-    size_t ox, ob, os, bytes = 0;
+    long long x_elems = (out_kind == OUT_GEMV && max_kb <= kXSmemElems) ? max_kb : 0;
+    const int stage_rows = max_words + kSlackRows;
+    const int out_words = static_cast<int>(max_chunk * bits / 32) + 2 * kLanes;  // + the not-ready sink
+    long long chunks = 0;
+    for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
+    // Spread the chunks evenly over the SMs: small inputs get one CTA per SM
+    // with one warp per chunk; large ones run persistent CTAs of 16 warps.
+    int warps = (int)std::min<long long>(kMaxWarps, std::max<long long>(1, (chunks + di.sms - 1) / di.sms));
+    SmemOffsets so;
     for (;;) {
-        bytes = smem_layout(warps, x_floats, max_words, &ox, &ob, &os);
-        if ((int)bytes <= di.smem_optin) break;
-        if (warps > 1) warps >>= 1;
-        else if (x_floats) { x_floats = 0; warps = kMaxWarps; }
+        so = smem_layout(warps, x_elems, stage_rows, out_words);
+        if ((long long)so.total <= di.smem_optin) break;
+        if (warps > 1) warps--;
+        else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
         else return ENTRO_E_LIMIT;
     }
+    const size_t bytes = so.total;
     LanesFn fn = pick_lanes(bits, out_kind, slow, bpad);
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, bytes, &per_sm) != ENTRO_OK)
         return ENTRO_E_CUDA;
-    long long chunks = 0;
-    for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
     long long grid = std::min<long long>((chunks + warps - 1) / warps, (long long)per_sm * di.sms);
     grid = std::max<long long>(grid, 1);
     LaunchArgs a;
@@ -905,9 +1073,10 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     a.one = one;
     a.count = count;
     a.batch = batch;
-    a.x_in_smem = x_floats > 0;
-    a.max_words = max_words;
-    a.x_floats = x_floats;
+    a.x_in_smem = x_elems > 0;
+    a.stage_rows = stage_rows;
+    a.out_words = out_words;
+    a.x_elems = x_elems;
     a.total_syms = total;
     a.status = status;
     fn<<<(unsigned)grid, warps * 32, bytes, st>>>(a);
@@ -919,8 +1088,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
     const DevTensor &d = t->d;
     if (d.n_chunks == 0) return ENTRO_OK;
     LanesFn fn = pick_single(d.bits, out_kind, t->slow);
-    size_t ox, ob, os;
-    const size_t bytes = smem_layout(0, 0, 0, &ox, &ob, &os);
+    const size_t bytes = smem_layout(0, 0, 0, 0).total;
     const int threads = 32;
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), t->device, threads, bytes, &per_sm) != ENTRO_OK)
