@@ -299,5 +299,6 @@ def version() -> int:
 
 
 __all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "EXPORTS",
+
            "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES", "GROUP_GEMV",
            "GROUP_BF16", "SCHEME_UNSIGNED", "SCHEME_ASYM"]

@@ -762,11 +762,12 @@ struct DeviceInfo {
 };
 
 static std::mutex g_mu;
-static std::vector<DeviceInfo> g_dev;
+constexpr int kMaxDevices = 64;
+static DeviceInfo g_dev[kMaxDevices];
 
 static int device_info(int dev, DeviceInfo *out) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+    if (dev < 0 || dev >= kMaxDevices) return ENTRO_E_LIMIT;
     DeviceInfo &di = g_dev[dev];
     if (di.sms == 0) {
         cudaError_t e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
@@ -985,25 +986,31 @@ struct KernelOptIn {
     int device;
     size_t bytes;
 };
-static std::vector<KernelConfig> g_kcfg;
-static std::vector<KernelOptIn> g_optin;
+// Fixed-size caches: a launch never touches the host heap.
+constexpr int kMaxConfigs = 512;
+static KernelConfig g_kcfg[kMaxConfigs];
+static int g_nkcfg = 0;
+static KernelOptIn g_optin[kMaxConfigs];
+static int g_noptin = 0;
 
 static int kernel_config(const void *fn, int device, int threads, size_t bytes, int *per_sm) {
     std::lock_guard<std::mutex> lk(g_mu);
     KernelOptIn *opt = nullptr;
-    for (KernelOptIn &o : g_optin)
-        if (o.fn == fn && o.device == device) opt = &o;
+    for (int i = 0; i < g_noptin; i++)
+        if (g_optin[i].fn == fn && g_optin[i].device == device) opt = &g_optin[i];
     if (!opt || opt->bytes < bytes) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         if (opt) opt->bytes = bytes;
-        else g_optin.push_back({fn, device, bytes});
+        else if (g_noptin < kMaxConfigs) g_optin[g_noptin++] = {fn, device, bytes};
     }
-    for (const KernelConfig &k : g_kcfg)
+    for (int i = 0; i < g_nkcfg; i++) {
+        const KernelConfig &k = g_kcfg[i];
         if (k.fn == fn && k.device == device && k.threads == threads && k.bytes == bytes) {
             *per_sm = k.per_sm;
             return ENTRO_OK;
         }
+    }
     int n = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
@@ -1011,7 +1018,7 @@ static int kernel_config(const void *fn, int device, int threads, size_t bytes, 
         snprintf(g_cuda_msg, sizeof(g_cuda_msg), "no CTA of %d threads and %zu bytes fits an SM", threads, bytes);
         return ENTRO_E_CUDA;
     }
-    g_kcfg.push_back({fn, device, threads, bytes, n});
+    if (g_nkcfg < kMaxConfigs) g_kcfg[g_nkcfg++] = {fn, device, threads, bytes, n};
     *per_sm = n;
     return ENTRO_OK;
 }
