@@ -60,7 +60,8 @@ class _Info(ctypes.Structure):
 EXPORTS = ["entro_encode", "entro_blob_from_bytes", "entro_blob_bytes", "entro_blob_info", "entro_blob_free",
            "entro_device_bytes", "entro_upload", "entro_tensor_free", "entro_decode_codes",
            "entro_decode_dequant_bf16", "entro_decode_gemv", "entro_group_table_bytes", "entro_group_prepare",
-           "entro_group_launch", "entro_group_free", "entro_strerror", "entro_version", "entro_last_cuda_error"]
+           "entro_group_launch", "entro_group_free", "entro_strerror", "entro_version", "entro_last_cuda_error",
+           "entro_decode_gemv_group_static"]
 
 
 def _load() -> ctypes.CDLL:
@@ -89,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "entro_strerror": ([I32], ctypes.c_char_p),
         "entro_version": ([], I32),
         "entro_last_cuda_error": ([], ctypes.c_char_p),
+        "entro_decode_gemv_group_static": ([P, P, P, I32, I32, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -294,11 +296,25 @@ class Group:
         self.close()
 
 
+STATIC_GROUP_MAX = 512
+
+
+def decode_gemv_group_static(tensors: Sequence[DeviceTensor], xs: Sequence[torch.Tensor],
+                             ys: Sequence[torch.Tensor], batch: int = 1, status: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Grouped fused GEMV whose work table lives inside the library (no device allocation)."""
+    count = len(tensors)
+    arr = ctypes.c_void_p * count
+    _check(_lib.entro_decode_gemv_group_static(arr(*[t._h for t in tensors]), arr(*[x.data_ptr() for x in xs]),
+                                               arr(*[y.data_ptr() for y in ys]), count, batch, _dptr(status),
+                                               _stream_ptr(stream)), "entro_decode_gemv_group_static")
+
+
 def version() -> int:
     return int(_lib.entro_version())
 
 
 __all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "EXPORTS",
-
+           "decode_gemv_group_static", "STATIC_GROUP_MAX",
            "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES", "GROUP_GEMV",
            "GROUP_BF16", "SCHEME_UNSIGNED", "SCHEME_ASYM"]

@@ -67,6 +67,8 @@ struct GroupEntry {
     long long sym_begin;     // prefix over entries, in symbols
 };
 
+static_assert(sizeof(GroupEntry) == 176, "the fixed group table is documented as 176-byte entries");
+
 struct LaunchArgs {
     const GroupEntry *table;  // device array, or nullptr: use `one`
     GroupEntry one;
@@ -1243,6 +1245,82 @@ extern "C" int entro_group_launch(const entro_group *group, int32_t *d_status, v
 }
 
 extern "C" void entro_group_free(entro_group *group) { delete reinterpret_cast<GroupHandle *>(group); }
+
+// ------------------------------------------------------------------ grouped GEMV without allocation
+//
+// Some callers may not allocate device memory at all -- for instance code that
+// runs inside a caching allocator's own hooks, or a serving runtime that
+// reserves all device memory up front and forbids cudaMalloc afterwards.  For
+// them the grouped GEMV can take its work table from a fixed array inside the
+// library instead of from caller memory.  The array costs every GPU that loads
+// the library kStaticGroupMax * sizeof(GroupEntry) bytes until process exit.
+
+namespace entro {
+constexpr int kStaticGroupMax = ENTRO_STATIC_GROUP_MAX;
+constexpr int kStaticBatchCopy = 32;  // entries staged per host-to-device copy (a stack buffer)
+static __device__ __align__(256) GroupEntry g_static_table[kStaticGroupMax];
+// Device address of g_static_table, per device; the host-side name is only a
+// stand-in, so the address comes from cudaGetSymbolAddress on first use.
+static void *g_static_addr[kMaxDevices];
+}  // namespace entro
+
+extern "C" int entro_decode_gemv_group_static(const entro_tensor *const *tensors, const void *const *xs,
+                                              float *const *ys, int32_t count, int32_t batch, int32_t *d_status,
+                                              void *stream) {
+    if (!tensors || !xs || !ys || count < 1) return ENTRO_E_INVAL;
+    if (count > kStaticGroupMax) {
+        snprintf(g_cuda_msg, sizeof(g_cuda_msg), "entro_decode_gemv_group_static: %d tensors exceed the fixed table "
+                 "of %d entries", (int)count, kStaticGroupMax);
+        return ENTRO_E_LIMIT;
+    }
+    const TensorHandle *const *ts = reinterpret_cast<const TensorHandle *const *>(tensors);
+    for (int i = 0; i < count; i++) {
+        const TensorHandle *t = ts[i];
+        if (!t || t->d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
+        const int r = gemv_check(t, xs[i], batch, ys[i]);
+        if (r != ENTRO_OK) return r;
+        if (t->device != ts[0]->device || t->d.bits != ts[0]->d.bits) return ENTRO_E_INVAL;
+    }
+    const int dev = ts[0]->device;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != dev || dev >= kMaxDevices) return ENTRO_E_INVAL;
+    void *table = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_static_addr[dev]) {
+            void *p = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&p, g_static_table);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+            g_static_addr[dev] = p;
+        }
+        table = g_static_addr[dev];
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    GroupEntry stage[kStaticBatchCopy];
+    GroupEntry first;
+    long long chunks = 0, syms = 0;
+    for (int i0 = 0; i0 < count; i0 += kStaticBatchCopy) {
+        const int m = std::min(kStaticBatchCopy, count - i0);
+        for (int k = 0; k < m; k++) {
+            const TensorHandle *t = ts[i0 + k];
+            GroupEntry &g = stage[k];
+            std::memset(&g, 0, sizeof(g));
+            g.d = t->d;
+            g.x = static_cast<const __nv_bfloat16 *>(xs[i0 + k]);
+            g.y = ys[i0 + k];
+            g.chunk_begin = chunks;
+            g.sym_begin = syms;
+            chunks += t->d.n_chunks;
+            syms += t->d.n;
+        }
+        if (i0 == 0) first = stage[0];
+        // pageable source: the call returns once `stage` has been consumed
+        const cudaError_t e = cudaMemcpyAsync(static_cast<GroupEntry *>(table) + i0, stage, sizeof(GroupEntry) * m,
+                                              cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (static group table)");
+    }
+    return launch_lanes(ts, count, OUT_GEMV, batch, static_cast<const GroupEntry *>(table), first, d_status, st);
+}
 
 extern "C" const char *entro_strerror(int code) {
     switch (code) {

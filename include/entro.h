@@ -178,6 +178,29 @@ ENTRO_API void entro_group_free(entro_group *group);
 
 ENTRO_API const char *entro_strerror(int code);
 
+/* The grouped fused GEMV (ENTRO_GROUP_GEMV) for callers that cannot allocate
+ * device memory -- code running inside an allocator's hooks, or a runtime
+ * that reserves the whole device up front and allows no cudaMalloc later.  No
+ * counterpart on the EntroLLM or LazyWeights pages: it only changes where the
+ * launch's work table lives.  The table is a fixed array inside the library
+ * (ENTRO_STATIC_GROUP_MAX entries of 176 bytes, about 88 KB, held on every
+ * GPU that loads the library until the process exits); the caller still
+ * passes the uploaded tensors, the activations xs[i] (bf16 [batch, cols_i])
+ * and the outputs ys[i] (fp32 [batch, rows_i]), with the rules of
+ * entro_decode_gemv for each.  Each call rewrites the table from host memory
+ * on `stream` and launches; nothing is allocated or freed, on the host heap
+ * or on the device.  The tensors' device must be the current device.  The
+ * first call on a device looks up the table's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one table, so calls whose launches may overlap on the
+ * GPU (other streams, other host threads) race: serialise them.  Errors:
+ * ENTRO_E_LIMIT when count > ENTRO_STATIC_GROUP_MAX, otherwise as
+ * entro_decode_gemv. */
+#define ENTRO_STATIC_GROUP_MAX 512
+ENTRO_API int entro_decode_gemv_group_static(const entro_tensor *const *tensors, const void *const *xs,
+                                             float *const *ys, int32_t count, int32_t batch, int32_t *d_status,
+                                             void *stream);
+
 /* Text of the last CUDA runtime error behind an ENTRO_E_CUDA return on the
  * calling host thread ("" if none). */
 ENTRO_API const char *entro_last_cuda_error(void);
