@@ -402,6 +402,77 @@ def _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status):
                     "three decodes, results copied to pinned host memory; wall clock per step"}
 
 
+def run_model(args, dist, rank, world, local_rank):
+    """One step = one grouped launch over every tensor of a model-shaped workload:
+    the fused GEMV of a whole decode step (tok/s) or a whole-model decode to bf16."""
+    import huffman_decode_canonical_b200 as entro
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from model_helpers import encode_workload
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    W = workloads.get(args.workload)
+    dts, infos, t_enc = encode_workload(entro, W, device=device)
+    n = sum(i["n"] for i in infos)
+    coded = sum(i["coded_bits"] for i in infos) / 8.0
+    payload = sum(i["payload_bytes"] for i in infos)
+    index = sum(i["index_bytes"] for i in infos)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    gemv = args.workload != "smollm_1p7b_u8"
+    if gemv:
+        xs = [workloads.activations(W.seed, args.batch, d.cols).to(device) for d in dts]
+        ys = [torch.empty((args.batch, d.rows), dtype=torch.float32, device=device) for d in dts]
+        g = entro.Group(dts, entro.GROUP_GEMV, xs=xs, ys=ys, batch=args.batch)
+        out_bytes = sum(2 * x.numel() for x in xs) + sum(4 * y.numel() for y in ys)
+    else:
+        outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device=device) for d in dts]
+        g = entro.Group(dts, entro.GROUP_BF16, outs=outs)
+        out_bytes = 2 * n
+    for _ in range(args.warmup):
+        g.launch(status=status)
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        g.launch(status=status)
+        torch.cuda.synchronize(device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    _barrier(dist, device)
+    torch.cuda.synchronize(device)
+    torch.cuda._sleep(int(args.steps * 100e-6 * 2.0e9))
+    for s_ in range(args.steps):
+        ev[s_].record(stream)
+        g.launch(status=status)
+    ev[args.steps].record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    ms = sum(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)) / args.steps
+    ms = _max_over_ranks(dist, ms, device)
+    if rank != 0:
+        return 0
+    peak, peak_kind = _peaks()
+    alg = coded + index + out_bytes
+    achieved = alg / (ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(world / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
+            "unit": f"tok/s (batch {args.batch})" if gemv else "Gsym/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": f"u{W.bits} codes -> bf16" + (" x bf16 -> fp32" if gemv else ""),
+            "data": "synthetic", "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
+                                            "batch": args.batch if gemv else None,
+                                            "l2": "working set larger than L2 (whole model)"},
+            "gsym_s": round(n / (ms * 1e-3) / 1e9, 1),
+            "bits_per_weight": {"coded": round(8 * coded / n, 4), "payload": round(8 * payload / n, 4)},
+            "roofline": {"bound": "hbm", "kernel": "lanes_kernel grouped launch", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None},
+            "host_encode_s": round(t_enc, 2), "gpu_launches": args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -409,6 +480,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "smollm_1p7b_u8", "mistral_7b_u4",
+                                                             "phi3_mini_u8"],
+                    help="model-scale workloads time one grouped launch per step (not the default line)")
+    ap.add_argument("--batch", type=int, default=1, help="GEMV batch for the model-scale GEMV workloads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -416,6 +491,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.workload != WORKLOAD:
+            return run_model(args, dist, rank, world, local_rank)
         return run_native(args, dist, rank, world, local_rank)
     finally:
         if dist is not None:

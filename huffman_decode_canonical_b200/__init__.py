@@ -177,7 +177,7 @@ class Blob:
         return n.value
 
     def close(self):
-        if getattr(self, "_h", None):
+        if getattr(self, "_h", None) and _lib is not None:
             _lib.entro_blob_free(self._h)
             self._h = None
 
@@ -250,7 +250,7 @@ class DeviceTensor:
         return y
 
     def close(self):
-        if getattr(self, "_h", None):
+        if getattr(self, "_h", None) and _lib is not None:
             _lib.entro_tensor_free(self._h)
             self._h = None
 
@@ -288,7 +288,7 @@ class Group:
         _check(_lib.entro_group_launch(self._h, _dptr(status), _stream_ptr(stream)), "entro_group_launch")
 
     def close(self):
-        if getattr(self, "_h", None):
+        if getattr(self, "_h", None) and _lib is not None:
             _lib.entro_group_free(self._h)
             self._h = None
 

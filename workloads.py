@@ -15,7 +15,8 @@ available here, so these seeded tensors stand in for them.  Value laws:
 * ``laplace(b)``: Laplace(0, b); "Laplace with std s" means b = s / sqrt(2).
 * ``shifted``: ``w - min(w)`` (a non-negative tensor).
 * ``uniform``: U(-1, 1).
-* ``skew``: 0 with probability 0.9, else 0.02 * t(4).
+* ``skew``: 0 with probability 0.9, else +-0.02 * (1 + |t(4)|): the non-zero
+  draws stay clear of the zero code, so the most frequent code has p = 0.9.
 
 Small single tensors (the 1024x1024 and 4096x4096 cases) come from NumPy's
 ``default_rng([config_seed, tensor_index])``; model-sized tensors come from
@@ -174,7 +175,8 @@ def _draw_torch(spec: TensorSpec, seed: int, device) -> torch.Tensor:
             w = (spec.param / math.sqrt(2.0)) * t
         else:
             keep = torch.rand(shape, generator=g, device=device) >= 0.9
-            w = torch.where(keep, spec.param * t, torch.zeros_like(t))
+            mag = spec.param * (1.0 + t.abs())
+            w = torch.where(keep, torch.sign(t) * mag, torch.zeros_like(t))
     elif spec.law == "laplace":
         u = torch.rand(shape, generator=g, device=device, dtype=torch.float32).clamp_min(1e-7) - 0.5
         w = -spec.param * torch.sign(u) * torch.log1p(-2.0 * u.abs())
