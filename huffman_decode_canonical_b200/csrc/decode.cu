@@ -291,69 +291,103 @@ __device__ __forceinline__ float warp_sum(float v) {
 // written to the warp's code stage at word 32*t + lane (4-bit) or double-word
 // 32*t + lane (8-bit), i.e. in output order, without bank conflicts.
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(lo), "r"(hi) : "memory");
+}
+
 template <int BITS, bool SLOW>
 struct LaneDecoder {
-    const uint32_t *buf;  // word j of this lane at buf[32 * j]
-    uint32_t *ost;        // this lane's first staged run; run t at ost[32 * t] (words or double-words)
-    uint32_t *sink;       // a private scratch slot that absorbs not-ready stores
-    int jcap, j, nb;
+    static constexpr int kRunBits = 8 * BITS;
+    static constexpr uint32_t kRunStride = kLanes * BITS;  // bytes between a lane's runs in the stage
+    uint32_t lut;         // shared address of the decode table
+    uint32_t bufa;        // shared address of this lane's word 0; word j at bufa + 128 j
+    uint32_t bufcap;      // shared address of the last readable word of this lane
+    uint32_t osta;        // shared address of this lane's current run slot
+    int nb;
+    uint32_t wnext;       // the next word, loaded one refill ahead (off the window's dependency chain)
     uint64_t win;
-    uint64_t pend;        // pending symbols, first at bit 0
-    uint32_t pend_hi;     // 8-bit: symbols 8.. of the pending set
-    int pc;               // pending count
-    int t;                // runs stored
+    uint32_t p0, p1, p2;  // pending codes as one bit string, first code at bit 0 of p0
+    int pb;               // pending bits (BITS per code); below one run whenever codes are appended
+    int t;                // runs completed
+
+    __device__ __forceinline__ void init(const Smem &s, const uint32_t *b, uint32_t *o, int cap) {
+        lut = smem_addr(s.lut);
+        bufa = smem_addr(b);
+        bufcap = bufa + 4u * kLanes * static_cast<uint32_t>(cap);
+        osta = smem_addr(o);
+        win = (static_cast<uint64_t>(lds32(bufa)) << 32) | lds32(bufa + 4 * kLanes);
+        nb = 64;
+        bufa += 8 * kLanes;
+        wnext = lds32(min(bufa, bufcap));
+        p0 = p1 = p2 = 0;
+        pb = 0;
+        t = 0;
+    }
 
     __device__ __forceinline__ void refill() {
-        const uint32_t w = buf[kLanes * min(j, jcap)];
         if (nb <= 32) {
-            win |= static_cast<uint64_t>(w) << (32 - nb);
+            win |= static_cast<uint64_t>(wnext) << (32 - nb);
             nb += 32;
-            j++;
+            bufa += 4 * kLanes;
+            wnext = lds32(min(bufa, bufcap));
         }
     }
 
-    // one table lookup; appends its symbols to the pending set
+    // one table lookup; appends its codes to the pending bit string
     __device__ __forceinline__ void lookup(const Smem &s, int max_len, int32_t *status) {
-        const uint32_t e = s.lut[static_cast<uint32_t>(win >> (64 - kMaxLutBits))];
-        uint32_t cnt = (e >> 4) & 15u, syms = e >> 8, bits = e & 15u;
-        if (SLOW && cnt == 0) {
+        const uint32_t e = lds32(lut + (static_cast<uint32_t>(win >> (64 - kMaxLutBits)) << 2));
+        uint32_t syms = e >> 8, bits = e & 15u;
+        // count * BITS straight from the entry's count field (bits 4..7)
+        int add = static_cast<int>(BITS == 4 ? (e >> 2) & 0x3Cu : (e >> 1) & 0x78u);
+        if (SLOW && add == 0) {
             const uint32_t se = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, status);
             bits = se & 31u;
             syms = (se >> 8) & 0xFFu;
-            cnt = 1;
+            add = BITS;
         }
         win <<= bits;
         nb -= static_cast<int>(bits);
-        if (BITS == 4) {
-            pend |= static_cast<uint64_t>(syms) << (4 * pc);
+        const int q = pb & 31;
+        const uint32_t lo = syms << q, hi = __funnelshift_l(syms, 0u, q);  // (0:syms) << q, 24-bit codes
+        if (BITS == 4 || pb < 32) {
+            p0 |= lo;
+            p1 |= hi;
         } else {
-            const int sh = 8 * pc;  // < 64: appends happen only while fewer than 8 are pending
-            pend |= static_cast<uint64_t>(syms) << sh;
-            if (sh > 40) pend_hi |= syms >> (64 - sh);
+            p1 |= lo;
+            p2 |= hi;
         }
-        pc += static_cast<int>(cnt);
+        pb += add;
     }
 
-    // After a lookup at most one run is complete (pending < 16).  The store is
-    // issued either way -- to the run's slot when ready, else to the sink --
-    // so the warp stays converged.
-    __device__ __forceinline__ void emit(int full_runs) {
-        const bool ready = pc >= 8 && t < full_runs;
-        if (BITS == 4) {
-            uint32_t *dst = ready ? ost + kLanes * t : sink;
-            *dst = static_cast<uint32_t>(pend);
-            if (ready) pend >>= 32;
-        } else {
-            uint64_t *dst = ready ? reinterpret_cast<uint64_t *>(ost) + kLanes * t : reinterpret_cast<uint64_t *>(sink);
-            *dst = pend;
-            if (ready) {
-                pend = pend_hi;
-                pend_hi = 0;
+    // Store the current run's pending codes to its slot -- harmless while the
+    // run is incomplete, since the slot is rewritten until it is -- and move on
+    // once the run is whole.  At most one run completes per lookup.
+    __device__ __forceinline__ void emit() {
+        if (BITS == 4) sts32(osta, p0);
+        else sts64(osta, p0, p1);
+        if (pb >= kRunBits) {
+            if (BITS == 4) {
+                p0 = p1;
+                p1 = 0;
+            } else {
+                p0 = p2;
+                p1 = 0;
+                p2 = 0;
             }
+            pb -= kRunBits;
+            t++;
+            osta += kRunStride;
         }
-        pc -= ready ? 8 : 0;
-        t += ready ? 1 : 0;
     }
+
 };
 
 // ------------------------------------------------------------------ phase 2: stage -> output
@@ -488,21 +522,10 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
     const int nc = static_cast<int>(remain < d.chunk_symbols ? remain : d.chunk_symbols);
     const bool refill_each = SLOW && d.max_len > 16;
     uint32_t *lost = ost + (BITS == 4 ? lane : 2 * lane);
-    uint32_t *sink = ost + (static_cast<size_t>(d.chunk_symbols) * BITS / 32) + (BITS == 4 ? lane : 2 * lane);
     LaneDecoder<BITS, SLOW> ld;
-    ld.buf = buf + lane;
-    ld.ost = lost;
-    ld.sink = sink;
-    ld.jcap = stage_rows - 1;
-    ld.j = 0;
-    ld.nb = 0;
-    ld.win = 0;
-    ld.pend = 0;
-    ld.pend_hi = 0;
-    ld.pc = 0;
-    ld.t = 0;
-    ld.refill();
-    ld.refill();
+    ld.init(s, buf + lane, lost, stage_rows - 1);
+    // a valid lane never loads past its words plus the two read-ahead rows
+    const uint32_t read_limit = smem_addr(buf + lane) + 4u * kLanes * static_cast<uint32_t>(words + kSlackRows);
     bool ok = true;
     if (nc == d.chunk_symbols) {
         const int runs = nc / kStepSymbols;
@@ -514,15 +537,15 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
             while (ld.t < te) {
                 ld.refill();
                 ld.lookup(s, d.max_len, status);
-                ld.emit(runs);
+                ld.emit();
                 if (SLOW && refill_each) ld.refill();
                 ld.lookup(s, d.max_len, status);
-                ld.emit(runs);
+                ld.emit();
             }
             __syncwarp();
             emit_runs<BITS, OUT, BPAD>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
         }
-        ok = ld.j <= words + kSlackRows;
+        ok = ld.bufa <= read_limit;
     } else {
         // symbols of this lane: positions 256*t + 8*lane + i < nc
         const int full_steps = nc / kStepSymbols, rem = nc % kStepSymbols;
@@ -532,20 +555,19 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
             while (ld.t < full_runs) {
                 ld.refill();
                 ld.lookup(s, d.max_len, status);
-                ld.emit(full_runs);
+                ld.emit();
                 if (SLOW && refill_each) ld.refill();
                 ld.lookup(s, d.max_len, status);
-                ld.emit(full_runs);
+                ld.emit();
             }
             if (tail) {
-                while (ld.pc < tail) {
+                while (ld.pb < tail * BITS) {
                     ld.refill();
                     ld.lookup(s, d.max_len, status);
                 }
-                if (BITS == 4) lost[kLanes * ld.t] = static_cast<uint32_t>(ld.pend);
-                else reinterpret_cast<uint64_t *>(lost)[kLanes * ld.t] = ld.pend;
+                ld.emit();
             }
-            ok = ld.j <= words + kSlackRows;
+            ok = ld.bufa <= read_limit;
         }
         __syncwarp();
         emit_ragged<BITS, OUT>(g, s, ost, first, nc);
@@ -1055,7 +1077,8 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
     long long x_elems = (out_kind == OUT_GEMV && max_kb <= kXSmemElems) ? max_kb : 0;
     const int stage_rows = max_words + kSlackRows;
-    const int out_words = static_cast<int>(max_chunk * bits / 32) + 2 * kLanes;  // + the not-ready sink
+    // + slack for runs that lanes begin past the chunk's last (up to 2 runs of 2 words for 8-bit)
+    const int out_words = static_cast<int>(max_chunk * bits / 32) + 4 * kLanes;
     long long chunks = 0;
     for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
     // Spread the chunks evenly over the SMs: small inputs get one CTA per SM
