@@ -705,9 +705,72 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 }
 
 // ------------------------------------------------------------------ single-stream format
+//
+// One warp per chunk of the one-bitstream format (EntroLLM technical summary:
+// the coded chunks decode in parallel).  The chunk's bits [B0, B1) are cut
+// into 32 equal segments.  Lane i decodes from the start of segment i until it
+// crosses into segment i+1 and notes where it stopped and how many codes it
+// read.  Lane 0 starts on a code boundary; a lane whose start differs from
+// where its left neighbour stopped decodes again from there, until no start
+// changes (at most 32 rounds; Huffman codes resynchronise within a few codes,
+// so two rounds are typical).  An exclusive warp-shuffle scan of the counts
+// then gives every lane its first output position, and a last pass writes the
+// codes or their bf16 values.
+
+struct BitReader {
+    const uint32_t *words;
+    long long limit;  // readable words (payload + pad)
+    long long k;      // next word to load
+    uint64_t win;
+    int nb;
+
+    __device__ __forceinline__ uint32_t word(long long i) const { return i < limit ? __ldg(words + i) : 0u; }
+    __device__ __forceinline__ void seek(uint64_t pos) {
+        k = static_cast<long long>(pos >> 5);
+        const int sh = static_cast<int>(pos & 31);
+        win = ((static_cast<uint64_t>(word(k)) << 32) | word(k + 1)) << sh;
+        nb = 64 - sh;
+        k += 2;
+    }
+    __device__ __forceinline__ void refill() {
+        if (nb <= 32) {
+            win |= static_cast<uint64_t>(word(k)) << (32 - nb);
+            nb += 32;
+            k++;
+        }
+    }
+    // one code; returns its table entry (length | symbol << 8)
+    template <bool SLOW>
+    __device__ __forceinline__ uint32_t next(const Smem &s, int max_len, int32_t *status) {
+        refill();
+        uint32_t e = s.lut[static_cast<uint32_t>(win >> (64 - kMaxLutBits))];
+        if (SLOW && (e & 31u) == 0) e = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, status);
+        const uint32_t len = e & 31u;
+        win <<= len;
+        nb -= static_cast<int>(len);
+        return e;
+    }
+};
+
+// Decode from bit `pos` (a code boundary) until crossing `stop`; returns the
+// stop position and the number of codes read.
+template <bool SLOW>
+__device__ __forceinline__ uint64_t scan_segment(BitReader &br, const Smem &s, int max_len, uint64_t pos,
+                                                 uint64_t stop, int max_codes, int *count, int32_t *status) {
+    int n = 0;
+    if (pos < stop) {
+        br.seek(pos);
+        while (pos < stop && n < max_codes) {
+            pos += br.next<SLOW>(s, max_len, status) & 31u;
+            n++;
+        }
+    }
+    *count = n;
+    return pos;
+}
 
 template <int BITS, int OUT, bool SLOW>
-__global__ void __launch_bounds__(128) single_kernel(const __grid_constant__ LaunchArgs a) {
+__global__ void __launch_bounds__(256) single_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const Smem s = carve(smem_raw, 0, 0, 0, 0);
     const GroupEntry &g = a.one;
@@ -720,54 +783,77 @@ __global__ void __launch_bounds__(128) single_kernel(const __grid_constant__ Lau
         set_status(a.status, ENTRO_E_TIMEOUT);
         return;
     }
-    const long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const long long c = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (c >= d.n_chunks) return;
-    const uint64_t bit0 = d.index[2 * c], bit1 = d.index[2 * c + 2];
+    const uint64_t B0 = d.index[2 * c], B1 = d.index[2 * c + 2];
     const long long first = static_cast<long long>(d.index[2 * c + 1]);
-    const long long last = static_cast<long long>(d.index[2 * c + 3]);
-    if (bit1 < bit0 || (bit1 + 31) / 32 > static_cast<uint64_t>(d.payload_words) || last < first) {
-        set_status(a.status, ENTRO_E_CORRUPT);
+    const long long nc = static_cast<long long>(d.index[2 * c + 3]) - first;
+    if (B1 < B0 || (B1 + 31) / 32 > static_cast<uint64_t>(d.payload_words) || nc < 0 || nc > d.chunk_symbols) {
+        if (lane == 0) set_status(a.status, ENTRO_E_CORRUPT);
         return;
     }
-    const long long limit_words = d.payload_words + kPadWords;
-    long long wi = static_cast<long long>(bit0 >> 5);
-    const int sh = static_cast<int>(bit0 & 31);
-    uint64_t win = (static_cast<uint64_t>(d.payload[wi]) << 32) | d.payload[wi + 1];
-    win <<= sh;
-    int nb = 64 - sh;
-    wi += 2;
+    BitReader br{d.payload, d.payload_words + kPadWords, 0, 0, 0};
+    const uint64_t L = B1 - B0;
+    const uint64_t seg0 = B0 + L * lane / 32, seg1 = (lane == 31) ? B1 : B0 + L * (lane + 1) / 32;
+    // every code takes at least one bit: a segment never holds more codes than bits
+    const int cap = static_cast<int>(min(static_cast<long long>(seg1 - seg0) + 64, nc + 1));
+    uint64_t start = seg0;
+    int n = 0;
+    uint64_t end = scan_segment<SLOW>(br, s, d.max_len, start, seg1, cap, &n, a.status);
+    for (int round = 0; round < 32; round++) {
+        uint64_t prev = __shfl_up_sync(0xffffffffu, end, 1);
+        if (lane == 0) prev = B0;
+        const bool redo = prev != start;
+        if (!__any_sync(0xffffffffu, redo)) break;
+        if (redo) {
+            start = prev;
+            end = scan_segment<SLOW>(br, s, d.max_len, start, seg1, cap, &n, a.status);
+        }
+    }
+    // output position of this lane's first code: exclusive scan of the counts
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint64_t last_end = __shfl_sync(0xffffffffu, end, 31);
+    if (total != nc || last_end != B1) {
+        if (lane == 0) set_status(a.status, ENTRO_E_CORRUPT);
+        return;
+    }
+    long long p = first + (incl - n);
+    if (n > 0) br.seek(start);
     uint8_t *o8 = reinterpret_cast<uint8_t *>(g.out);
     uint16_t *o16 = reinterpret_cast<uint16_t *>(g.out);
+    // 4-bit codes: chunks start on even symbols (checked on the host), so only
+    // a lane's first and last codes can share a byte with a neighbour lane;
+    // those nibbles go through a word-wide atomic, the rest as whole bytes.
     uint32_t pending = 0;
-    for (long long p = first; p < last; p++) {
-        if (nb <= 32) {
-            const uint32_t w = wi < limit_words ? d.payload[wi] : 0u;
-            win |= static_cast<uint64_t>(w) << (32 - nb);
-            nb += 32;
-            wi++;
-        }
-        uint32_t e = s.lut[static_cast<uint32_t>(win >> (64 - kMaxLutBits))];
-        if (SLOW && (e & 31u) == 0) e = slow_entry(win, d.max_len, s.slim, s.soffs, s.ssyms, a.status);
-        const uint32_t len = e & 31u;
-        const uint32_t sym = (e >> 8) & 0xFFu;
-        win <<= len;
-        nb -= static_cast<int>(len);
+    for (int i = 0; i < n; i++, p++) {
+        const uint32_t sym = (br.next<SLOW>(s, d.max_len, a.status) >> 8) & 0xFFu;
         if (OUT == OUT_BF16) {
             o16[p] = static_cast<uint16_t>(s.vtab[sym]);
         } else if (BITS == 8) {
             o8[p] = static_cast<uint8_t>(sym);
-        } else {  // chunks start on even symbols (checked on the host): bytes are private
-            if ((p & 1) == 0) {
+        } else {
+            const bool lo_half = (p & 1) == 0;
+            const bool shared_byte = (lo_half && i == n - 1 && p + 1 < first + nc) || (!lo_half && i == 0);
+            if (shared_byte) {
+                uint32_t *word = reinterpret_cast<uint32_t *>(o8 + ((p >> 1) & ~3LL));
+                const int shift = static_cast<int>(((p >> 1) & 3) * 8 + (lo_half ? 0 : 4));
+                atomicAnd(word, ~(0xFu << shift));
+                atomicOr(word, sym << shift);
+            } else if (lo_half) {
                 pending = sym;
-                if (p + 1 == last) o8[p >> 1] = static_cast<uint8_t>(pending);
+                if (p + 1 == first + nc) o8[p >> 1] = static_cast<uint8_t>(pending);
             } else {
                 o8[p >> 1] = static_cast<uint8_t>(pending | (sym << 4));
             }
         }
     }
-    const uint64_t consumed = 32ull * static_cast<uint64_t>(wi - static_cast<long long>(bit0 >> 5)) -
-                              static_cast<uint64_t>(nb) - static_cast<uint64_t>(sh);
-    if (consumed != bit1 - bit0) set_status(a.status, ENTRO_E_CORRUPT);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1121,7 +1207,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
     if (d.n_chunks == 0) return ENTRO_OK;
     LanesFn fn = pick_single(d.bits, out_kind, t->slow);
     const size_t bytes = smem_layout(0, 0, 0, 0).total;
-    const int threads = 32;
+    const int threads = 64;  // two chunks per CTA: spreads small tensors over the SMs
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), t->device, threads, bytes, &per_sm) != ENTRO_OK)
         return ENTRO_E_CUDA;
@@ -1132,7 +1218,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
     a.count = 1;
     a.batch = 1;
     a.status = status;
-    const long long grid = (d.n_chunks + threads - 1) / threads;
+    const long long grid = (d.n_chunks * 32 + threads - 1) / threads;
     fn<<<(unsigned)grid, threads, bytes, st>>>(a);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "single kernel launch");
