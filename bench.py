@@ -5,11 +5,12 @@ tensor (32 word-interleaved lanes per 8192-symbol chunk):
     decode -> packed uint4 codes, decode -> dequantize -> bf16, and the fused
     decode -> dequantize -> GEMV (batch 1),
 each through the C ABI of libentro.  Inputs are resident in HBM.  The working
-set is made larger than L2: 8 replicas of the encoded tensor and of its outputs
-(~350 MB against a 126 MB L2) rotate so that every kernel reads a replica that
-no recent kernel touched and writes outputs whose lines must first be evicted
--- the steady state of decoding a model much larger than L2 (no flush kernel,
-so the decode code and tables stay warm as they would in serving).  Kernel
+set is made larger than L2: 40 replicas of the encoded tensor (160 MB of coded
+payload alone, against a 126 MB L2) and of its outputs rotate, each kernel on
+the next replica, so every kernel reads coded words that no recent kernel
+touched and writes outputs whose lines must first be evicted -- the steady
+state of decoding a model much larger than L2 (no flush kernel, so the decode
+code stays warm as it would in serving).  Kernel
 times come from CUDA events on the launching stream.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
@@ -40,7 +41,7 @@ import workloads  # noqa: E402
 
 METRIC = "decoded Gsym/s and % HBM roofline (Huffman decode+dequant); fused GEMV tok/s"
 WORKLOAD = "laplace_4096x4096_u4"
-REPLICAS = 8
+REPLICAS = 40
 
 
 def _peaks():

@@ -303,6 +303,13 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(lo), "r"(hi) : "memory");
 }
 
+// Runs are staged in a ring of kRing slots per lane: a warp emits every
+// kEmitBlock runs, and a lane can only start up to two runs beyond the block
+// it is decoding, so kRing >= kEmitBlock + 2 keeps the slots being emitted
+// apart from the slots being written.
+constexpr int kEmitBlock = 8;
+constexpr int kRing = 16;
+
 template <int BITS, bool SLOW>
 struct LaneDecoder {
     static constexpr int kRunBits = 8 * BITS;
@@ -310,6 +317,7 @@ struct LaneDecoder {
     uint32_t lut;         // shared address of the decode table
     uint32_t bufa;        // shared address of this lane's word 0; word j at bufa + 128 j
     uint32_t bufcap;      // shared address of the last readable word of this lane
+    uint32_t ostb;        // shared address of this lane's slot 0 of the run ring
     uint32_t osta;        // shared address of this lane's current run slot
     int nb;
     uint32_t wnext;       // the next word, loaded one refill ahead (off the window's dependency chain)
@@ -322,7 +330,7 @@ struct LaneDecoder {
         lut = smem_addr(s.lut);
         bufa = smem_addr(b);
         bufcap = bufa + 4u * kLanes * static_cast<uint32_t>(cap);
-        osta = smem_addr(o);
+        ostb = osta = smem_addr(o);
         win = (static_cast<uint64_t>(lds32(bufa)) << 32) | lds32(bufa + 4 * kLanes);
         nb = 64;
         bufa += 8 * kLanes;
@@ -384,8 +392,16 @@ struct LaneDecoder {
             }
             pb -= kRunBits;
             t++;
-            osta += kRunStride;
+            osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
         }
+    }
+
+    // store the current (possibly partial) run and count it done
+    __device__ __forceinline__ void close_run() {
+        if (BITS == 4) sts32(osta, p0);
+        else sts64(osta, p0, p1);
+        t++;
+        osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
     }
 
 };
@@ -419,14 +435,15 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
     if (OUT == OUT_CODES) {
-        // staged codes are packed and in output order: 16-byte copies
+        // staged codes are packed and in output order (the block's slots do not wrap): 16-byte copies
         constexpr int kU4PerRun = kLanes * BITS / 16;  // uint4 per run of the warp (8 or 16)
-        const uint4 *src = reinterpret_cast<const uint4 *>(ost) + tb * kU4PerRun;
+        const uint4 *src = reinterpret_cast<const uint4 *>(ost) + (tb & (kRing - 1)) * kU4PerRun;
         uint4 *dst = reinterpret_cast<uint4 *>(g.out) + first * BITS / 128 + tb * kU4PerRun;
         for (int i = lane; i < (te - tb) * kU4PerRun; i += kLanes) dst[i] = src[i];
     } else if (OUT == OUT_BF16) {
         uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(g.out) + first);
-        for (int t = tb; t < te; t++) dst[kLanes * t + lane] = values8<BITS>(s, ost, kLanes * t + lane);
+        for (int t = tb; t < te; t++)
+            dst[kLanes * t + lane] = values8<BITS>(s, ost, kLanes * (t & (kRing - 1)) + lane);
     } else {
         // fused GEMV: run t covers columns 256*(t % spr) + 8*lane .. +7 of row t / spr
         const int K = static_cast<int>(d.cols);
@@ -436,7 +453,7 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
         for (int t = tb; t < te; t++) {
             const int st = t % spr;
-            const uint4 wv = values8<BITS>(s, ost, kLanes * t + lane);
+            const uint4 wv = values8<BITS>(s, ost, kLanes * (t & (kRing - 1)) + lane);
             const int xo = st * kLanes + lane;  // uint4 index within one x row
 #pragma unroll
             for (int b = 0; b < BPAD; b++) {
@@ -464,33 +481,32 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
     }
 }
 
-// Emit a ragged (last) chunk of nc codes after the whole chunk was staged.
+// Emit runs [tb, te) of a ragged (last) chunk of nc codes: only positions < nc.
 template <int BITS, int OUT>
 __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
-                                            int nc) {
+                                            int nc, int tb, int te) {
     const int lane = threadIdx.x & 31;
-    const int words = (nc + 7) >> 3;
-    if (OUT == OUT_CODES) {
-        uint8_t *o = reinterpret_cast<uint8_t *>(g.out) + first * BITS / 8;
-        for (int w = lane; w < words; w += kLanes) {
-            const int cnt = min(8, nc - 8 * w);
+    for (int t = tb; t < te; t++) {
+        const int w = kLanes * t + lane;        // output word: positions 8w .. 8w+7
+        const int cnt = min(8, nc - 8 * w);
+        if (cnt <= 0) continue;
+        const int slot = kLanes * (t & (kRing - 1)) + lane;
+        if (OUT == OUT_CODES) {
+            uint8_t *o = reinterpret_cast<uint8_t *>(g.out) + first * BITS / 8;
             if (BITS == 4) {
-                const uint32_t c = ost[w];
+                const uint32_t c = ost[slot];
                 for (int k = 0; 2 * k < cnt; k++) {
                     uint32_t b = (c >> (8 * k)) & 0xFFu;
                     if (2 * k + 1 >= cnt) b &= 0xFu;
                     o[4 * w + k] = static_cast<uint8_t>(b);
                 }
             } else {
-                const uint8_t *c = reinterpret_cast<const uint8_t *>(ost) + 8 * w;
+                const uint8_t *c = reinterpret_cast<const uint8_t *>(ost) + 8 * slot;
                 for (int k = 0; k < cnt; k++) o[8 * w + k] = c[k];
             }
-        }
-    } else if (OUT == OUT_BF16) {
-        for (int w = lane; w < words; w += kLanes) {
-            const uint4 v = values8<BITS>(s, ost, w);
+        } else if (OUT == OUT_BF16) {
+            const uint4 v = values8<BITS>(s, ost, slot);
             uint16_t *o = reinterpret_cast<uint16_t *>(g.out) + first + 8 * w;
-            const int cnt = min(8, nc - 8 * w);
             if (cnt == 8) {
                 *reinterpret_cast<uint4 *>(o) = v;
             } else {
@@ -502,8 +518,6 @@ __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, 
         }
     }
 }
-
-constexpr int kEmitBlock = 8;  // runs decoded between two emission rounds
 
 // Decode chunk c of entry g from its staged words.  Whole chunks are emitted
 // every kEmitBlock runs, so the stores of one block drain while the lanes
@@ -544,6 +558,7 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
             }
             __syncwarp();
             emit_runs<BITS, OUT, BPAD>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
+            __syncwarp();  // the ring slots just read are rewritten by the next block
         }
         ok = ld.bufa <= read_limit;
     } else {
@@ -551,8 +566,11 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
         const int full_steps = nc / kStepSymbols, rem = nc % kStepSymbols;
         const int S = 8 * full_steps + max(0, min(8, rem - 8 * lane));
         const int full_runs = S >> 3, tail = S & 7;
-        if (S > 0) {
-            while (ld.t < full_runs) {
+        const int steps = (nc + kStepSymbols - 1) / kStepSymbols;
+        for (int tb = 0; tb < steps; tb += kEmitBlock) {
+            const int te = min(tb + kEmitBlock, steps);
+            const int tf = min(te, full_runs);
+            while (ld.t < tf) {
                 ld.refill();
                 ld.lookup(s, d.max_len, status);
                 ld.emit();
@@ -560,17 +578,18 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
                 ld.lookup(s, d.max_len, status);
                 ld.emit();
             }
-            if (tail) {
+            if (tail && ld.t == full_runs && full_runs < te) {
                 while (ld.pb < tail * BITS) {
                     ld.refill();
                     ld.lookup(s, d.max_len, status);
                 }
-                ld.emit();
+                ld.close_run();
             }
-            ok = ld.bufa <= read_limit;
+            __syncwarp();
+            emit_ragged<BITS, OUT>(g, s, ost, first, nc, tb, te);
+            __syncwarp();
         }
-        __syncwarp();
-        emit_ragged<BITS, OUT>(g, s, ost, first, nc);
+        if (S > 0) ok = ld.bufa <= read_limit;
     }
     if (!ok) set_status(status, ENTRO_E_OVERRUN);
     __syncwarp();
@@ -1163,8 +1182,7 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
     long long x_elems = (out_kind == OUT_GEMV && max_kb <= kXSmemElems) ? max_kb : 0;
     const int stage_rows = max_words + kSlackRows;
-    // + slack for runs that lanes begin past the chunk's last (up to 2 runs of 2 words for 8-bit)
-    const int out_words = static_cast<int>(max_chunk * bits / 32) + 4 * kLanes;
+    const int out_words = kRing * kLanes * bits / 4;  // the run ring: kRing runs of 8 codes per lane
     long long chunks = 0;
     for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
     // Spread the chunks evenly over the SMs: small inputs get one CTA per SM
