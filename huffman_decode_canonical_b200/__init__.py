@@ -44,7 +44,7 @@ class EntroError(RuntimeError):
 class _Opts(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("quant_mode", ctypes.c_int32), ("max_len", ctypes.c_int32),
                 ("format", ctypes.c_int32), ("chunk_symbols", ctypes.c_int64), ("threads", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("lanes", ctypes.c_int32)]
 
 
 class _Info(ctypes.Structure):
@@ -53,7 +53,7 @@ class _Info(ctypes.Structure):
                 ("n", ctypes.c_int64), ("chunk_symbols", ctypes.c_int64), ("n_chunks", ctypes.c_int64),
                 ("scale", ctypes.c_float), ("zero", ctypes.c_int32), ("payload_bytes", ctypes.c_uint64),
                 ("index_bytes", ctypes.c_uint64), ("blob_bytes", ctypes.c_uint64), ("coded_bits", ctypes.c_uint64),
-                ("max_chunk_words", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+                ("max_chunk_words", ctypes.c_uint32), ("lanes", ctypes.c_uint32),
                 ("lengths", ctypes.c_uint8 * 256)]
 
 
@@ -138,13 +138,13 @@ class Blob:
 
     @classmethod
     def encode(cls, w, bits: int = 8, quant_mode: int = QUANT_AUTO, max_len: int = 0,
-               fmt: int = FORMAT_LANES, chunk_symbols: int = 0, threads: int = 0) -> "Blob":
+               fmt: int = FORMAT_LANES, chunk_symbols: int = 0, threads: int = 0, lanes: int = 0) -> "Blob":
         if isinstance(w, torch.Tensor):
             w = w.detach().to("cpu", torch.float32).numpy()
         w = np.ascontiguousarray(w, dtype=np.float32)
         if w.ndim != 2:
             raise ValueError("w must be 2-D [rows, cols]")
-        opts = _Opts(bits, quant_mode, max_len, fmt, chunk_symbols, threads, 0)
+        opts = _Opts(bits, quant_mode, max_len, fmt, chunk_symbols, threads, lanes)
         h = ctypes.c_void_p()
         _check(_lib.entro_encode(w.ctypes.data_as(ctypes.c_void_p) if w.size else None, w.shape[0], w.shape[1],
                                  ctypes.byref(opts), ctypes.byref(h)), "entro_encode")
@@ -167,7 +167,7 @@ class Blob:
     def info(self) -> dict:
         i = _Info()
         _check(_lib.entro_blob_info(self._h, ctypes.byref(i)), "entro_blob_info")
-        d = {f: getattr(i, f) for f, _ in _Info._fields_ if f not in ("lengths", "reserved")}
+        d = {f: getattr(i, f) for f, _ in _Info._fields_ if f != "lengths"}
         d["lengths"] = np.frombuffer(bytes(i.lengths), np.uint8).copy()
         return d
 

@@ -8,11 +8,11 @@
 //               of the chunk (lanes); the last entry holds the totals
 //   payload     payload_words x u32, codes MSB-first within each word
 //
-// Lanes format: a chunk of n_c symbols is split over 32 lanes; lane l codes
-// the runs of 8 consecutive symbols at chunk positions 256*t + 8*l + (0..7),
-// t = 0, 1, ...  Every lane of a chunk is padded with zero bits to the
+// Lanes format: a chunk of n_c symbols is split over L = 32 or 64 lanes; lane
+// l codes the runs of 8 consecutive symbols at chunk positions 8*L*t + 8*l +
+// (0..7), t = 0, 1, ...  Every lane of a chunk is padded with zero bits to the
 // chunk's longest lane (W_c words), and word j of lane l sits at
-// payload[chunk_start + 32*j + l], so one 128-byte row holds word j of all
+// payload[chunk_start + L*j + l], so one row of 4L bytes holds word j of all
 // lanes (the interleaved lanes of the LazyWeights abstract; the run of 8
 // makes each lane's output 8 adjacent weights).
 #pragma once
@@ -24,9 +24,10 @@ constexpr uint32_t kMagic = 0x52544E45u;  // "ENTR"
 constexpr uint32_t kVersion = 1;
 constexpr int kHeaderBytes = 128;
 constexpr int kLengthsBytes = 256;
-constexpr int kLanes = 32;
+constexpr int kLanes = 32;                   // lanes of a warp, and the default lane count
+constexpr int kMaxLanes = 64;
 constexpr int kRun = 8;
-constexpr int kStepSymbols = kLanes * kRun;  // 256 symbols per lane step
+constexpr int kStepSymbols = kLanes * kRun;  // 256 symbols per lane step with 32 lanes
 constexpr int kMaxLutBits = 12;
 constexpr int kMaxLenLimit = 24;
 constexpr int64_t kMaxLanesChunk = 16384;

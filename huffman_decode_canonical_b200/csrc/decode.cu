@@ -55,7 +55,7 @@ struct DevTensor {
     const uint32_t *payload;
     long long n, rows, cols, chunk_symbols, n_chunks, payload_words;
     float scale;
-    int zero, bits, max_len, format, max_chunk_words, n_codes;
+    int zero, bits, max_len, format, max_chunk_words, n_codes, lanes;
 };
 
 struct GroupEntry {
@@ -197,7 +197,8 @@ struct SmemOffsets {
 };
 
 // shared-memory carve-up; identical on host (sizing) and device
-__host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_rows, int out_words) {
+// stage_words: 32-bit words of one staging buffer (rows x lanes)
+__host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_words, int out_words) {
     SmemOffsets o;
     size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
     p = align_up(p, 16);
@@ -208,7 +209,7 @@ __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems,
     p += (size_t)(warps + 1) * 2 * 8;
     p = align_up(p, 128);
     o.stage = p;
-    p += (size_t)warps * 2 * (size_t)stage_rows * kLanes * 4;
+    p += (size_t)warps * 2 * (size_t)stage_words * 4;
     p = align_up(p, 16);
     o.ostage = p;
     p += (size_t)warps * (size_t)out_words * 4;
@@ -216,8 +217,8 @@ __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems,
     return o;
 }
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_rows, int out_words) {
-    const SmemOffsets o = smem_layout(warps, x_elems, stage_rows, out_words);
+__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_words, int out_words) {
+    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words);
     Smem s;
     s.lut = reinterpret_cast<uint32_t *>(base);
     s.vtab = s.lut + kLutSize;
@@ -310,12 +311,13 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
 constexpr int kEmitBlock = 8;
 constexpr int kRing = 16;
 
-template <int BITS, bool SLOW>
+template <int BITS, bool SLOW, int LANES>
 struct LaneDecoder {
     static constexpr int kRunBits = 8 * BITS;
-    static constexpr uint32_t kRunStride = kLanes * BITS;  // bytes between a lane's runs in the stage
+    static constexpr uint32_t kRowBytes = 4 * LANES;           // one staged word of every lane
+    static constexpr uint32_t kRunStride = LANES * BITS;       // bytes between a lane's ring slots
     uint32_t lut;         // shared address of the decode table
-    uint32_t bufa;        // shared address of this lane's word 0; word j at bufa + 128 j
+    uint32_t bufa;        // shared address of this lane's next word; word j at word 0 + kRowBytes j
     uint32_t bufcap;      // shared address of the last readable word of this lane
     uint32_t ostb;        // shared address of this lane's slot 0 of the run ring
     uint32_t osta;        // shared address of this lane's current run slot
@@ -329,11 +331,11 @@ struct LaneDecoder {
     __device__ __forceinline__ void init(const Smem &s, const uint32_t *b, uint32_t *o, int cap) {
         lut = smem_addr(s.lut);
         bufa = smem_addr(b);
-        bufcap = bufa + 4u * kLanes * static_cast<uint32_t>(cap);
+        bufcap = bufa + kRowBytes * static_cast<uint32_t>(cap);
         ostb = osta = smem_addr(o);
-        win = (static_cast<uint64_t>(lds32(bufa)) << 32) | lds32(bufa + 4 * kLanes);
+        win = (static_cast<uint64_t>(lds32(bufa)) << 32) | lds32(bufa + kRowBytes);
         nb = 64;
-        bufa += 8 * kLanes;
+        bufa += 2 * kRowBytes;
         wnext = lds32(min(bufa, bufcap));
         p0 = p1 = p2 = 0;
         pb = 0;
@@ -344,7 +346,7 @@ struct LaneDecoder {
         if (nb <= 32) {
             win |= static_cast<uint64_t>(wnext) << (32 - nb);
             nb += 32;
-            bufa += 4 * kLanes;
+            bufa += kRowBytes;
             wnext = lds32(min(bufa, bufcap));
         }
     }
@@ -428,42 +430,52 @@ __device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int
     return v;
 }
 
-// Emit runs [tb, te) of a whole chunk (every lane owns 8 codes per run).
-template <int BITS, int OUT, int BPAD>
+// Emit runs [tb, te) of a whole chunk (every lane owns 8 codes per run);
+// thread `lane` serves the format lanes lane, lane + 32, ...
+template <int BITS, int OUT, int BPAD, int LANES>
 __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
                                           int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD]) {
+    constexpr int LPT = LANES / kLanes;
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
     if (OUT == OUT_CODES) {
         // staged codes are packed and in output order (the block's slots do not wrap): 16-byte copies
-        constexpr int kU4PerRun = kLanes * BITS / 16;  // uint4 per run of the warp (8 or 16)
+        constexpr int kU4PerRun = LANES * BITS / 16;  // uint4 per run of the chunk
         const uint4 *src = reinterpret_cast<const uint4 *>(ost) + (tb & (kRing - 1)) * kU4PerRun;
         uint4 *dst = reinterpret_cast<uint4 *>(g.out) + first * BITS / 128 + tb * kU4PerRun;
         for (int i = lane; i < (te - tb) * kU4PerRun; i += kLanes) dst[i] = src[i];
     } else if (OUT == OUT_BF16) {
         uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(g.out) + first);
         for (int t = tb; t < te; t++)
-            dst[kLanes * t + lane] = values8<BITS>(s, ost, kLanes * (t & (kRing - 1)) + lane);
+#pragma unroll
+            for (int k = 0; k < LPT; k++) {
+                const int l = lane + kLanes * k;
+                dst[LANES * t + l] = values8<BITS>(s, ost, LANES * (t & (kRing - 1)) + l);
+            }
     } else {
-        // fused GEMV: run t covers columns 256*(t % spr) + 8*lane .. +7 of row t / spr
+        // fused GEMV: run t covers columns 8*LANES*(t % spr) + 8*l .. +7 of row t / spr
         const int K = static_cast<int>(d.cols);
-        const int spr = K / kStepSymbols;
+        const int spr = K / (kRun * LANES);
         const long long row0 = first / K;
         const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
         for (int t = tb; t < te; t++) {
             const int st = t % spr;
-            const uint4 wv = values8<BITS>(s, ost, kLanes * (t & (kRing - 1)) + lane);
-            const int xo = st * kLanes + lane;  // uint4 index within one x row
 #pragma unroll
-            for (int b = 0; b < BPAD; b++) {
-                if (b < batch) {
-                    const int xi = b * (K >> 3) + xo;
-                    const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
-                    acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
-                    acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
-                    acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
-                    acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
+            for (int k = 0; k < LPT; k++) {
+                const int l = lane + kLanes * k;
+                const uint4 wv = values8<BITS>(s, ost, LANES * (t & (kRing - 1)) + l);
+                const int xo = st * LANES + l;  // uint4 index within one x row
+#pragma unroll
+                for (int b = 0; b < BPAD; b++) {
+                    if (b < batch) {
+                        const int xi = b * (K >> 3) + xo;
+                        const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                        acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
+                        acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
+                        acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
+                        acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
+                    }
                 }
             }
             if (st == spr - 1) {
@@ -482,114 +494,141 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
 }
 
 // Emit runs [tb, te) of a ragged (last) chunk of nc codes: only positions < nc.
-template <int BITS, int OUT>
+template <int BITS, int OUT, int LANES>
 __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
                                             int nc, int tb, int te) {
+    constexpr int LPT = LANES / kLanes;
     const int lane = threadIdx.x & 31;
     for (int t = tb; t < te; t++) {
-        const int w = kLanes * t + lane;        // output word: positions 8w .. 8w+7
-        const int cnt = min(8, nc - 8 * w);
-        if (cnt <= 0) continue;
-        const int slot = kLanes * (t & (kRing - 1)) + lane;
-        if (OUT == OUT_CODES) {
-            uint8_t *o = reinterpret_cast<uint8_t *>(g.out) + first * BITS / 8;
-            if (BITS == 4) {
-                const uint32_t c = ost[slot];
-                for (int k = 0; 2 * k < cnt; k++) {
-                    uint32_t b = (c >> (8 * k)) & 0xFFu;
-                    if (2 * k + 1 >= cnt) b &= 0xFu;
-                    o[4 * w + k] = static_cast<uint8_t>(b);
+        for (int k = 0; k < LPT; k++) {
+            const int l = lane + kLanes * k;
+            const int w = LANES * t + l;            // output word: positions 8w .. 8w+7
+            const int cnt = min(8, nc - 8 * w);
+            if (cnt <= 0) continue;
+            const int slot = LANES * (t & (kRing - 1)) + l;
+            if (OUT == OUT_CODES) {
+                uint8_t *o = reinterpret_cast<uint8_t *>(g.out) + first * BITS / 8;
+                if (BITS == 4) {
+                    const uint32_t c = ost[slot];
+                    for (int q = 0; 2 * q < cnt; q++) {
+                        uint32_t b = (c >> (8 * q)) & 0xFFu;
+                        if (2 * q + 1 >= cnt) b &= 0xFu;
+                        o[4 * w + q] = static_cast<uint8_t>(b);
+                    }
+                } else {
+                    const uint8_t *c = reinterpret_cast<const uint8_t *>(ost) + 8 * slot;
+                    for (int q = 0; q < cnt; q++) o[8 * w + q] = c[q];
                 }
-            } else {
-                const uint8_t *c = reinterpret_cast<const uint8_t *>(ost) + 8 * slot;
-                for (int k = 0; k < cnt; k++) o[8 * w + k] = c[k];
-            }
-        } else if (OUT == OUT_BF16) {
-            const uint4 v = values8<BITS>(s, ost, slot);
-            uint16_t *o = reinterpret_cast<uint16_t *>(g.out) + first + 8 * w;
-            if (cnt == 8) {
-                *reinterpret_cast<uint4 *>(o) = v;
-            } else {
-                for (int k = 0; k < cnt; k++) {
-                    const uint32_t pair = (k < 2) ? v.x : (k < 4) ? v.y : (k < 6) ? v.z : v.w;
-                    o[k] = static_cast<uint16_t>(pair >> (16 * (k & 1)));
+            } else if (OUT == OUT_BF16) {
+                const uint4 v = values8<BITS>(s, ost, slot);
+                uint16_t *o = reinterpret_cast<uint16_t *>(g.out) + first + 8 * w;
+                if (cnt == 8) {
+                    *reinterpret_cast<uint4 *>(o) = v;
+                } else {
+                    for (int q = 0; q < cnt; q++) {
+                        const uint32_t pair = (q < 2) ? v.x : (q < 4) ? v.y : (q < 6) ? v.z : v.w;
+                        o[q] = static_cast<uint16_t>(pair >> (16 * (q & 1)));
+                    }
                 }
             }
         }
     }
 }
 
-// Decode chunk c of entry g from its staged words.  Whole chunks are emitted
-// every kEmitBlock runs, so the stores of one block drain while the lanes
-// decode the next.
-template <int BITS, int OUT, bool SLOW, int BPAD>
+// Decode chunk c of entry g from its staged words.  Thread `lane` decodes the
+// format lanes lane, lane + 32, ... as independent interleaved streams.  Whole
+// chunks are emitted every kEmitBlock runs, so the stores of one block drain
+// while the lanes decode the next.
+template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
 __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const uint32_t *buf,
                                              uint32_t *ost, int stage_rows, long long c, int batch, int x_in_smem,
                                              int32_t *status) {
+    constexpr int LPT = LANES / kLanes;
+    constexpr int kStep = kRun * LANES;  // symbols per lane step
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
     const long long st = static_cast<long long>(d.index[2 * c]);
     const long long nx = static_cast<long long>(d.index[2 * c + 2]);
-    const int words = static_cast<int>((nx - st) / kLanes);
+    const int words = static_cast<int>((nx - st) / LANES);
     const long long first = c * d.chunk_symbols;
     const long long remain = d.n - first;
     const int nc = static_cast<int>(remain < d.chunk_symbols ? remain : d.chunk_symbols);
     const bool refill_each = SLOW && d.max_len > 16;
-    uint32_t *lost = ost + (BITS == 4 ? lane : 2 * lane);
-    LaneDecoder<BITS, SLOW> ld;
-    ld.init(s, buf + lane, lost, stage_rows - 1);
-    // a valid lane never loads past its words plus the two read-ahead rows
-    const uint32_t read_limit = smem_addr(buf + lane) + 4u * kLanes * static_cast<uint32_t>(words + kSlackRows);
+    LaneDecoder<BITS, SLOW, LANES> ld[LPT];
+    uint32_t read_limit[LPT];
+#pragma unroll
+    for (int k = 0; k < LPT; k++) {
+        const int l = lane + kLanes * k;
+        ld[k].init(s, buf + l, ost + (BITS == 4 ? l : 2 * l), stage_rows - 1);
+        // a valid lane never loads past its words plus the two read-ahead rows
+        read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kSlackRows);
+    }
     bool ok = true;
     if (nc == d.chunk_symbols) {
-        const int runs = nc / kStepSymbols;
+        const int runs = nc / kStep;
         float acc[BPAD];
 #pragma unroll
         for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
-            while (ld.t < te) {
-                ld.refill();
-                ld.lookup(s, d.max_len, status);
-                ld.emit();
-                if (SLOW && refill_each) ld.refill();
-                ld.lookup(s, d.max_len, status);
-                ld.emit();
+            bool more = true;
+            while (more) {
+                more = false;
+#pragma unroll
+                for (int k = 0; k < LPT; k++) {
+                    if (ld[k].t < te) {
+                        ld[k].refill();
+                        ld[k].lookup(s, d.max_len, status);
+                        ld[k].emit();
+                        if (SLOW && refill_each) ld[k].refill();
+                        ld[k].lookup(s, d.max_len, status);
+                        ld[k].emit();
+                        more = more || ld[k].t < te;
+                    }
+                }
             }
             __syncwarp();
-            emit_runs<BITS, OUT, BPAD>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
+            emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
             __syncwarp();  // the ring slots just read are rewritten by the next block
         }
-        ok = ld.bufa <= read_limit;
+#pragma unroll
+        for (int k = 0; k < LPT; k++) ok = ok && ld[k].bufa <= read_limit[k];
     } else {
-        // symbols of this lane: positions 256*t + 8*lane + i < nc
-        const int full_steps = nc / kStepSymbols, rem = nc % kStepSymbols;
-        const int S = 8 * full_steps + max(0, min(8, rem - 8 * lane));
-        const int full_runs = S >> 3, tail = S & 7;
-        const int steps = (nc + kStepSymbols - 1) / kStepSymbols;
+        // symbols of lane l: positions kStep*t + 8*l + i < nc
+        const int full_steps = nc / kStep, rem = nc % kStep;
+        const int steps = (nc + kStep - 1) / kStep;
+        int S[LPT];
+#pragma unroll
+        for (int k = 0; k < LPT; k++) S[k] = 8 * full_steps + max(0, min(8, rem - 8 * (lane + kLanes * k)));
         for (int tb = 0; tb < steps; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, steps);
-            const int tf = min(te, full_runs);
-            while (ld.t < tf) {
-                ld.refill();
-                ld.lookup(s, d.max_len, status);
-                ld.emit();
-                if (SLOW && refill_each) ld.refill();
-                ld.lookup(s, d.max_len, status);
-                ld.emit();
-            }
-            if (tail && ld.t == full_runs && full_runs < te) {
-                while (ld.pb < tail * BITS) {
-                    ld.refill();
-                    ld.lookup(s, d.max_len, status);
+#pragma unroll
+            for (int k = 0; k < LPT; k++) {
+                const int full_runs = S[k] >> 3, tail = S[k] & 7;
+                const int tf = min(te, full_runs);
+                while (ld[k].t < tf) {
+                    ld[k].refill();
+                    ld[k].lookup(s, d.max_len, status);
+                    ld[k].emit();
+                    if (SLOW && refill_each) ld[k].refill();
+                    ld[k].lookup(s, d.max_len, status);
+                    ld[k].emit();
                 }
-                ld.close_run();
+                if (tail && ld[k].t == full_runs && full_runs < te) {
+                    while (ld[k].pb < tail * BITS) {
+                        ld[k].refill();
+                        ld[k].lookup(s, d.max_len, status);
+                    }
+                    ld[k].close_run();
+                }
             }
             __syncwarp();
-            emit_ragged<BITS, OUT>(g, s, ost, first, nc, tb, te);
+            emit_ragged<BITS, OUT, LANES>(g, s, ost, first, nc, tb, te);
             __syncwarp();
         }
-        if (S > 0) ok = ld.bufa <= read_limit;
+#pragma unroll
+        for (int k = 0; k < LPT; k++)
+            if (S[k] > 0) ok = ok && ld[k].bufa <= read_limit[k];
     }
     if (!ok) set_status(status, ENTRO_E_OVERRUN);
     __syncwarp();
@@ -599,35 +638,35 @@ __device__ __forceinline__ const GroupEntry &entry_at(const LaunchArgs &a, int i
     return a.table ? a.table[i] : a.one;
 }
 
-__device__ __forceinline__ bool chunk_words_ok(const DevTensor &d, long long c, int stage_rows) {
+__device__ __forceinline__ bool chunk_words_ok(const DevTensor &d, long long c, int stage_rows, int lanes) {
     const uint64_t st = d.index[2 * c], nx = d.index[2 * c + 2];
-    return nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % kLanes == 0 &&
-           (nx - st) / kLanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
+    return nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % lanes == 0 &&
+           (nx - st) / lanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
 }
 
 // Issue the staging copy of a chunk whose words are [st, nx) (one lane).  An
 // inconsistent index arrives with no bytes; the consumer re-checks and skips.
 __device__ __forceinline__ void issue_words(const DevTensor &d, uint64_t st, uint64_t nx, uint32_t *buf,
-                                            uint64_t *bar, int stage_rows) {
-    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % kLanes == 0 &&
-                    (nx - st) / kLanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
+                                            uint64_t *bar, int stage_rows, int lanes) {
+    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % lanes == 0 &&
+                    (nx - st) / lanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
     const uint32_t bytes = ok ? static_cast<uint32_t>((nx - st) * 4) : 0u;
     mbar_arrive_expect_tx(bar, bytes);
     if (bytes) bulk_copy_g2s(buf, d.payload + st, bytes, bar);
 }
 
 __device__ __forceinline__ void issue_chunk(const DevTensor &d, long long c, uint32_t *buf, uint64_t *bar,
-                                            int stage_rows) {
-    issue_words(d, d.index[2 * c], d.index[2 * c + 2], buf, bar, stage_rows);
+                                            int stage_rows, int lanes) {
+    issue_words(d, d.index[2 * c], d.index[2 * c + 2], buf, bar, stage_rows, lanes);
 }
 
-template <int BITS, int OUT, bool SLOW, int BPAD>
+template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows, a.out_words);
+    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words);
     uint64_t *bar = s.bars + 2 * warp;
-    const size_t buf_words = static_cast<size_t>(a.stage_rows) * kLanes;
+    const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
     uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
     uint32_t *ost = s.ostage + static_cast<size_t>(warp) * a.out_words;
     if (lane == 0) {
@@ -675,8 +714,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
             const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
             if (lane == 0) {
-                if (c < cb) issue_words(g.d, st0, nx0, stage, bar, a.stage_rows);
-                if (c + warps < cb) issue_words(g.d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows);
+                if (c < cb) issue_words(g.d, st0, nx0, stage, bar, a.stage_rows, LANES);
+                if (c + warps < cb) issue_words(g.d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES);
             }
             pend0 = c < cb;
             pend1 = c + warps < cb;
@@ -699,15 +738,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
                 }
                 if (b) { phase1++; pend1 = false; }
                 else { phase0++; pend0 = false; }
-                if (chunk_words_ok(g.d, c, a.stage_rows))
-                    decode_chunk<BITS, OUT, SLOW, BPAD>(g, s, stage + b * buf_words, ost, a.stage_rows, c, a.batch,
-                                                        a.x_in_smem, a.status);
+                if (chunk_words_ok(g.d, c, a.stage_rows, LANES))
+                    decode_chunk<BITS, OUT, SLOW, BPAD, LANES>(g, s, stage + b * buf_words, ost, a.stage_rows, c,
+                                                               a.batch, a.x_in_smem, a.status);
                 else
                     set_status(a.status, ENTRO_E_CORRUPT);
                 if (c + 2 * warps < cb) {
                     if (lane == 0) {
                         fence_proxy_async();
-                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows);
+                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES);
                     }
                     if (b) pend1 = true;
                     else pend0 = true;
@@ -1055,6 +1094,7 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     d.format = (int)b.header.format;
     d.max_chunk_words = (int)b.max_chunk_words;
     d.n_codes = n_codes;
+    d.lanes = (int)b.header.lanes;
     t->device = dev;
     t->slow = d.max_len > kMaxLutBits || n_codes == 1;
     t->device_bytes = L.total;
@@ -1068,27 +1108,28 @@ namespace entro {
 
 using LanesFn = void (*)(LaunchArgs);
 
-template <int BITS, int OUT, bool SLOW>
+template <int BITS, int OUT, bool SLOW, int LANES>
 static LanesFn pick_bpad(int bpad) {
-    if (OUT != OUT_GEMV) return lanes_kernel<BITS, OUT, SLOW, 1>;
+    if (OUT != OUT_GEMV) return lanes_kernel<BITS, OUT, SLOW, 1, LANES>;
     switch (bpad) {
-        case 1: return lanes_kernel<BITS, OUT, SLOW, 1>;
-        case 2: return lanes_kernel<BITS, OUT, SLOW, 2>;
-        case 4: return lanes_kernel<BITS, OUT, SLOW, 4>;
-        case 8: return lanes_kernel<BITS, OUT, SLOW, 8>;
-        default: return lanes_kernel<BITS, OUT, SLOW, 16>;
+        case 1: return lanes_kernel<BITS, OUT, SLOW, 1, LANES>;
+        case 2: return lanes_kernel<BITS, OUT, SLOW, 2, LANES>;
+        case 4: return lanes_kernel<BITS, OUT, SLOW, 4, LANES>;
+        case 8: return lanes_kernel<BITS, OUT, SLOW, 8, LANES>;
+        default: return lanes_kernel<BITS, OUT, SLOW, 16, LANES>;
     }
 }
 
-static LanesFn pick_lanes(int bits, int out, bool slow, int bpad) {
-    if (bits == 4) {
-        if (out == OUT_CODES) return slow ? pick_bpad<4, OUT_CODES, true>(1) : pick_bpad<4, OUT_CODES, false>(1);
-        if (out == OUT_BF16) return slow ? pick_bpad<4, OUT_BF16, true>(1) : pick_bpad<4, OUT_BF16, false>(1);
-        return slow ? pick_bpad<4, OUT_GEMV, true>(bpad) : pick_bpad<4, OUT_GEMV, false>(bpad);
-    }
-    if (out == OUT_CODES) return slow ? pick_bpad<8, OUT_CODES, true>(1) : pick_bpad<8, OUT_CODES, false>(1);
-    if (out == OUT_BF16) return slow ? pick_bpad<8, OUT_BF16, true>(1) : pick_bpad<8, OUT_BF16, false>(1);
-    return slow ? pick_bpad<8, OUT_GEMV, true>(bpad) : pick_bpad<8, OUT_GEMV, false>(bpad);
+template <int BITS, int LANES>
+static LanesFn pick_out(int out, bool slow, int bpad) {
+    if (out == OUT_CODES) return slow ? pick_bpad<BITS, OUT_CODES, true, LANES>(1) : pick_bpad<BITS, OUT_CODES, false, LANES>(1);
+    if (out == OUT_BF16) return slow ? pick_bpad<BITS, OUT_BF16, true, LANES>(1) : pick_bpad<BITS, OUT_BF16, false, LANES>(1);
+    return slow ? pick_bpad<BITS, OUT_GEMV, true, LANES>(bpad) : pick_bpad<BITS, OUT_GEMV, false, LANES>(bpad);
+}
+
+static LanesFn pick_lanes(int bits, int out, bool slow, int bpad, int lanes) {
+    if (bits == 4) return lanes == 64 ? pick_out<4, 64>(out, slow, bpad) : pick_out<4, 32>(out, slow, bpad);
+    return lanes == 64 ? pick_out<8, 64>(out, slow, bpad) : pick_out<8, 32>(out, slow, bpad);
 }
 
 static LanesFn pick_single(int bits, int out, bool slow) {
@@ -1164,12 +1205,12 @@ static constexpr long long kXSmemElems = 48 * 1024;  // up to 96 KB of bf16 acti
 static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
                         const GroupEntry &one, int32_t *status, cudaStream_t st) {
     bool slow = false;
-    const int bits = ts[0]->d.bits;
+    const int bits = ts[0]->d.bits, lanes = ts[0]->d.lanes;
     int max_words = 0;
     long long max_kb = 0, max_chunk = 0, total = 0;
     for (int i = 0; i < count; i++) {
         const DevTensor &d = ts[i]->d;
-        if (d.bits != bits) return ENTRO_E_INVAL;
+        if (d.bits != bits || d.lanes != lanes) return ENTRO_E_INVAL;
         slow = slow || ts[i]->slow;
         max_words = std::max(max_words, d.max_chunk_words);
         max_chunk = std::max(max_chunk, d.chunk_symbols);
@@ -1182,7 +1223,7 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
     long long x_elems = (out_kind == OUT_GEMV && max_kb <= kXSmemElems) ? max_kb : 0;
     const int stage_rows = max_words + kSlackRows;
-    const int out_words = kRing * kLanes * bits / 4;  // the run ring: kRing runs of 8 codes per lane
+    const int out_words = kRing * lanes * bits / 4;  // the run ring: kRing runs of 8 codes per lane
     long long chunks = 0;
     for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
     // Spread the chunks evenly over the SMs: small inputs get one CTA per SM
@@ -1190,14 +1231,14 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     int warps = (int)std::min<long long>(kMaxWarps, std::max<long long>(1, (chunks + di.sms - 1) / di.sms));
     SmemOffsets so;
     for (;;) {
-        so = smem_layout(warps, x_elems, stage_rows, out_words);
+        so = smem_layout(warps, x_elems, stage_rows * lanes, out_words);
         if ((long long)so.total <= di.smem_optin) break;
         if (warps > 1) warps--;
         else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
         else return ENTRO_E_LIMIT;
     }
     const size_t bytes = so.total;
-    LanesFn fn = pick_lanes(bits, out_kind, slow, bpad);
+    LanesFn fn = pick_lanes(bits, out_kind, slow, bpad, lanes);
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, bytes, &per_sm) != ENTRO_OK)
         return ENTRO_E_CUDA;
@@ -1265,7 +1306,7 @@ static int gemv_check(const TensorHandle *t, const void *x, int batch, const flo
     if (reinterpret_cast<uintptr_t>(x) & 15) return ENTRO_E_INVAL;
     const DevTensor &d = t->d;
     if (d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
-    if (d.cols <= 0 || d.cols % kStepSymbols || d.chunk_symbols % d.cols) return ENTRO_E_INVAL;
+    if (d.cols <= 0 || d.cols % (kRun * d.lanes) || d.chunk_symbols % d.cols) return ENTRO_E_INVAL;
     return ENTRO_OK;
 }
 

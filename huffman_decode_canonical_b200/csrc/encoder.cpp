@@ -320,13 +320,16 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     if (o->bits != 4 && o->bits != 8) return ENTRO_E_INVAL;
     if (o->quant_mode < 0 || o->quant_mode > 2) return ENTRO_E_INVAL;
     if (o->format != ENTRO_FORMAT_SINGLE && o->format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
-    if (o->reserved != 0 || o->threads < 0) return ENTRO_E_INVAL;
+    if (o->threads < 0) return ENTRO_E_INVAL;
     const int bits = o->bits, nsym = 1 << bits;
     const int max_len = o->max_len ? o->max_len : (bits == 8 ? 16 : 12);
     if (max_len < 1 || max_len > kMaxLenLimit) return ENTRO_E_INVAL;
     const bool lanes = o->format == ENTRO_FORMAT_LANES;
+    const int L = lanes ? (o->lanes ? o->lanes : kLanes) : 1;
+    if (lanes && L != 32 && L != 64) return ENTRO_E_INVAL;
+    const int64_t step = (int64_t)kRun * L;
     int64_t C = o->chunk_symbols ? o->chunk_symbols : (lanes ? 8192 : 4096);
-    if (lanes && (C < kStepSymbols || C > kMaxLanesChunk || C % kStepSymbols)) return ENTRO_E_INVAL;
+    if (lanes && (C < step || C > kMaxLanesChunk || C % step)) return ENTRO_E_INVAL;
     if (!lanes && (C < 1 || C > kMaxSingleChunk)) return ENTRO_E_INVAL;
     const int64_t n = rows * cols;
     const int threads = pick_threads(o->threads, n);
@@ -371,11 +374,11 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
                 for (int64_t i = a; i < b; i++) s += len[q[i]];
                 csize[c] = s;
             } else {
-                uint64_t lb[kLanes] = {0};
-                for (int64_t p = 0; p < b - a; p++) lb[(p % kStepSymbols) / kRun] += len[q[a + p]];
+                uint64_t lb[kMaxLanes] = {0};
+                for (int64_t p = 0; p < b - a; p++) lb[(p % step) / kRun] += len[q[a + p]];
                 uint64_t wmax = 0;
-                for (int l = 0; l < kLanes; l++) wmax = std::max<uint64_t>(wmax, (lb[l] + 31) / 32);
-                csize[c] = wmax * kLanes;
+                for (int l = 0; l < L; l++) wmax = std::max<uint64_t>(wmax, (lb[l] + 31) / 32);
+                csize[c] = wmax * (uint64_t)L;
             }
         }
     });
@@ -400,7 +403,7 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     h.scheme = (uint32_t)qp.scheme;
     h.max_len = (uint32_t)max_len;
     h.format = (uint32_t)o->format;
-    h.lanes = lanes ? kLanes : 1;
+    h.lanes = (uint32_t)L;
     h.run = lanes ? kRun : 1;
     h.rows = (uint64_t)rows;
     h.cols = (uint64_t)cols;
@@ -444,9 +447,9 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
                 }
             } else {
                 uint32_t *cbase = payload + start[c];
-                for (int l = 0; l < kLanes; l++) {
-                    BitSink s{cbase + l, kLanes};
-                    for (int64_t t0 = 0; t0 < b - a; t0 += kStepSymbols) {
+                for (int l = 0; l < L; l++) {
+                    BitSink s{cbase + l, L};
+                    for (int64_t t0 = 0; t0 < b - a; t0 += step) {
                         const int64_t p0 = t0 + (int64_t)l * kRun;
                         const int64_t p1 = std::min<int64_t>(b - a, p0 + kRun);
                         for (int64_t p = p0; p < p1; p++) s.put(code[q[a + p]], len[q[a + p]]);
@@ -482,9 +485,11 @@ int Blob::finalize_info() {
     if (h.max_len < 1 || h.max_len > (uint32_t)kMaxLenLimit) return ENTRO_E_FORMAT;
     const bool lanes = h.format == ENTRO_FORMAT_LANES;
     if (!lanes && h.format != ENTRO_FORMAT_SINGLE) return ENTRO_E_FORMAT;
-    if (h.lanes != (lanes ? (uint32_t)kLanes : 1u) || h.run != (lanes ? (uint32_t)kRun : 1u)) return ENTRO_E_FORMAT;
+    if (lanes ? (h.lanes != 32 && h.lanes != 64) : h.lanes != 1) return ENTRO_E_FORMAT;
+    if (h.run != (lanes ? (uint32_t)kRun : 1u)) return ENTRO_E_FORMAT;
     if (h.chunk_symbols == 0) return ENTRO_E_FORMAT;
-    if (lanes && (h.chunk_symbols % kStepSymbols || h.chunk_symbols > (uint64_t)kMaxLanesChunk)) return ENTRO_E_FORMAT;
+    if (lanes && (h.chunk_symbols % (kRun * h.lanes) || h.chunk_symbols > (uint64_t)kMaxLanesChunk))
+        return ENTRO_E_FORMAT;
     if (!lanes && h.chunk_symbols > (uint64_t)kMaxSingleChunk) return ENTRO_E_FORMAT;
     if (h.cols != 0 && h.rows > UINT64_MAX / h.cols) return ENTRO_E_FORMAT;
     if (h.n != h.rows * h.cols) return ENTRO_E_FORMAT;
@@ -516,8 +521,8 @@ int Blob::finalize_info() {
         if (c == 0 ? st != 0 : st < prev) return ENTRO_E_FORMAT;
         if (c > 0 && lanes) {
             const uint64_t wc = st - prev;
-            if (wc % kLanes) return ENTRO_E_FORMAT;
-            maxw = std::max<uint64_t>(maxw, wc / kLanes);
+            if (wc % h.lanes) return ENTRO_E_FORMAT;
+            maxw = std::max<uint64_t>(maxw, wc / h.lanes);
         }
         if (c > 0 && !lanes) maxw = std::max<uint64_t>(maxw, (st + 31) / 32 - prev / 32);
         prev = st;
@@ -590,6 +595,7 @@ extern "C" int entro_blob_info(const entro_blob *blob, entro_info *out) {
     out->index_bytes = 16 * (h.n_chunks + 1);
     out->blob_bytes = b->bytes.size();
     out->max_chunk_words = (uint32_t)b->max_chunk_words;
+    out->lanes = h.lanes;
     std::memcpy(out->lengths, b->lengths, 256);
     out->coded_bits = b->coded_bits;
     return ENTRO_OK;

@@ -72,10 +72,11 @@ typedef struct entro_encode_opts {
     int32_t quant_mode;    /* ENTRO_QUANT_* */
     int32_t max_len;       /* code length limit, 1..24; 0 = 16 for 8-bit, 12 for 4-bit */
     int32_t format;        /* ENTRO_FORMAT_* */
-    int64_t chunk_symbols; /* 0 = 4096 (single) / 8192 (lanes).  Lanes: a multiple of 256 in
-                              [256, 16384].  Single: 1 .. 2^20. */
+    int64_t chunk_symbols; /* 0 = 4096 (single) / 8192 (lanes).  Lanes: a multiple of 8 * lanes
+                              in [8 * lanes, 16384].  Single: 1 .. 2^20. */
     int32_t threads;       /* host threads for encoding; 0 = all hardware threads */
-    int32_t reserved;      /* must be 0 */
+    int32_t lanes;         /* lanes format: 32 (also 0) or 64 interleaved lanes per chunk; a chunk
+                              must then hold a multiple of 8 * lanes symbols */
 } entro_encode_opts;
 
 typedef struct entro_blob entro_blob;     /* host copy of one encoded tensor (serialized bytes) */
@@ -92,13 +93,14 @@ typedef struct entro_info {
     uint64_t coded_bits;      /* sum of the code lengths of all symbols (0 if unknown: a lanes
                                  blob read back with entro_blob_from_bytes) */
     uint32_t max_chunk_words; /* lanes: longest lane of any chunk in 32-bit words */
-    uint32_t reserved;
+    uint32_t lanes;           /* interleaved lanes per chunk (1 for the single-stream format) */
     uint8_t lengths[256];     /* code length per symbol, 0 = symbol absent */
 } entro_info;
 
 /* Quantize a row-major fp32 [rows, cols] tensor on the host, build its
  * length-limited canonical Huffman code (package-merge, RFC 1951 canonical
- * order) and encode it in chunks.  *out receives a library-owned blob; free it
+ * order) and encode it in chunks (LazyWeights abstract: "interleaved lanes"; the
+ * lane count is a format parameter).  *out receives a library-owned blob; free it
  * with entro_blob_free.  rows*cols may be 0 (an empty blob).  Errors:
  * E_INVAL (NaN/Inf weight, bad option, null pointer, UNSIGNED with a negative
  * weight), E_LIMIT (more distinct codes than 2^max_len allows, zero point
@@ -147,8 +149,8 @@ ENTRO_API int entro_decode_dequant_bf16(const entro_tensor *t, void *d_out, int3
  * r < rows, d_y[b*rows + r] = sum_k w[r,k] * x[b*cols + k], w the bf16
  * weights of entro_decode_dequant_bf16 (never written to memory), x bf16
  * [batch, cols], accumulation in fp32.  Needs the lanes format, cols a
- * multiple of 256 and chunk_symbols a multiple of cols (chunks of whole
- * rows); batch in 1..16; d_x 16-byte aligned.  Rows are reduced in a fixed
+ * multiple of 8 * lanes (256 or 512) and chunk_symbols a multiple of cols
+ * (chunks of whole rows); batch in 1..16; d_x 16-byte aligned.  Rows are reduced in a fixed
  * order, so results are bit-reproducible. */
 ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t batch, float *d_y,
                       int32_t *d_status, void *stream);

@@ -63,7 +63,7 @@ def _load():
             lib.or_entropy.restype = ctypes.c_double
             lib.or_code_lengths.argtypes = [P, i32, i32, P]
             lib.or_canonical_codes.argtypes = [P, i32, P]
-            lib.or_encode.argtypes = [P, i64, i64, i32, i32, i32, i32, i64, P, u64, P]
+            lib.or_encode.argtypes = [P, i64, i64, i32, i32, i32, i32, i64, i32, P, u64, P]
             lib.or_decode.argtypes = [P, u64, P]
             lib.or_decode_chunks.argtypes = [P, u64, u64, u64, P]
             lib.or_blob_params.argtypes = [P, u64, P]
@@ -123,18 +123,19 @@ def canonical_codes(lengths: np.ndarray) -> np.ndarray:
     return out
 
 
-def encode(w: np.ndarray, bits: int, mode: int, max_len: int, fmt: int, chunk_symbols: int) -> bytes:
-    """Whole encoder: fp32 [rows, cols] -> serialized blob bytes."""
+def encode(w: np.ndarray, bits: int, mode: int, max_len: int, fmt: int, chunk_symbols: int,
+           lanes: int = 32) -> bytes:
+    """Whole encoder: fp32 [rows, cols] -> serialized blob bytes (lanes: 32 or 64 for the lanes format)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     if w.ndim != 2:
         raise ValueError("w must be 2-D")
     rows, cols = w.shape
     size = np.zeros(1, np.uint64)
     lib = _load()
-    _check(lib.or_encode(_ptr(w), rows, cols, bits, mode, max_len, fmt, chunk_symbols,
+    _check(lib.or_encode(_ptr(w), rows, cols, bits, mode, max_len, fmt, chunk_symbols, lanes,
                          None, 0, _ptr(size)), "encode(size)")
     out = np.zeros(int(size[0]), np.uint8)
-    _check(lib.or_encode(_ptr(w), rows, cols, bits, mode, max_len, fmt, chunk_symbols,
+    _check(lib.or_encode(_ptr(w), rows, cols, bits, mode, max_len, fmt, chunk_symbols, lanes,
                          _ptr(out), out.size, _ptr(size)), "encode")
     return out.tobytes()
 

@@ -33,9 +33,10 @@
  *  - package-merge ties: leaves sorted by (count, symbol); at equal weight a
  *    leaf precedes a package; a one-symbol alphabet gets length 1;
  *  - codes are written MSB-first into 32-bit words;
- *  - lane layout: 32 lanes, lane l holds runs of 8 consecutive symbols at
- *    chunk positions 256*t + 8*l + (0..7), each lane padded to the chunk's
- *    longest lane, word j of lane l stored at chunk_word_base + 32*j + l.
+ *  - lane layout: L lanes (32 or 64, a format parameter), lane l holds runs
+ *    of 8 consecutive symbols at chunk positions 8*L*t + 8*l + (0..7), each
+ *    lane padded to the chunk's longest lane, word j of lane l stored at
+ *    chunk_word_base + L*j + l.
  *
  * Numeric formulas checked elsewhere against independent pins (see tests).
  */
@@ -61,7 +62,6 @@
 #define OR_FMT_SINGLE 1
 #define OR_FMT_LANES 2
 
-#define OR_LANES 32
 #define OR_RUN 8
 #define OR_HEADER_BYTES 128
 #define OR_LENGTHS_BYTES 256
@@ -384,14 +384,18 @@ static void put_code(bitw *bw, uint32_t code, int length) {
  */
 
 int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, int max_len,
-              int format, int64_t chunk_symbols, uint8_t *out, uint64_t cap, uint64_t *out_size) {
+              int format, int64_t chunk_symbols, int lanes, uint8_t *out, uint64_t cap, uint64_t *out_size) {
     if (rows < 0 || cols < 0 || (bits != 4 && bits != 8)) return OR_EINVAL;
     if (format != OR_FMT_SINGLE && format != OR_FMT_LANES) return OR_EINVAL;
     if (max_len == 0) max_len = (bits == 8) ? 16 : 12;
     if (max_len < 1 || max_len > 24) return OR_EINVAL;
     if (chunk_symbols == 0) chunk_symbols = (format == OR_FMT_SINGLE) ? 4096 : 8192;
     if (format == OR_FMT_SINGLE && (chunk_symbols < 1 || chunk_symbols > (1 << 20))) return OR_EINVAL;
-    if (format == OR_FMT_LANES && (chunk_symbols < 256 || chunk_symbols > 16384 || chunk_symbols % 256 != 0))
+    if (format == OR_FMT_LANES && lanes == 0) lanes = 32;
+    if (format == OR_FMT_LANES && lanes != 32 && lanes != 64) return OR_EINVAL;
+    const int64_t step = (int64_t)OR_RUN * lanes; /* symbols per lane step */
+    if (format == OR_FMT_LANES &&
+        (chunk_symbols < step || chunk_symbols > 16384 || chunk_symbols % step != 0))
         return OR_EINVAL;
     int64_t n = rows * cols;
     int nsym = 1 << bits;
@@ -435,14 +439,14 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
             uint64_t a = c * (uint64_t)chunk_symbols, b = a + (uint64_t)chunk_symbols;
             if (b > (uint64_t)n) b = (uint64_t)n;
             uint64_t nc = b - a, wmax = 0;
-            for (int l = 0; l < OR_LANES; l++) {
+            for (int l = 0; l < lanes; l++) {
                 uint64_t lane_bits = 0;
                 for (uint64_t p = 0; p < nc; p++)
-                    if ((p % 256) / OR_RUN == (uint64_t)l) lane_bits += len[q[a + p]];
+                    if ((p % (uint64_t)step) / OR_RUN == (uint64_t)l) lane_bits += len[q[a + p]];
                 uint64_t wl = (lane_bits + 31) / 32;
                 if (wl > wmax) wmax = wl;
             }
-            wpos += wmax * OR_LANES;
+            wpos += wmax * (uint64_t)lanes;
         }
         start[n_chunks] = wpos;
         payload_words = wpos;
@@ -460,7 +464,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     put_u32(out + 12, (uint32_t)scheme);
     put_u32(out + 16, (uint32_t)max_len);
     put_u32(out + 20, (uint32_t)format);
-    put_u32(out + 24, format == OR_FMT_SINGLE ? 1u : (uint32_t)OR_LANES);
+    put_u32(out + 24, format == OR_FMT_SINGLE ? 1u : (uint32_t)lanes);
     put_u32(out + 28, format == OR_FMT_SINGLE ? 1u : (uint32_t)OR_RUN);
     put_u64(out + 32, (uint64_t)rows);
     put_u64(out + 40, (uint64_t)cols);
@@ -492,15 +496,15 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
             uint64_t a = c * (uint64_t)chunk_symbols, b = a + (uint64_t)chunk_symbols;
             if (b > (uint64_t)n) b = (uint64_t)n;
             uint64_t nc = b - a;
-            uint64_t wmax = (start[c + 1] - start[c]) / OR_LANES;
+            uint64_t wmax = (start[c + 1] - start[c]) / (uint64_t)lanes;
             uint32_t *lane_words = (uint32_t *)calloc(wmax ? wmax : 1, sizeof(uint32_t));
             if (!lane_words) { free(q); free(start); free(payload); return OR_ENOMEM; }
-            for (int l = 0; l < OR_LANES; l++) {
+            for (int l = 0; l < lanes; l++) {
                 memset(lane_words, 0, sizeof(uint32_t) * (wmax ? wmax : 1));
                 bitw bw = {lane_words, 0};
                 for (uint64_t p = 0; p < nc; p++)
-                    if ((p % 256) / OR_RUN == (uint64_t)l) put_code(&bw, code[q[a + p]], len[q[a + p]]);
-                for (uint64_t j = 0; j < wmax; j++) payload[start[c] + OR_LANES * j + l] = lane_words[j];
+                    if ((p % (uint64_t)step) / OR_RUN == (uint64_t)l) put_code(&bw, code[q[a + p]], len[q[a + p]]);
+                for (uint64_t j = 0; j < wmax; j++) payload[start[c] + (uint64_t)lanes * j + l] = lane_words[j];
             }
             free(lane_words);
         }
@@ -551,6 +555,8 @@ static int parse(const uint8_t *blob, uint64_t size, or_blob *b) {
     b->payload_words = get_u64(blob + 80);
     if (b->bits != 4 && b->bits != 8) return OR_EFORMAT;
     if (b->format != OR_FMT_SINGLE && b->format != OR_FMT_LANES) return OR_EFORMAT;
+    if (b->format == OR_FMT_LANES && b->lanes != 32 && b->lanes != 64) return OR_EFORMAT;
+    if (b->format == OR_FMT_SINGLE && b->lanes != 1) return OR_EFORMAT;
     if (b->max_len < 1 || b->max_len > 24) return OR_EFORMAT;
     if (b->chunk_symbols == 0 || b->n != b->rows * b->cols) return OR_EFORMAT;
     if (b->n_chunks != (b->n + b->chunk_symbols - 1) / b->chunk_symbols) return OR_EFORMAT;
@@ -583,7 +589,7 @@ typedef int (*bit_fn)(const or_blob *, const void *ctx, uint64_t pos);
 
 typedef struct {
     uint64_t word_base;
-    int lane;
+    int lane, lanes;
     uint64_t words;
 } lane_ctx;
 
@@ -591,7 +597,7 @@ static int bit_lane(const or_blob *b, const void *ctx, uint64_t pos) {
     const lane_ctx *lc = (const lane_ctx *)ctx;
     uint64_t j = pos >> 5;
     if (j >= lc->words) return -1;
-    uint32_t word = get_u32(b->payload + 4 * (lc->word_base + OR_LANES * j + (uint64_t)lc->lane));
+    uint32_t word = get_u32(b->payload + 4 * (lc->word_base + (uint64_t)lc->lanes * j + (uint64_t)lc->lane));
     return (int)((word >> (31 - (pos & 31))) & 1u);
 }
 
@@ -634,13 +640,14 @@ static int decode_chunk(const or_blob *b, uint64_t c, uint8_t *out /* chunk-loca
         }
         if (pos != next) return OR_ECORRUPT;
     } else {
-        if (next < start || next > b->payload_words || (next - start) % OR_LANES) return OR_ECORRUPT;
-        lane_ctx lc = {start, 0, (next - start) / OR_LANES};
-        for (int l = 0; l < OR_LANES; l++) {
+        const uint64_t L = (uint64_t)b->lanes, step = OR_RUN * L;
+        if (next < start || next > b->payload_words || (next - start) % L) return OR_ECORRUPT;
+        lane_ctx lc = {start, 0, b->lanes, (next - start) / L};
+        for (int l = 0; l < b->lanes; l++) {
             lc.lane = l;
             uint64_t pos = 0;
             for (uint64_t p = 0; p < nc; p++) {
-                if ((p % 256) / OR_RUN != (uint64_t)l) continue;
+                if ((p % step) / OR_RUN != (uint64_t)l) continue;
                 int s = decode_symbol(b, bit_lane, &lc, &pos);
                 if (s < 0) return s;
                 out[p] = (uint8_t)s;

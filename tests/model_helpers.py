@@ -24,7 +24,7 @@ def encode_workload(entro, W: workloads.Workload, device="cuda", limit=None):
         w = workloads.weights(W, spec, device=device).cpu().numpy()
         t0 = time.perf_counter()
         blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
-                                 chunk_symbols=W.chunk_symbols(spec.cols))
+                                 chunk_symbols=W.chunk_symbols(spec.cols), lanes=W.lanes)
         t_enc += time.perf_counter() - t0
         del w
         dts.append(entro.upload(blob, device=device))

@@ -40,10 +40,11 @@ def _oracle_mode(m):
     return {0: oracle.MODE_AUTO, 1: oracle.MODE_UNSIGNED, 2: oracle.MODE_ASYM}[m]
 
 
-def check_decode(entro, w, bits, mode, max_len, fmt, chunk):
+def check_decode(entro, w, bits, mode, max_len, fmt, chunk, lanes=32):
     """Decode codes and bf16 on the GPU; compare with the oracle bit for bit."""
     q, s, z, scheme = oracle.quantize(w, bits, _oracle_mode(mode))
-    blob = entro.Blob.encode(w, bits=bits, quant_mode=mode, max_len=max_len, fmt=fmt, chunk_symbols=chunk)
+    blob = entro.Blob.encode(w, bits=bits, quant_mode=mode, max_len=max_len, fmt=fmt, chunk_symbols=chunk,
+                             lanes=lanes)
     dt = entro.upload(blob)
     st = _status()
     codes = dt.decode_codes(status=st)
@@ -99,6 +100,11 @@ SMALL = [
     ("laplace", 4, 2, 12, 1, 4096, 100, 100),
     ("skew", 8, 2, 16, 1, 512, 50, 50),
     ("zeros", 4, 0, 12, 1, 50, 3, 33),
+    ("laplace", 4, 2, 12, 2, -8192, 129, 64),  # 64 lanes (negative chunk marks them)
+    ("laplace", 4, 2, 12, 2, -1024, 7, 333),   # 64 lanes, ragged
+    ("t4", 8, 0, 16, 2, -2048, 100, 100),
+    ("skew", 8, 2, 20, 2, -1024, 64, 100),     # 64 lanes, slow path, refill per symbol
+    ("constant", 8, 0, 16, 2, -512, 5, 77),
 ]
 
 
@@ -107,7 +113,7 @@ SMALL = [
 def test_decode_small_cases(entro, case):
     kind, bits, mode, lmax, fmt, chunk, rows, cols = case
     w = workloads.small_tensor(kind, rows, cols, seed=rows * 7 + cols)
-    check_decode(entro, w, bits, mode, lmax, fmt, chunk)
+    check_decode(entro, w, bits, mode, lmax, fmt, abs(chunk), lanes=64 if chunk < 0 else 32)
 
 
 def test_empty_tensor(entro):
@@ -135,15 +141,16 @@ def test_lanes_workload_and_gemv(entro):
     check_gemv(entro, dt, q, s, z, batch=1)
 
 
+@pytest.mark.parametrize("lanes", [32, 64])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("batch", [1, 2, 3, 4, 16])
-@pytest.mark.parametrize("shape", [(96, 256), (40, 3072), (24, 14336)])
-def test_gemv_shapes_and_batches(entro, bits, batch, shape):
+@pytest.mark.parametrize("shape", [(96, 512), (40, 3072), (24, 14336)])
+def test_gemv_shapes_and_batches(entro, bits, batch, shape, lanes):
     rows, cols = shape
     w = workloads.small_tensor("t4" if bits == 8 else "laplace", rows, cols, seed=cols + bits)
     chunk = max(1, 8192 // cols) * cols
     q, s, z, _ = oracle.quantize(w, bits, oracle.MODE_ASYM)
-    blob = entro.Blob.encode(w, bits=bits, quant_mode=entro.QUANT_ASYM, chunk_symbols=chunk)
+    blob = entro.Blob.encode(w, bits=bits, quant_mode=entro.QUANT_ASYM, chunk_symbols=chunk, lanes=lanes)
     dt = entro.upload(blob)
     check_gemv(entro, dt, q, s, z, batch=batch, seed=batch)
 

@@ -54,6 +54,9 @@ CASES = [
     ("two_values", 4, oracle.MODE_ASYM, 12, 2, 256, 1, 1),
     ("t4", 4, oracle.MODE_ASYM, 4, 2, 512, 9, 100),
     ("t4", 8, oracle.MODE_ASYM, 16, 2, 256, 0, 16),
+    ("laplace", 4, oracle.MODE_ASYM, 12, 2, -1024, 7, 333),     # 64 lanes (negative chunk marks them)
+    ("t4", 8, oracle.MODE_AUTO, 16, 2, -6144, 20, 3072),
+    ("skew", 8, oracle.MODE_ASYM, 16, 2, -14336, 3, 14336),
 ]
 
 
@@ -61,17 +64,19 @@ CASES = [
                                              for c in CASES])
 def test_encoder_blob_identical_to_oracle(case):
     kind, bits, mode, lmax, fmt, chunk, rows, cols = case
+    lanes = 64 if chunk < 0 else 32
+    chunk = abs(chunk)
     w = workloads.small_tensor(kind, max(rows, 1), cols, seed=rows * 7 + cols)[:rows]
-    ref = oracle.encode(w, bits, mode, lmax, fmt, chunk)
+    ref = oracle.encode(w, bits, mode, lmax, fmt, chunk, lanes=lanes)
     for threads in (1, 3):
         blob = entro.Blob.encode(w, bits=bits, quant_mode=_MODE[mode], max_len=lmax, fmt=fmt,
-                                 chunk_symbols=chunk, threads=threads)
+                                 chunk_symbols=chunk, threads=threads, lanes=lanes)
         got = blob.to_bytes()
         assert len(got) == len(ref)
         assert got == ref
     info = blob.info()
     prm = oracle.params(ref)
-    for k in ("bits", "scheme", "max_len", "format", "rows", "cols", "n", "chunk_symbols", "n_chunks"):
+    for k in ("bits", "scheme", "max_len", "format", "rows", "cols", "n", "chunk_symbols", "n_chunks", "lanes"):
         assert info[k] == prm[k], k
     assert info["scale"] == prm["scale"] and info["zero"] == prm["zero"]
     assert (info["lengths"] == prm["lengths"]).all()
@@ -99,9 +104,9 @@ def test_encoder_identical_on_model_shaped_tensor():
     w = workloads.weights(W, spec).numpy()[:512]
     C = W.chunk_symbols(spec.cols)
     assert C == 6144
-    ref = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, C)
+    ref = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, C, lanes=W.lanes)
     got = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
-                            chunk_symbols=C).to_bytes()
+                            chunk_symbols=C, lanes=W.lanes).to_bytes()
     assert got == ref
 
 
@@ -121,7 +126,8 @@ def test_encoder_errors_match_oracle():
     assert e.value.code == entro.E_LIMIT
     with pytest.raises(oracle.OracleError):
         oracle.encode(many, 8, oracle.MODE_ASYM, 7, 2, 256)
-    for kw in ({"bits": 5}, {"fmt": 3}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25}):
+    for kw in ({"bits": 5}, {"fmt": 3}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25},
+               {"lanes": 48}, {"lanes": 64, "chunk_symbols": 768}):
         with pytest.raises(entro.EntroError):
             entro.Blob.encode(many, **kw)
 

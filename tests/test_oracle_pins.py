@@ -290,20 +290,22 @@ def _two_code_tensor(bits01):
     return np.where(np.asarray(bits01) == 1, 0.875, -1.0).astype(np.float32)
 
 
-def test_lane_layout_closed_form():
-    n = 2 * 256 + 40                                     # two full lane steps + a ragged tail
+@pytest.mark.parametrize("lanes", [32, 64])
+def test_lane_layout_closed_form(lanes):
+    step = 8 * lanes
+    n = 2 * step + 40                                    # two full lane steps + a ragged tail
     p = np.arange(n)
     b = ((p * 7) % 5 == 1).astype(np.uint8)
     blob = oracle.encode(_two_code_tensor(b).reshape(1, n), 4, oracle.MODE_ASYM, 12,
-                         oracle.FMT_LANES, 1024)
+                         oracle.FMT_LANES, 2048, lanes=lanes)
     prm = oracle.params(blob)
     assert prm["lengths"][0] == 1 and prm["lengths"][15] == 1 and prm["lengths"].sum() == 2
-    assert prm["n_chunks"] == 1 and prm["payload_words"] == 32
+    assert prm["lanes"] == lanes and prm["n_chunks"] == 1 and prm["payload_words"] == lanes
     idx = np.frombuffer(blob, np.uint64, 4, 384)
-    assert list(idx) == [0, 0, 32, n]
-    words = np.frombuffer(blob, np.uint32, 32, 384 + 32)
-    for lane in range(32):
-        seq = [int(b[q]) for t in range(3) for q in range(256 * t + 8 * lane, 256 * t + 8 * lane + 8)
+    assert list(idx) == [0, 0, lanes, n]
+    words = np.frombuffer(blob, np.uint32, lanes, 384 + 32)
+    for lane in range(lanes):
+        seq = [int(b[q]) for t in range(3) for q in range(step * t + 8 * lane, step * t + 8 * lane + 8)
                if q < n]
         expect = 0
         for i, bit in enumerate(seq):
@@ -346,14 +348,18 @@ CASES = [
     ("zeros", 4, oracle.MODE_AUTO, 12, oracle.FMT_SINGLE, 50, 3, 33),
     ("two_values", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, 256, 1, 1),
     ("t4", 4, oracle.MODE_ASYM, 4, oracle.FMT_LANES, 512, 9, 100),
+    ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, -1024, 7, 333),    # 64 lanes
+    ("t4", 8, oracle.MODE_AUTO, 16, oracle.FMT_LANES, -8192, 40, 300),        # 64 lanes
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}-b{c[1]}-f{c[4]}-c{c[5]}-{c[6]}x{c[7]}" for c in CASES])
 def test_encode_decode_identity(case):
     kind, bits, mode, lmax, fmt, chunk, rows, cols = case
+    lanes = 64 if chunk < 0 else 32                      # a negative chunk size marks the 64-lane cases
+    chunk = abs(chunk)
     w = workloads.small_tensor(kind, rows, cols, seed=rows + cols)
-    blob = oracle.encode(w, bits, mode, lmax, fmt, chunk)
+    blob = oracle.encode(w, bits, mode, lmax, fmt, chunk, lanes=lanes)
     q, s, z, scheme = oracle.quantize(w, bits, mode)
     assert (oracle.decode(blob) == q).all()
     prm = oracle.params(blob)

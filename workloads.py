@@ -68,6 +68,7 @@ class Workload:
     chunk_rule: str     # "fixed:<C>" or "rows" (whole rows, about 8192 symbols)
     tensors: Tuple[TensorSpec, ...]
     description: str
+    lanes: int = 32     # interleaved lanes per chunk of the lanes format
 
     def chunk_symbols(self, cols: int) -> int:
         if self.chunk_rule.startswith("fixed:"):
@@ -141,7 +142,7 @@ WORKLOADS = {
         "mistral_7b_u4", 3, 4, QUANT_ASYM, 12, FORMAT_LANES, "rows",
         _mistral_7b(),
         "Mistral-7B-shaped (32 layers), Laplace with std 0.02, asymmetric 4-bit, "
-        "row-aligned chunks, fused GEMV at batch 1"),
+        "row-aligned chunks, 64 lanes per chunk, fused GEMV at batch 1", 64),
     "phi3_mini_u8": Workload(
         "phi3_mini_u8", 4, 8, QUANT_AUTO, 16, FORMAT_LANES, "rows",
         _phi3_mini(4),
