@@ -351,12 +351,25 @@ def run_native(args, dist, rank, world, local_rank):
     return 0
 
 
+def _kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ("huffman_decode_canonical_b200/csrc/decode.cu", "huffman_decode_canonical_b200/csrc/blob_format.h"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def _traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary of the current kernels, if any."""
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
+    summary was taken on other kernel sources (profiles/traffic.json records their hash)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            return json.load(f).get(kernel)
+            t = json.load(f)
+        if t.get("source_sha256_16") != _kernel_source_hash():
+            return None
+        return t["kernels"].get(kernel)
     except Exception:
         return None
 
@@ -414,7 +427,7 @@ def run_model(args, dist, rank, world, local_rank):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     W = workloads.get(args.workload)
-    dts, infos, t_enc = encode_workload(entro, W, device=device)
+    dts, infos, t_enc = encode_workload(entro, W, device=device, limit=args.tensors or None)
     n = sum(i["n"] for i in infos)
     coded = sum(i["coded_bits"] for i in infos) / 8.0
     payload = sum(i["payload_bytes"] for i in infos)
@@ -457,8 +470,10 @@ def run_model(args, dist, rank, world, local_rank):
     peak, peak_kind = _peaks()
     alg = coded + index + out_bytes
     achieved = alg / (ms * 1e-3) / 1e9
+    partial = " (first %d tensors)" % len(dts) if args.tensors else ""
     line = {"metric": METRIC, "value": round(world / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
-            "unit": f"tok/s (batch {args.batch})" if gemv else "Gsym/s", "n_gpus": world, "steps": args.steps,
+            "unit": (f"tok/s (batch {args.batch})" if gemv else "Gsym/s") + partial, "n_gpus": world,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": f"u{W.bits} codes -> bf16" + (" x bf16 -> fp32" if gemv else ""),
             "data": "synthetic", "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
@@ -485,6 +500,7 @@ def main(argv=None):
                                                              "phi3_mini_u8"],
                     help="model-scale workloads time one grouped launch per step (not the default line)")
     ap.add_argument("--batch", type=int, default=1, help="GEMV batch for the model-scale GEMV workloads")
+    ap.add_argument("--tensors", type=int, default=0, help="model-scale workloads: only the first N tensors")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
