@@ -41,6 +41,7 @@ constexpr int kLutSize = 1 << kMaxLutBits;   // 4096 entries, 16 KB of shared me
 constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
 constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
+constexpr int kPackedFmaBatch = 4;  // from this padded batch on, the GEMV uses fp32 tables and f32x2 FMAs
 constexpr int kSlackRows = 2;                 // staging rows past a chunk's longest lane (read-ahead)
 
 enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
@@ -160,6 +161,25 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
     return acc;
 }
 
+// Two fp32 FMAs in one instruction: (a.x*b.x + c.x, a.y*b.y + c.y), each
+// rounded once (fma.rn.f32x2).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%1, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "mov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+        : "=l"(r)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
+}
+
+// bf16 pair (low half first) -> two fp32 values (exact)
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
 // Canonical decode of a code longer than the table's 12 bits: the code length
 // is the first l with (top max_len bits) < limit[l].  Returns length | symbol
 // << 8, or a 1-bit entry after flagging corruption.
@@ -180,6 +200,7 @@ struct Smem {
     uint32_t *lut;    // decode table (multi-symbol for the lanes kernel)
     uint32_t *vtab;   // bf16 value of each code, low half
     uint32_t *vpair;  // 4-bit: bf16 values of the two codes of a byte
+    float *wtab;      // GEMV: fp32 weight of each code (8-bit), or of both codes of a byte (4-bit, pairs)
     uint32_t *slim;
     int32_t *soffs;
     uint8_t *ssyms;
@@ -197,10 +218,12 @@ struct SmemOffsets {
 };
 
 // shared-memory carve-up; identical on host (sizing) and device
-// stage_words: 32-bit words of one staging buffer (rows x lanes)
-__host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_words, int out_words) {
+// stage_words: 32-bit words of one staging buffer (rows x lanes); wtab: the
+// fp32 weight table of the batched GEMV
+__host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_words, int out_words,
+                                                   bool wtab = false) {
     SmemOffsets o;
-    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
+    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256 + (wtab ? 256 * 8 : 0);
     p = align_up(p, 16);
     o.x = p;
     p += (size_t)x_elems * 2;
@@ -217,8 +240,9 @@ __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems,
     return o;
 }
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_words, int out_words) {
-    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words);
+__device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_words, int out_words,
+                                      bool wtab = false) {
+    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words, wtab);
     Smem s;
     s.lut = reinterpret_cast<uint32_t *>(base);
     s.vtab = s.lut + kLutSize;
@@ -226,6 +250,7 @@ __device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elem
     s.slim = s.vpair + 256;
     s.soffs = reinterpret_cast<int32_t *>(s.slim + 32);
     s.ssyms = reinterpret_cast<uint8_t *>(s.soffs + 32);
+    s.wtab = reinterpret_cast<float *>(s.ssyms + 256);
     s.xs = reinterpret_cast<__nv_bfloat16 *>(base + o.x);
     s.tbar = reinterpret_cast<uint64_t *>(base + o.bars);
     s.bars = s.tbar + 2;
@@ -259,7 +284,7 @@ __device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int
     if (xbytes) bulk_copy_g2s(s.xs, g.x, xbytes, s.tbar);
 }
 
-template <int OUT, bool SLOW>
+template <int OUT, bool SLOW, bool WTAB = false>
 __device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphase) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const DevTensor &d = g.d;
@@ -270,6 +295,14 @@ __device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphas
             if (d.bits == 4)
                 s.vpair[q] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
                              (dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
+            if (WTAB) {
+                if (d.bits == 4) {
+                    s.wtab[2 * q] = __uint_as_float(dequant_bf16_bits(q & 15, d.zero, d.scale) << 16);
+                    s.wtab[2 * q + 1] = __uint_as_float(dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
+                } else {
+                    s.wtab[q] = __uint_as_float(v << 16);
+                }
+            }
         }
     }
     const bool ok = mbar_wait(s.tbar, tphase & 1);
@@ -434,7 +467,7 @@ __device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int
 // thread `lane` serves the format lanes lane, lane + 32, ...
 template <int BITS, int OUT, int BPAD, int LANES>
 __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
-                                          int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD]) {
+                                          int tb, int te, int batch, int x_in_smem, float2 (&acc)[BPAD]) {
     constexpr int LPT = LANES / kLanes;
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
@@ -453,28 +486,64 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
                 dst[LANES * t + l] = values8<BITS>(s, ost, LANES * (t & (kRing - 1)) + l);
             }
     } else {
-        // fused GEMV: run t covers columns 8*LANES*(t % spr) + 8*l .. +7 of row t / spr
+        // fused GEMV: run t covers columns 8*LANES*(t % spr) + 8*l .. +7 of row t / spr.
+        // Each lane keeps two fp32 partial sums per batch row (even / odd column of
+        // each pair) and adds them at the row end, then the warp reduces.  Small
+        // batches multiply the bf16 weights and activations directly
+        // (fma.rn.f32.bf16); from kPackedFmaBatch on, the per-code fp32 weights
+        // come from a table and two FMAs issue as one (fma.rn.f32x2).
+        constexpr bool kPacked = BPAD >= kPackedFmaBatch;
         const int K = static_cast<int>(d.cols);
         const int spr = K / (kRun * LANES);
         const long long row0 = first / K;
         const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
+        const float2 *wp = reinterpret_cast<const float2 *>(s.wtab);
         for (int t = tb; t < te; t++) {
             const int st = t % spr;
 #pragma unroll
             for (int k = 0; k < LPT; k++) {
                 const int l = lane + kLanes * k;
-                const uint4 wv = values8<BITS>(s, ost, LANES * (t & (kRing - 1)) + l);
+                const int slot = LANES * (t & (kRing - 1)) + l;
                 const int xo = st * LANES + l;  // uint4 index within one x row
+                if (kPacked) {
+                    float2 w0, w1, w2, w3;  // weights of codes (0,1) (2,3) (4,5) (6,7) of the run
+                    if (BITS == 4) {
+                        const uint32_t c = ost[slot];
+                        w0 = wp[c & 0xFFu];
+                        w1 = wp[(c >> 8) & 0xFFu];
+                        w2 = wp[(c >> 16) & 0xFFu];
+                        w3 = wp[c >> 24];
+                    } else {
+                        const uint2 c = reinterpret_cast<const uint2 *>(ost)[slot];
+                        w0 = make_float2(s.wtab[c.x & 0xFFu], s.wtab[(c.x >> 8) & 0xFFu]);
+                        w1 = make_float2(s.wtab[(c.x >> 16) & 0xFFu], s.wtab[c.x >> 24]);
+                        w2 = make_float2(s.wtab[c.y & 0xFFu], s.wtab[(c.y >> 8) & 0xFFu]);
+                        w3 = make_float2(s.wtab[(c.y >> 16) & 0xFFu], s.wtab[c.y >> 24]);
+                    }
 #pragma unroll
-                for (int b = 0; b < BPAD; b++) {
-                    if (b < batch) {
-                        const int xi = b * (K >> 3) + xo;
-                        const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
-                        acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
-                        acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
-                        acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
-                        acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
+                    for (int b = 0; b < BPAD; b++) {
+                        if (b < batch) {
+                            const int xi = b * (K >> 3) + xo;
+                            const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                            acc[b] = ffma2(w0, bf16x2_to_float2(xv.x), acc[b]);
+                            acc[b] = ffma2(w1, bf16x2_to_float2(xv.y), acc[b]);
+                            acc[b] = ffma2(w2, bf16x2_to_float2(xv.z), acc[b]);
+                            acc[b] = ffma2(w3, bf16x2_to_float2(xv.w), acc[b]);
+                        }
+                    }
+                } else {
+                    const uint4 wv = values8<BITS>(s, ost, slot);
+#pragma unroll
+                    for (int b = 0; b < BPAD; b++) {
+                        if (b < batch) {
+                            const int xi = b * (K >> 3) + xo;
+                            const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                            acc[b].x = fma2_bf16(wv.x, xv.x, acc[b].x);
+                            acc[b].x = fma2_bf16(wv.y, xv.y, acc[b].x);
+                            acc[b].x = fma2_bf16(wv.z, xv.z, acc[b].x);
+                            acc[b].x = fma2_bf16(wv.w, xv.w, acc[b].x);
+                        }
                     }
                 }
             }
@@ -483,10 +552,10 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
 #pragma unroll
                 for (int b = 0; b < BPAD; b++) {
                     if (b < batch) {
-                        const float v = warp_sum(acc[b]);
+                        const float v = warp_sum(acc[b].x + acc[b].y);
                         if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row] = v;
                     }
-                    acc[b] = 0.f;
+                    acc[b] = make_float2(0.f, 0.f);
                 }
             }
         }
@@ -566,9 +635,9 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
     bool ok = true;
     if (nc == d.chunk_symbols) {
         const int runs = nc / kStep;
-        float acc[BPAD];
+        float2 acc[BPAD];
 #pragma unroll
-        for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
+        for (int b = 0; b < BPAD; b++) acc[b] = make_float2(0.f, 0.f);
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
             bool more = true;
@@ -664,7 +733,8 @@ template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words);
+    constexpr bool kWtab = OUT == OUT_GEMV && BPAD >= kPackedFmaBatch;
+    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words, kWtab);
     uint64_t *bar = s.bars + 2 * warp;
     const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
     uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
@@ -720,7 +790,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             pend0 = c < cb;
             pend1 = c + warps < cb;
         }
-        const bool tables_ok = finish_tables<OUT, SLOW>(g, s, tphase);
+        const bool tables_ok = finish_tables<OUT, SLOW, kWtab>(g, s, tphase);
         tphase++;
         if (!tables_ok) {
             set_status(a.status, ENTRO_E_TIMEOUT);
@@ -1231,7 +1301,8 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     int warps = (int)std::min<long long>(kMaxWarps, std::max<long long>(1, (chunks + di.sms - 1) / di.sms));
     SmemOffsets so;
     for (;;) {
-        so = smem_layout(warps, x_elems, stage_rows * lanes, out_words);
+        so = smem_layout(warps, x_elems, stage_rows * lanes, out_words,
+                         out_kind == OUT_GEMV && bpad >= kPackedFmaBatch);
         if ((long long)so.total <= di.smem_optin) break;
         if (warps > 1) warps--;
         else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
