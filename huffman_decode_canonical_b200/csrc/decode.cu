@@ -17,10 +17,14 @@
 //     high half of the table entry, or feeds the bf16 weights straight into an
 //     fp32 GEMV with a warp-shuffle reduction per row (weights never touch
 //     memory).
+//   * gemv_mma kernel: the fused GEMV for batches of 3 to 16 activation rows.
+//     The warps of a CTA decode consecutive rows in lockstep and multiply the
+//     decoded weights with warp-level tensor-core MMAs (mma.sync m16n8k16,
+//     bf16 in, fp32 out), reading the B operand from the warps' code rings.
 //   * single kernel: the one-bitstream-per-chunk format, one thread per chunk.
-// No tensor cores: the work is bit manipulation and streaming, not a dense
-// contraction.  Errors are reported through a status word, never by trapping;
-// every wait on a copy is bounded.
+// The decode itself is bit manipulation and streaming, not a dense
+// contraction; only the batched GEMV is MMA-shaped.  Errors are reported
+// through a status word, never by trapping; every wait on a copy is bounded.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,7 +45,6 @@ constexpr int kLutSize = 1 << kMaxLutBits;   // 4096 entries, 16 KB of shared me
 constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
 constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
-constexpr int kPackedFmaBatch = 4;  // from this padded batch on, the GEMV uses fp32 tables and f32x2 FMAs
 constexpr int kSlackRows = 2;                 // staging rows past a chunk's longest lane (read-ahead)
 
 enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
@@ -161,25 +164,6 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
     return acc;
 }
 
-// Two fp32 FMAs in one instruction: (a.x*b.x + c.x, a.y*b.y + c.y), each
-// rounded once (fma.rn.f32x2).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    unsigned long long r;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%1, %2};\n\t"
-        "mov.b64 rb, {%3, %4};\n\t"
-        "mov.b64 rc, {%5, %6};\n\t"
-        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
-        : "=l"(r)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return make_float2(__uint_as_float(static_cast<uint32_t>(r)), __uint_as_float(static_cast<uint32_t>(r >> 32)));
-}
-
-// bf16 pair (low half first) -> two fp32 values (exact)
-__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
-    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
-}
-
 // Canonical decode of a code longer than the table's 12 bits: the code length
 // is the first l with (top max_len bits) < limit[l].  Returns length | symbol
 // << 8, or a 1-bit entry after flagging corruption.
@@ -200,7 +184,6 @@ struct Smem {
     uint32_t *lut;    // decode table (multi-symbol for the lanes kernel)
     uint32_t *vtab;   // bf16 value of each code, low half
     uint32_t *vpair;  // 4-bit: bf16 values of the two codes of a byte
-    float *wtab;      // GEMV: fp32 weight of each code (8-bit), or of both codes of a byte (4-bit, pairs)
     uint32_t *slim;
     int32_t *soffs;
     uint8_t *ssyms;
@@ -209,21 +192,22 @@ struct Smem {
     uint64_t *bars;
     uint32_t *stage;
     uint32_t *ostage;
+    float *red;       // tensor-core GEMV: per-warp partial sums for the cross-warp row reduction
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct SmemOffsets {
-    size_t x, bars, stage, ostage, total;
+    size_t x, bars, stage, ostage, red, total;
 };
 
 // shared-memory carve-up; identical on host (sizing) and device
-// stage_words: 32-bit words of one staging buffer (rows x lanes); wtab: the
-// fp32 weight table of the batched GEMV
+// stage_words: 32-bit words of one staging buffer (rows x lanes); red_bytes:
+// the cross-warp partial sums of the tensor-core GEMV
 __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_words, int out_words,
-                                                   bool wtab = false) {
+                                                   size_t red_bytes = 0) {
     SmemOffsets o;
-    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256 + (wtab ? 256 * 8 : 0);
+    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
     p = align_up(p, 16);
     o.x = p;
     p += (size_t)x_elems * 2;
@@ -236,13 +220,16 @@ __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems,
     p = align_up(p, 16);
     o.ostage = p;
     p += (size_t)warps * (size_t)out_words * 4;
+    p = align_up(p, 16);
+    o.red = p;
+    p += red_bytes;
     o.total = p;
     return o;
 }
 
 __device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_words, int out_words,
-                                      bool wtab = false) {
-    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words, wtab);
+                                      size_t red_bytes = 0) {
+    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words, red_bytes);
     Smem s;
     s.lut = reinterpret_cast<uint32_t *>(base);
     s.vtab = s.lut + kLutSize;
@@ -250,12 +237,12 @@ __device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elem
     s.slim = s.vpair + 256;
     s.soffs = reinterpret_cast<int32_t *>(s.slim + 32);
     s.ssyms = reinterpret_cast<uint8_t *>(s.soffs + 32);
-    s.wtab = reinterpret_cast<float *>(s.ssyms + 256);
     s.xs = reinterpret_cast<__nv_bfloat16 *>(base + o.x);
     s.tbar = reinterpret_cast<uint64_t *>(base + o.bars);
     s.bars = s.tbar + 2;
     s.stage = reinterpret_cast<uint32_t *>(base + o.stage);
     s.ostage = reinterpret_cast<uint32_t *>(base + o.ostage);
+    s.red = reinterpret_cast<float *>(base + o.red);
     return s;
 }
 
@@ -284,7 +271,7 @@ __device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int
     if (xbytes) bulk_copy_g2s(s.xs, g.x, xbytes, s.tbar);
 }
 
-template <int OUT, bool SLOW, bool WTAB = false>
+template <int OUT, bool SLOW>
 __device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphase) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const DevTensor &d = g.d;
@@ -295,14 +282,6 @@ __device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphas
             if (d.bits == 4)
                 s.vpair[q] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
                              (dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
-            if (WTAB) {
-                if (d.bits == 4) {
-                    s.wtab[2 * q] = __uint_as_float(dequant_bf16_bits(q & 15, d.zero, d.scale) << 16);
-                    s.wtab[2 * q + 1] = __uint_as_float(dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
-                } else {
-                    s.wtab[q] = __uint_as_float(v << 16);
-                }
-            }
         }
     }
     const bool ok = mbar_wait(s.tbar, tphase & 1);
@@ -467,7 +446,7 @@ __device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int
 // thread `lane` serves the format lanes lane, lane + 32, ...
 template <int BITS, int OUT, int BPAD, int LANES>
 __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
-                                          int tb, int te, int batch, int x_in_smem, float2 (&acc)[BPAD]) {
+                                          int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD]) {
     constexpr int LPT = LANES / kLanes;
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
@@ -486,19 +465,15 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
                 dst[LANES * t + l] = values8<BITS>(s, ost, LANES * (t & (kRing - 1)) + l);
             }
     } else {
-        // fused GEMV: run t covers columns 8*LANES*(t % spr) + 8*l .. +7 of row t / spr.
-        // Each lane keeps two fp32 partial sums per batch row (even / odd column of
-        // each pair) and adds them at the row end, then the warp reduces.  Small
-        // batches multiply the bf16 weights and activations directly
-        // (fma.rn.f32.bf16); from kPackedFmaBatch on, the per-code fp32 weights
-        // come from a table and two FMAs issue as one (fma.rn.f32x2).
-        constexpr bool kPacked = BPAD >= kPackedFmaBatch;
+        // fused GEMV (batch 1 and 2): run t covers columns 8*LANES*(t % spr) + 8*l .. +7
+        // of row t / spr.  Each lane keeps one fp32 sum per batch row, fed by
+        // mixed-precision FMAs of the bf16 weights and activations
+        // (fma.rn.f32.bf16), and the warp reduces at the row end.
         const int K = static_cast<int>(d.cols);
         const int spr = K / (kRun * LANES);
         const long long row0 = first / K;
         const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
-        const float2 *wp = reinterpret_cast<const float2 *>(s.wtab);
         for (int t = tb; t < te; t++) {
             const int st = t % spr;
 #pragma unroll
@@ -506,44 +481,16 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
                 const int l = lane + kLanes * k;
                 const int slot = LANES * (t & (kRing - 1)) + l;
                 const int xo = st * LANES + l;  // uint4 index within one x row
-                if (kPacked) {
-                    float2 w0, w1, w2, w3;  // weights of codes (0,1) (2,3) (4,5) (6,7) of the run
-                    if (BITS == 4) {
-                        const uint32_t c = ost[slot];
-                        w0 = wp[c & 0xFFu];
-                        w1 = wp[(c >> 8) & 0xFFu];
-                        w2 = wp[(c >> 16) & 0xFFu];
-                        w3 = wp[c >> 24];
-                    } else {
-                        const uint2 c = reinterpret_cast<const uint2 *>(ost)[slot];
-                        w0 = make_float2(s.wtab[c.x & 0xFFu], s.wtab[(c.x >> 8) & 0xFFu]);
-                        w1 = make_float2(s.wtab[(c.x >> 16) & 0xFFu], s.wtab[c.x >> 24]);
-                        w2 = make_float2(s.wtab[c.y & 0xFFu], s.wtab[(c.y >> 8) & 0xFFu]);
-                        w3 = make_float2(s.wtab[(c.y >> 16) & 0xFFu], s.wtab[c.y >> 24]);
-                    }
+                const uint4 wv = values8<BITS>(s, ost, slot);
 #pragma unroll
-                    for (int b = 0; b < BPAD; b++) {
-                        if (b < batch) {
-                            const int xi = b * (K >> 3) + xo;
-                            const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
-                            acc[b] = ffma2(w0, bf16x2_to_float2(xv.x), acc[b]);
-                            acc[b] = ffma2(w1, bf16x2_to_float2(xv.y), acc[b]);
-                            acc[b] = ffma2(w2, bf16x2_to_float2(xv.z), acc[b]);
-                            acc[b] = ffma2(w3, bf16x2_to_float2(xv.w), acc[b]);
-                        }
-                    }
-                } else {
-                    const uint4 wv = values8<BITS>(s, ost, slot);
-#pragma unroll
-                    for (int b = 0; b < BPAD; b++) {
-                        if (b < batch) {
-                            const int xi = b * (K >> 3) + xo;
-                            const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
-                            acc[b].x = fma2_bf16(wv.x, xv.x, acc[b].x);
-                            acc[b].x = fma2_bf16(wv.y, xv.y, acc[b].x);
-                            acc[b].x = fma2_bf16(wv.z, xv.z, acc[b].x);
-                            acc[b].x = fma2_bf16(wv.w, xv.w, acc[b].x);
-                        }
+                for (int b = 0; b < BPAD; b++) {
+                    if (b < batch) {
+                        const int xi = b * (K >> 3) + xo;
+                        const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                        acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
+                        acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
+                        acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
+                        acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
                     }
                 }
             }
@@ -552,10 +499,10 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
 #pragma unroll
                 for (int b = 0; b < BPAD; b++) {
                     if (b < batch) {
-                        const float v = warp_sum(acc[b].x + acc[b].y);
+                        const float v = warp_sum(acc[b]);
                         if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row] = v;
                     }
-                    acc[b] = make_float2(0.f, 0.f);
+                    acc[b] = 0.f;
                 }
             }
         }
@@ -604,6 +551,29 @@ __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, 
     }
 }
 
+// Advance every format lane the thread serves to run te (whole runs).  A lane
+// may write the first codes of run te before it stops: one slot past the block.
+template <int BITS, bool SLOW, int LANES, int LPT>
+__device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[LPT], const Smem &s, int te,
+                                          int max_len, bool refill_each, int32_t *status) {
+    bool more = true;
+    while (more) {
+        more = false;
+#pragma unroll
+        for (int k = 0; k < LPT; k++) {
+            if (ld[k].t < te) {
+                ld[k].refill();
+                ld[k].lookup(s, max_len, status);
+                ld[k].emit();
+                if (SLOW && refill_each) ld[k].refill();
+                ld[k].lookup(s, max_len, status);
+                ld[k].emit();
+                more = more || ld[k].t < te;
+            }
+        }
+    }
+}
+
 // Decode chunk c of entry g from its staged words.  Thread `lane` decodes the
 // format lanes lane, lane + 32, ... as independent interleaved streams.  Whole
 // chunks are emitted every kEmitBlock runs, so the stores of one block drain
@@ -633,29 +603,16 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
         read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kSlackRows);
     }
     bool ok = true;
-    if (nc == d.chunk_symbols) {
+    if (nc % kStep == 0) {
+        // whole runs in every lane: every chunk but a short last one, and any
+        // last chunk of whole rows (the GEMV's chunks always are)
         const int runs = nc / kStep;
-        float2 acc[BPAD];
+        float acc[BPAD];
 #pragma unroll
-        for (int b = 0; b < BPAD; b++) acc[b] = make_float2(0.f, 0.f);
+        for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
-            bool more = true;
-            while (more) {
-                more = false;
-#pragma unroll
-                for (int k = 0; k < LPT; k++) {
-                    if (ld[k].t < te) {
-                        ld[k].refill();
-                        ld[k].lookup(s, d.max_len, status);
-                        ld[k].emit();
-                        if (SLOW && refill_each) ld[k].refill();
-                        ld[k].lookup(s, d.max_len, status);
-                        ld[k].emit();
-                        more = more || ld[k].t < te;
-                    }
-                }
-            }
+            decode_to(ld, s, te, d.max_len, refill_each, status);
             __syncwarp();
             emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
             __syncwarp();  // the ring slots just read are rewritten by the next block
@@ -733,8 +690,7 @@ template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr bool kWtab = OUT == OUT_GEMV && BPAD >= kPackedFmaBatch;
-    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words, kWtab);
+    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words);
     uint64_t *bar = s.bars + 2 * warp;
     const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
     uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
@@ -790,7 +746,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             pend0 = c < cb;
             pend1 = c + warps < cb;
         }
-        const bool tables_ok = finish_tables<OUT, SLOW, kWtab>(g, s, tphase);
+        const bool tables_ok = finish_tables<OUT, SLOW>(g, s, tphase);
         tphase++;
         if (!tables_ok) {
             set_status(a.status, ENTRO_E_TIMEOUT);
@@ -829,6 +785,236 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             if (pend1) mbar_wait(bar + 1, phase1 & 1);
         }
         __syncthreads();  // every warp done with this entry's tables
+    }
+}
+
+// ------------------------------------------------------------------ batched GEMV on the tensor cores
+//
+// From batch 3 on, 3 to 16 products per decoded weight made the CUDA-core GEMV
+// the bottleneck, and every warp streamed its own columns of x from L2.  This
+// kernel decodes the same codes the same way, but the warps of a CTA work in
+// lockstep on consecutive chunks (= consecutive rows, since its tensors have
+// whole-row chunks) and multiply with mma.sync m16n8k16 (bf16 operands, fp32
+// accumulation):
+//   A = x[16 batch rows (zero-padded), 16 columns]      straight from global
+//   B = W^T[16 columns, 8 rows of the CTA]              from the warps' run rings
+//   D = y partials [16 batch rows, 8 rows]              registers, per warp
+// Each lockstep block covers E runs of every chunk (E divides the runs of a
+// row, E + 1 <= kRing); after a CTA barrier the block's columns are split
+// among the warps in groups of 32 (4 format lanes x 8 weights).  The k order
+// inside an MMA is permuted so that each thread's B registers are the 8
+// weights of one ring slot and its A registers one 16-byte load of x:
+//   k-step 0: k = 2j + e <-> column 8j + e, k = 2j + 8 + e <-> column 8j + 2 + e
+//   k-step 1: the same with columns 8j + 4 + e and 8j + 6 + e  (j = lane % 4)
+// The partial sums of a row are added across warps in warp order at the row's
+// end (fixed order: the result does not depend on timing).  The tensor pipe is
+// not the bound: the MMAs replace 16 FMAs per weight with 1/8 of an MMA issue,
+// and x is read once per CTA instead of once per warp.
+
+constexpr int kTileMaxBlock = kRing - 1;  // a block plus the slot a lane may write past it fit the ring
+constexpr int kTileBatch = 4;             // padded batch from which the tensor-core GEMV runs
+
+// Runs per lockstep block: the largest divisor of the runs per row that fits the ring.
+__host__ __device__ inline int tile_block_runs(long long cols, int lanes) {
+    const long long spr = cols / (kRun * lanes);
+    for (int e = kTileMaxBlock; e > 1; e--)
+        if (spr % e == 0) return e;
+    return 1;
+}
+
+// Ring words per warp for the tensor-core GEMV: the ring plus a pad of `bits`
+// words, which puts the rings of consecutive warps 4 (4-bit) or 8 (8-bit)
+// banks apart, so the B-fragment loads of 8 rows hit 32 different banks (per
+// half warp for the 8-byte loads of 8-bit codes).
+__host__ __device__ inline int tile_ring_words(int bits, int lanes) { return kRing * lanes * bits / 4 + bits; }
+
+__device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int BITS, bool SLOW, int LANES>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __grid_constant__ LaunchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    constexpr int LPT = LANES / kLanes;
+    constexpr int kGroupsPerRun = LANES / 4;  // 32-column groups in one run step of a chunk
+    const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
+    const Smem s = carve(smem_raw, warps, 0, a.stage_rows * LANES, a.out_words, static_cast<size_t>(warps) * 2 * 32 * 16);
+    uint64_t *bar = s.bars + 2 * warp;
+    const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
+    uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
+    uint32_t *ost = s.ostage + static_cast<size_t>(warp) * a.out_words;
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
+    }
+    if (threadIdx.x == 0) mbar_init(s.tbar, 1);
+    fence_mbar_init();
+    __syncthreads();
+
+    const long long s0 = a.total_syms * blockIdx.x / gridDim.x;
+    const long long s1 = a.total_syms * (blockIdx.x + 1) / gridDim.x;
+    int ei = 0;
+    {
+        int lo = 0, hi = a.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (entry_at(a, mid).sym_begin <= s0) lo = mid;
+            else hi = mid - 1;
+        }
+        ei = lo;
+    }
+    const int batch = a.batch;
+    uint32_t phase0 = 0, phase1 = 0, tphase = 0;
+    bool dead = false;  // this warp gave up on a copy: it decodes nothing more but keeps every barrier
+    for (; ei < a.count; ei++) {
+        const GroupEntry &g = entry_at(a, ei);
+        if (g.sym_begin >= s1) break;
+        const DevTensor &d = g.d;
+        const long long C = d.chunk_symbols;
+        long long ca = s0 > g.sym_begin ? (s0 - g.sym_begin + C - 1) / C : 0;
+        long long cb = (s1 - g.sym_begin + C - 1) / C;
+        if (cb > d.n_chunks) cb = d.n_chunks;
+        if (ca >= cb) continue;
+        issue_tables<OUT_GEMV, SLOW>(g, s, true, batch, 0);
+        bool pend0 = false, pend1 = false;
+        if (!dead) {
+            const long long c = ca + warp;
+            const long long cq = (lane < 2) ? c : c + warps;
+            uint64_t iv = 0;
+            if (lane < 4 && cq < cb) iv = d.index[2 * cq + 2 * (lane & 1)];
+            const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
+            const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
+            if (lane == 0) {
+                if (c < cb) issue_words(d, st0, nx0, stage, bar, a.stage_rows, LANES);
+                if (c + warps < cb) issue_words(d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES);
+            }
+            pend0 = c < cb;
+            pend1 = c + warps < cb;
+        }
+        const bool tables_ok = finish_tables<OUT_GEMV, SLOW>(g, s, tphase);
+        tphase++;
+        if (!tables_ok) {
+            set_status(a.status, ENTRO_E_TIMEOUT);
+            dead = true;
+        }
+        const int K = static_cast<int>(d.cols);
+        const int spr = K / (kRun * LANES);                      // runs per row
+        const int E = tile_block_runs(K, LANES);
+        const int runs = static_cast<int>(C / (kRun * LANES));  // runs per chunk (whole rows)
+        const int rows_per_chunk = static_cast<int>(C / K);
+        const int groups = E * kGroupsPerRun;
+        const bool refill_each = SLOW && d.max_len > 16;
+        const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
+        const int xrow = K >> 3;  // uint4 per row of x
+        int k = 0;
+        for (long long c0 = ca; c0 < cb; c0 += warps, k++) {
+            const long long c = c0 + warp;
+            const int nrows = static_cast<int>(cb - c0 < warps ? cb - c0 : warps);  // chunks (rows of W) in this group
+            // a short last chunk holds whole rows, hence whole runs: it stops decoding early and its
+            // missing rows are not written
+            const int my_runs = c == d.n_chunks - 1 ? static_cast<int>((d.n - c * C) / (kRun * LANES)) : runs;
+            const int b = k & 1;
+            bool active = c < cb && !dead;
+            if (active) {
+                const uint32_t phase = b ? phase1 : phase0;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar + b, phase & 1))) {
+                    set_status(a.status, ENTRO_E_TIMEOUT);
+                    dead = true;
+                    active = false;
+                } else {
+                    if (b) { phase1++; pend1 = false; }
+                    else { phase0++; pend0 = false; }
+                    if (!chunk_words_ok(d, c, a.stage_rows, LANES)) {
+                        set_status(a.status, ENTRO_E_CORRUPT);
+                        active = false;
+                    }
+                }
+            }
+            const uint32_t *buf = stage + b * buf_words;
+            LaneDecoder<BITS, SLOW, LANES> ld[LPT];
+            uint32_t read_limit[LPT];
+            if (active) {
+                const int words = static_cast<int>((d.index[2 * c + 2] - d.index[2 * c]) / LANES);
+#pragma unroll
+                for (int q = 0; q < LPT; q++) {
+                    const int l = lane + kLanes * q;
+                    ld[q].init(s, buf + l, ost + (BITS == 4 ? l : 2 * l), a.stage_rows - 1);
+                    read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kSlackRows);
+                }
+            }
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int tb = 0; tb < runs; tb += E) {
+                const int te = tb + E;
+                if (active && tb < my_runs) decode_to(ld, s, te, d.max_len, refill_each, a.status);
+                __syncthreads();  // the block's runs of every row are in the rings
+                const int col0 = (tb % spr) * (kRun * LANES);
+                for (int q = warp; q < groups; q += warps) {
+                    const int t = tb + q / kGroupsPerRun;
+                    const int slot = LANES * (t & (kRing - 1)) + 4 * (q % kGroupsPerRun) + tig;
+                    const int xo = ((col0 + 32 * q) >> 3) + tig;
+                    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 xa = gid < batch ? __ldg(xg + gid * xrow + xo) : z4;
+                    const uint4 xb = gid + 8 < batch ? __ldg(xg + (gid + 8) * xrow + xo) : z4;
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++) {
+                        if (8 * nt >= nrows) break;
+                        const int r = 8 * nt + gid;
+                        const uint4 w = r < nrows ? values8<BITS>(s, s.ostage + static_cast<size_t>(r) * a.out_words, slot)
+                                                  : z4;
+                        mma_16816_bf16(acc[nt], xa.x, xb.x, xa.y, xb.y, w.x, w.y);
+                        mma_16816_bf16(acc[nt], xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                    }
+                }
+                if (te % spr == 0) {
+                    // row end: partial sums of every warp, added in warp order
+                    float4 *rd = reinterpret_cast<float4 *>(s.red);
+                    rd[(2 * warp) * 32 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+                    rd[(2 * warp + 1) * 32 + lane] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+                    __syncthreads();
+                    const long long row_in_chunk = tb / spr;
+                    for (int o = threadIdx.x; o < 256; o += blockDim.x) {
+                        const int bb = o >> 4, r = o & 15;
+                        const long long row = (c0 + r) * rows_per_chunk + row_in_chunk;
+                        if (bb < batch && r < nrows && row < d.rows) {
+                            const int nt = r >> 3, n = r & 7;
+                            const int src = ((4 * (bb & 7) + (n >> 1)) << 2) + ((bb >> 3) << 1) + (n & 1);
+                            float v = 0.f;
+                            for (int w = 0; w < warps; w++) v += s.red[(2 * w + nt) * 128 + src];
+                            g.y[static_cast<long long>(bb) * d.rows + row] = v;
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                        for (int i = 0; i < 4; i++) acc[nt][i] = 0.f;
+                }
+                __syncthreads();  // every warp is done reading the rings before they are rewritten
+            }
+            if (active) {
+                bool ok = true;
+#pragma unroll
+                for (int q = 0; q < LPT; q++) ok = ok && ld[q].bufa <= read_limit[q];
+                if (!ok) set_status(a.status, ENTRO_E_OVERRUN);
+            }
+            if (c < cb && !dead && c + 2 * warps < cb) {
+                if (lane == 0) {
+                    fence_proxy_async();
+                    issue_chunk(d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES);
+                }
+                if (b) pend1 = true;
+                else pend0 = true;
+            }
+        }
+        if (dead) {
+            if (pend0) mbar_wait(bar, phase0 & 1);
+            if (pend1) mbar_wait(bar + 1, phase1 & 1);
+        }
+        __syncthreads();
     }
 }
 
@@ -1184,9 +1370,7 @@ static LanesFn pick_bpad(int bpad) {
     switch (bpad) {
         case 1: return lanes_kernel<BITS, OUT, SLOW, 1, LANES>;
         case 2: return lanes_kernel<BITS, OUT, SLOW, 2, LANES>;
-        case 4: return lanes_kernel<BITS, OUT, SLOW, 4, LANES>;
-        case 8: return lanes_kernel<BITS, OUT, SLOW, 8, LANES>;
-        default: return lanes_kernel<BITS, OUT, SLOW, 16, LANES>;
+        default: return nullptr;  // padded batch 4 to 16: gemv_mma_kernel
     }
 }
 
@@ -1200,6 +1384,20 @@ static LanesFn pick_out(int out, bool slow, int bpad) {
 static LanesFn pick_lanes(int bits, int out, bool slow, int bpad, int lanes) {
     if (bits == 4) return lanes == 64 ? pick_out<4, 64>(out, slow, bpad) : pick_out<4, 32>(out, slow, bpad);
     return lanes == 64 ? pick_out<8, 64>(out, slow, bpad) : pick_out<8, 32>(out, slow, bpad);
+}
+
+static LanesFn pick_mma(int bits, bool slow, int lanes) {
+    if (bits == 4) {
+        if (lanes == 64) return slow ? gemv_mma_kernel<4, true, 64> : gemv_mma_kernel<4, false, 64>;
+        return slow ? gemv_mma_kernel<4, true, 32> : gemv_mma_kernel<4, false, 32>;
+    }
+    if (lanes == 64) return slow ? gemv_mma_kernel<8, true, 64> : gemv_mma_kernel<8, false, 64>;
+    return slow ? gemv_mma_kernel<8, true, 32> : gemv_mma_kernel<8, false, 32>;
+}
+
+// The tensor-core GEMV needs chunks of whole rows (every GEMV tensor has them).
+static bool mma_eligible(const DevTensor &d) {
+    return d.cols > 0 && d.chunk_symbols % d.cols == 0;
 }
 
 static LanesFn pick_single(int bits, int out, bool slow) {
@@ -1291,9 +1489,12 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     DeviceInfo di;
     if (device_info(ts[0]->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
-    long long x_elems = (out_kind == OUT_GEMV && max_kb <= kXSmemElems) ? max_kb : 0;
+    bool mma = out_kind == OUT_GEMV && bpad >= kTileBatch;
+    for (int i = 0; mma && i < count; i++) mma = mma_eligible(ts[i]->d);
+    long long x_elems = (out_kind == OUT_GEMV && !mma && max_kb <= kXSmemElems) ? max_kb : 0;
     const int stage_rows = max_words + kSlackRows;
-    const int out_words = kRing * lanes * bits / 4;  // the run ring: kRing runs of 8 codes per lane
+    // the run ring: kRing runs of 8 codes per lane (padded for the tensor-core GEMV's cross-warp reads)
+    const int out_words = mma ? tile_ring_words(bits, lanes) : kRing * lanes * bits / 4;
     long long chunks = 0;
     for (int i = 0; i < count; i++) chunks += ts[i]->d.n_chunks;
     // Spread the chunks evenly over the SMs: small inputs get one CTA per SM
@@ -1302,14 +1503,15 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     SmemOffsets so;
     for (;;) {
         so = smem_layout(warps, x_elems, stage_rows * lanes, out_words,
-                         out_kind == OUT_GEMV && bpad >= kPackedFmaBatch);
+                         mma ? static_cast<size_t>(warps) * 2 * 32 * 16 : 0);
         if ((long long)so.total <= di.smem_optin) break;
         if (warps > 1) warps--;
         else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
         else return ENTRO_E_LIMIT;
     }
     const size_t bytes = so.total;
-    LanesFn fn = pick_lanes(bits, out_kind, slow, bpad, lanes);
+    LanesFn fn = mma ? pick_mma(bits, slow, lanes) : pick_lanes(bits, out_kind, slow, bpad, lanes);
+    if (!fn) return ENTRO_E_INVAL;  // a batched GEMV whose chunks are not whole rows
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, bytes, &per_sm) != ENTRO_OK)
         return ENTRO_E_CUDA;

@@ -155,6 +155,37 @@ def test_gemv_shapes_and_batches(entro, bits, batch, shape, lanes):
     check_gemv(entro, dt, q, s, z, batch=batch, seed=batch)
 
 
+@pytest.mark.parametrize("bits,lanes,batch,shape", [(8, 32, 16, (2405, 8192)), (4, 64, 5, (2406, 3072)),
+                                                     (4, 32, 3, (600, 14336))])
+def test_gemv_batched_many_warps(entro, bits, lanes, batch, shape):
+    """Batched GEMV over enough whole-row chunks for many warps per CTA (16 at K = 8192), so
+    chunk groups end part-way through a CTA's warps; two launches give identical results."""
+    rows, cols = shape
+    w = workloads.small_tensor("t4" if bits == 8 else "laplace", rows, cols, seed=rows + bits)
+    chunk = max(1, 8192 // cols) * cols
+    q, s, z, _ = oracle.quantize(w, bits, oracle.MODE_ASYM)
+    dt = entro.upload(entro.Blob.encode(w, bits=bits, quant_mode=entro.QUANT_ASYM, chunk_symbols=chunk,
+                                        lanes=lanes))
+    x = workloads.activations(bits + batch, batch, cols)
+    st = _status()
+    y1 = dt.decode_gemv(x.cuda(), status=st)
+    y2 = dt.decode_gemv(x.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(y1, y2)
+    y_ref, mag = oracle.gemv(oracle.dequant_bf16(q, s, z).reshape(rows, cols), workloads.bf16_bits(x))
+    assert gemv_error(y1.cpu().numpy(), y_ref, mag) <= GEMV_TOL
+
+
+@pytest.mark.parametrize("batch", [4, 16])
+def test_gemv_batched_partial_last_chunk(entro, batch):
+    """33 rows in chunks of 2 rows: the last chunk is half a chunk (the CUDA-core batched path)."""
+    w = workloads.small_tensor("t4", 33, 3072, seed=33)
+    q, s, z, _ = oracle.quantize(w, 8, oracle.MODE_ASYM)
+    dt = entro.upload(entro.Blob.encode(w, bits=8, quant_mode=entro.QUANT_ASYM, chunk_symbols=6144))
+    check_gemv(entro, dt, q, s, z, batch=batch, seed=batch)
+
+
 def test_gemv_rejects_unsupported_layouts(entro):
     w = workloads.small_tensor("t4", 16, 300, seed=0)
     dt = entro.upload(entro.Blob.encode(w, bits=8, chunk_symbols=4096))
