@@ -46,6 +46,11 @@ constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
 constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
 constexpr int kSlackRows = 2;                 // staging rows past a chunk's longest lane (read-ahead)
+// A lane's window may run past its last word by the lookups made after its last
+// run completes (up to 3 of at most 24 bits, plus the word loaded one ahead):
+// reads stay inside the staging buffer (clamped); a lane that moved more than
+// this many rows past its words has decoded a corrupt stream.
+constexpr int kOverrunRows = 5;
 
 enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
 
@@ -317,11 +322,25 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
 }
 
 // Runs are staged in a ring of kRing slots per lane: a warp emits every
-// kEmitBlock runs, and a lane can only start up to two runs beyond the block
-// it is decoding, so kRing >= kEmitBlock + 2 keeps the slots being emitted
-// apart from the slots being written.
+// kEmitBlock runs, and a lane writes at most kLookupsPerCheck - 1 slots beyond
+// the block it is decoding, so kRing >= kEmitBlock + kLookupsPerCheck - 1
+// keeps the slots being emitted apart from the slots being written.
 constexpr int kEmitBlock = 8;
 constexpr int kRing = 16;
+constexpr int kLookupsPerCheck = 4;  // lanes kernel: table lookups between two checks of a lane's run count
+static_assert(kRing >= kEmitBlock + kLookupsPerCheck - 1, "ring too small for the decode overshoot");
+
+// Shifts that give 0 for a shift of 32 (PTX clamps the amount to the width).
+__device__ __forceinline__ uint32_t shl_clamp(uint32_t v, uint32_t n) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(n));
+    return r;
+}
+__device__ __forceinline__ uint32_t shr_clamp(uint32_t v, uint32_t n) {
+    uint32_t r;
+    asm("shr.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(n));
+    return r;
+}
 
 template <int BITS, bool SLOW, int LANES>
 struct LaneDecoder {
@@ -333,9 +352,9 @@ struct LaneDecoder {
     uint32_t bufcap;      // shared address of the last readable word of this lane
     uint32_t ostb;        // shared address of this lane's slot 0 of the run ring
     uint32_t osta;        // shared address of this lane's current run slot
-    int nb;
+    int nb;               // valid bits in the window
     uint32_t wnext;       // the next word, loaded one refill ahead (off the window's dependency chain)
-    uint64_t win;
+    uint32_t hi, lo;      // 64-bit window, MSB first: the next bits of the stream start at bit 31 of hi
     uint32_t p0, p1, p2;  // pending codes as one bit string, first code at bit 0 of p0
     int pb;               // pending bits (BITS per code); below one run whenever codes are appended
     int t;                // runs completed
@@ -345,7 +364,8 @@ struct LaneDecoder {
         bufa = smem_addr(b);
         bufcap = bufa + kRowBytes * static_cast<uint32_t>(cap);
         ostb = osta = smem_addr(o);
-        win = (static_cast<uint64_t>(lds32(bufa)) << 32) | lds32(bufa + kRowBytes);
+        hi = lds32(bufa);
+        lo = lds32(bufa + kRowBytes);
         nb = 64;
         bufa += 2 * kRowBytes;
         wnext = lds32(min(bufa, bufcap));
@@ -354,37 +374,42 @@ struct LaneDecoder {
         t = 0;
     }
 
+    // Top the window up to more than 32 bits: the next word lands right below
+    // the nb valid bits.  Branch-free apart from the predicated load.
     __device__ __forceinline__ void refill() {
-        if (nb <= 32) {
-            win |= static_cast<uint64_t>(wnext) << (32 - nb);
-            nb += 32;
-            bufa += kRowBytes;
-            wnext = lds32(min(bufa, bufcap));
-        }
+        const bool need = nb <= 32;
+        const uint32_t n = static_cast<uint32_t>(nb);
+        hi |= need ? shr_clamp(wnext, n) : 0u;
+        lo |= need ? shl_clamp(wnext, 32u - n) : 0u;
+        nb += need ? 32 : 0;
+        bufa += need ? kRowBytes : 0u;
+        if (need) wnext = lds32(min(bufa, bufcap));
     }
 
     // one table lookup; appends its codes to the pending bit string
     __device__ __forceinline__ void lookup(const Smem &s, int max_len, int32_t *status) {
-        const uint32_t e = lds32(lut + (static_cast<uint32_t>(win >> (64 - kMaxLutBits)) << 2));
+        const uint32_t e = lds32(lut + ((hi >> (32 - kMaxLutBits)) << 2));
         uint32_t syms = e >> 8, bits = e & 15u;
         // count * BITS straight from the entry's count field (bits 4..7)
         int add = static_cast<int>(BITS == 4 ? (e >> 2) & 0x3Cu : (e >> 1) & 0x78u);
         if (SLOW && add == 0) {
+            const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
             const uint32_t se = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, status);
             bits = se & 31u;
             syms = (se >> 8) & 0xFFu;
             add = BITS;
         }
-        win <<= bits;
+        hi = __funnelshift_l(lo, hi, bits);  // bits <= 24: the top 32 bits of (hi:lo) << bits
+        lo <<= bits;
         nb -= static_cast<int>(bits);
         const int q = pb & 31;
-        const uint32_t lo = syms << q, hi = __funnelshift_l(syms, 0u, q);  // (0:syms) << q, 24-bit codes
+        const uint32_t plo = syms << q, phi = __funnelshift_l(syms, 0u, q);  // (0:syms) << q, 24-bit codes
         if (BITS == 4 || pb < 32) {
-            p0 |= lo;
-            p1 |= hi;
+            p0 |= plo;
+            p1 |= phi;
         } else {
-            p1 |= lo;
-            p2 |= hi;
+            p1 |= plo;
+            p2 |= phi;
         }
         pb += add;
     }
@@ -395,19 +420,18 @@ struct LaneDecoder {
     __device__ __forceinline__ void emit() {
         if (BITS == 4) sts32(osta, p0);
         else sts64(osta, p0, p1);
-        if (pb >= kRunBits) {
-            if (BITS == 4) {
-                p0 = p1;
-                p1 = 0;
-            } else {
-                p0 = p2;
-                p1 = 0;
-                p2 = 0;
-            }
-            pb -= kRunBits;
-            t++;
-            osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
+        const bool done = pb >= kRunBits;
+        if (BITS == 4) {
+            p0 = done ? p1 : p0;
+            p1 = done ? 0u : p1;
+        } else {
+            p0 = done ? p2 : p0;
+            p1 = done ? 0u : p1;
+            p2 = done ? 0u : p2;
         }
+        pb -= done ? kRunBits : 0;
+        t += done ? 1 : 0;
+        osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
     }
 
     // store the current (possibly partial) run and count it done
@@ -417,7 +441,6 @@ struct LaneDecoder {
         t++;
         osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
     }
-
 };
 
 // ------------------------------------------------------------------ phase 2: stage -> output
@@ -551,9 +574,11 @@ __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, 
     }
 }
 
-// Advance every format lane the thread serves to run te (whole runs).  A lane
-// may write the first codes of run te before it stops: one slot past the block.
-template <int BITS, bool SLOW, int LANES, int LPT>
+// Advance every format lane the thread serves to run te (whole runs), STEPS
+// (2 or 4) lookups per check.  A lane may write up to STEPS - 1 slots past the
+// block before it stops (and reads past its last word by as many lookups,
+// which the staging slack covers).
+template <int STEPS, int BITS, bool SLOW, int LANES, int LPT>
 __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[LPT], const Smem &s, int te,
                                           int max_len, bool refill_each, int32_t *status) {
     bool more = true;
@@ -562,12 +587,15 @@ __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[L
 #pragma unroll
         for (int k = 0; k < LPT; k++) {
             if (ld[k].t < te) {
-                ld[k].refill();
-                ld[k].lookup(s, max_len, status);
-                ld[k].emit();
-                if (SLOW && refill_each) ld[k].refill();
-                ld[k].lookup(s, max_len, status);
-                ld[k].emit();
+#pragma unroll
+                for (int h = 0; h < STEPS / 2; h++) {
+                    ld[k].refill();
+                    ld[k].lookup(s, max_len, status);
+                    ld[k].emit();
+                    if (SLOW && refill_each) ld[k].refill();
+                    ld[k].lookup(s, max_len, status);
+                    ld[k].emit();
+                }
                 more = more || ld[k].t < te;
             }
         }
@@ -599,8 +627,8 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
     for (int k = 0; k < LPT; k++) {
         const int l = lane + kLanes * k;
         ld[k].init(s, buf + l, ost + (BITS == 4 ? l : 2 * l), stage_rows - 1);
-        // a valid lane never loads past its words plus the two read-ahead rows
-        read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kSlackRows);
+        // a valid lane never moves more than kOverrunRows rows past its words
+        read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
     }
     bool ok = true;
     if (nc % kStep == 0) {
@@ -612,7 +640,7 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
         for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
-            decode_to(ld, s, te, d.max_len, refill_each, status);
+            decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, status);
             __syncwarp();
             emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
             __syncwarp();  // the ring slots just read are rewritten by the next block
@@ -944,13 +972,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                 for (int q = 0; q < LPT; q++) {
                     const int l = lane + kLanes * q;
                     ld[q].init(s, buf + l, ost + (BITS == 4 ? l : 2 * l), a.stage_rows - 1);
-                    read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kSlackRows);
+                    read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
                 }
             }
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
-                if (active && tb < my_runs) decode_to(ld, s, te, d.max_len, refill_each, a.status);
+                if (active && tb < my_runs) decode_to<2>(ld, s, te, d.max_len, refill_each, a.status);
                 __syncthreads();  // the block's runs of every row are in the rings
                 const int col0 = (tb % spr) * (kRun * LANES);
                 for (int q = warp; q < groups; q += warps) {
