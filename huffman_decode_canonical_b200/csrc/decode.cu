@@ -414,24 +414,92 @@ struct LaneDecoder {
         pb += add;
     }
 
-    // Store the current run's pending codes to its slot -- harmless while the
-    // run is incomplete, since the slot is rewritten until it is -- and move on
-    // once the run is whole.  At most one run completes per lookup.
-    __device__ __forceinline__ void emit() {
-        if (BITS == 4) sts32(osta, p0);
-        else sts64(osta, p0, p1);
-        const bool done = pb >= kRunBits;
-        if (BITS == 4) {
-            p0 = done ? p1 : p0;
-            p1 = done ? 0u : p1;
-        } else {
-            p0 = done ? p2 : p0;
-            p1 = done ? 0u : p1;
-            p2 = done ? 0u : p2;
+    // One table lookup and its run bookkeeping (the fast path of lookup() +
+    // emit()).  The window shift, the append of the entry's codes to the
+    // pending string, the slot store and the run completion are one block of
+    // hand-written PTX; a miss in the table (a code longer than 12 bits) goes
+    // through the canonical slow path and re-enters as a one-code entry.
+    __device__ __forceinline__ void step(const Smem &s, int max_len, int32_t *status) {
+        uint32_t e = lds32(lut + ((hi >> (32 - kMaxLutBits)) << 2));
+        uint32_t bits = e & 15u;
+        if (SLOW && (e & 0xF0u) == 0) {
+            const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
+            const uint32_t se = slow_entry(win, max_len, s.slim, s.soffs, s.ssyms, status);
+            bits = se & 31u;
+            e = (1u << 4) | (se & 0xFF00u);
         }
-        pb -= done ? kRunBits : 0;
-        t += done ? 1 : 0;
-        osta = ostb + static_cast<uint32_t>(t & (kRing - 1)) * kRunStride;
+        advance(e, bits);
+    }
+
+    // Consume `bits` of the window and append the entry's codes (count in bits
+    // 4..7 of e, codes from bit 8); store the current run's slot; move to the
+    // next slot when the run is whole.
+    __device__ __forceinline__ void advance(uint32_t e, uint32_t bits) {
+        if (BITS == 4) {
+            // pb < 32 before the append (a run completes at 32 bits)
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 add, syms, plo, phi, tw;\n\t"
+                ".reg .pred done;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %9;\n\t"
+                "shl.b32 %1, %1, %9;\n\t"
+                "sub.s32 %2, %2, %9;\n\t"
+                "and.b32 add, %8, 240;\n\t"
+                "shr.u32 add, add, 2;\n\t"
+                "shr.u32 syms, %8, 8;\n\t"
+                "shl.b32 plo, syms, %5;\n\t"
+                "shf.l.wrap.b32 phi, syms, 0, %5;\n\t"
+                "or.b32 %3, %3, plo;\n\t"
+                "or.b32 %4, %4, phi;\n\t"
+                "add.s32 %5, %5, add;\n\t"
+                "st.shared.u32 [%7], %3;\n\t"
+                "setp.ge.s32 done, %5, 32;\n\t"
+                "selp.b32 %3, %4, %3, done;\n\t"
+                "selp.b32 %4, 0, %4, done;\n\t"
+                "@done sub.s32 %5, %5, 32;\n\t"
+                "@done add.s32 %6, %6, 1;\n\t"
+                "and.b32 tw, %6, 15;\n\t"
+                "mad.lo.u32 %7, tw, %11, %10;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(nb), "+r"(p0), "+r"(p1), "+r"(pb), "+r"(t), "+r"(osta)
+                : "r"(e), "r"(bits), "r"(ostb), "n"(kRunStride)
+                : "memory");
+        } else {
+            // pb < 64 before the append; codes go to p0:p1 below bit 32 of the
+            // string's current word, to p1:p2 above
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 add, syms, plo, phi, q, tw;\n\t"
+                ".reg .pred lt, done;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %10;\n\t"
+                "shl.b32 %1, %1, %10;\n\t"
+                "sub.s32 %2, %2, %10;\n\t"
+                "shr.u32 add, %9, 1;\n\t"
+                "and.b32 add, add, 120;\n\t"
+                "shr.u32 syms, %9, 8;\n\t"
+                "and.b32 q, %6, 31;\n\t"
+                "shl.b32 plo, syms, q;\n\t"
+                "shf.l.wrap.b32 phi, syms, 0, q;\n\t"
+                "setp.lt.s32 lt, %6, 32;\n\t"
+                "@lt or.b32 %3, %3, plo;\n\t"
+                "@lt or.b32 %4, %4, phi;\n\t"
+                "@!lt or.b32 %4, %4, plo;\n\t"
+                "@!lt or.b32 %5, %5, phi;\n\t"
+                "add.s32 %6, %6, add;\n\t"
+                "st.shared.v2.u32 [%8], {%3, %4};\n\t"
+                "setp.ge.s32 done, %6, 64;\n\t"
+                "selp.b32 %3, %5, %3, done;\n\t"
+                "selp.b32 %4, 0, %4, done;\n\t"
+                "selp.b32 %5, 0, %5, done;\n\t"
+                "@done sub.s32 %6, %6, 64;\n\t"
+                "@done add.s32 %7, %7, 1;\n\t"
+                "and.b32 tw, %7, 15;\n\t"
+                "mad.lo.u32 %8, tw, %12, %11;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(nb), "+r"(p0), "+r"(p1), "+r"(p2), "+r"(pb), "+r"(t), "+r"(osta)
+                : "r"(e), "r"(bits), "r"(ostb), "n"(kRunStride)
+                : "memory");
+        }
     }
 
     // store the current (possibly partial) run and count it done
@@ -590,11 +658,9 @@ __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[L
 #pragma unroll
                 for (int h = 0; h < STEPS / 2; h++) {
                     ld[k].refill();
-                    ld[k].lookup(s, max_len, status);
-                    ld[k].emit();
+                    ld[k].step(s, max_len, status);
                     if (SLOW && refill_each) ld[k].refill();
-                    ld[k].lookup(s, max_len, status);
-                    ld[k].emit();
+                    ld[k].step(s, max_len, status);
                 }
                 more = more || ld[k].t < te;
             }
@@ -662,11 +728,9 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
                 const int tf = min(te, full_runs);
                 while (ld[k].t < tf) {
                     ld[k].refill();
-                    ld[k].lookup(s, d.max_len, status);
-                    ld[k].emit();
+                    ld[k].step(s, d.max_len, status);
                     if (SLOW && refill_each) ld[k].refill();
-                    ld[k].lookup(s, d.max_len, status);
-                    ld[k].emit();
+                    ld[k].step(s, d.max_len, status);
                 }
                 if (tail && ld[k].t == full_runs && full_runs < te) {
                     while (ld[k].pb < tail * BITS) {
@@ -828,7 +892,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 //   B = W^T[16 columns, 8 rows of the CTA]              from the warps' run rings
 //   D = y partials [16 batch rows, 8 rows]              registers, per warp
 // Each lockstep block covers E runs of every chunk (E divides the runs of a
-// row, E + 1 <= kRing); after a CTA barrier the block's columns are split
+// row; E plus the kLookupsPerCheck - 1 slots a lane may write past it fit the
+// ring); after a CTA barrier the block's columns are split
 // among the warps in groups of 32 (4 format lanes x 8 weights).  The k order
 // inside an MMA is permuted so that each thread's B registers are the 8
 // weights of one ring slot and its A registers one 16-byte load of x:
@@ -839,7 +904,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 // not the bound: the MMAs replace 16 FMAs per weight with 1/8 of an MMA issue,
 // and x is read once per CTA instead of once per warp.
 
-constexpr int kTileMaxBlock = kRing - 1;  // a block plus the slot a lane may write past it fit the ring
+constexpr int kTileMaxBlock = kRing - kLookupsPerCheck + 1;  // a block plus the slots a lane may write past it fit the ring
 constexpr int kTileBatch = 4;             // padded batch from which the tensor-core GEMV runs
 
 // Runs per lockstep block: the largest divisor of the runs per row that fits the ring.
@@ -978,7 +1043,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
-                if (active && tb < my_runs) decode_to<2>(ld, s, te, d.max_len, refill_each, a.status);
+                if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, a.status);
                 __syncthreads();  // the block's runs of every row are in the rings
                 const int col0 = (tb % spr) * (kRun * LANES);
                 for (int q = warp; q < groups; q += warps) {
