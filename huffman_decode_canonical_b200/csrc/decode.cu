@@ -548,8 +548,22 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
         uint4 *dst = reinterpret_cast<uint4 *>(g.out) + first * BITS / 128 + tb * kU4PerRun;
         for (int i = lane; i < (te - tb) * kU4PerRun; i += kLanes) dst[i] = src[i];
     } else if (OUT == OUT_BF16) {
+        // four runs per pass: their table lookups are all in flight before the stores
         uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(g.out) + first);
-        for (int t = tb; t < te; t++)
+        int t = tb;
+        for (; t + 4 <= te; t += 4) {
+            uint4 v[4][LPT];
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+#pragma unroll
+                for (int k = 0; k < LPT; k++)
+                    v[j][k] = values8<BITS>(s, ost, LANES * ((t + j) & (kRing - 1)) + lane + kLanes * k);
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+#pragma unroll
+                for (int k = 0; k < LPT; k++) dst[LANES * (t + j) + lane + kLanes * k] = v[j][k];
+        }
+        for (; t < te; t++)
 #pragma unroll
             for (int k = 0; k < LPT; k++) {
                 const int l = lane + kLanes * k;
@@ -557,43 +571,76 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
             }
     } else {
         // fused GEMV (batch 1 and 2): run t covers columns 8*LANES*(t % spr) + 8*l .. +7
-        // of row t / spr.  Each lane keeps one fp32 sum per batch row, fed by
-        // mixed-precision FMAs of the bf16 weights and activations
-        // (fma.rn.f32.bf16), and the warp reduces at the row end.
+        // of row t / spr.  Four runs per pass: each run's 8 weights are
+        // multiplied with mixed-precision FMAs of the bf16 weights and
+        // activations (fma.rn.f32.bf16) into a partial sum of its own, so the
+        // passes' loads and FMA chains overlap; the partials are then added to
+        // the lane's row sum in run order, and the warp reduces at the row end.
         const int K = static_cast<int>(d.cols);
         const int spr = K / (kRun * LANES);
-        const long long row0 = first / K;
+        const int xrow = K >> 3;  // uint4 per row of x
         const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
-        for (int t = tb; t < te; t++) {
-            const int st = t % spr;
+        int st = tb % spr;                       // run step within its row
+        long long row = first / K + tb / spr;    // the row run tb belongs to
+        for (int t = tb; t < te; t += 4) {
+            const int n = min(4, te - t);
+            int stj[4];
+            {
+                int sj = st;
 #pragma unroll
-            for (int k = 0; k < LPT; k++) {
-                const int l = lane + kLanes * k;
-                const int slot = LANES * (t & (kRing - 1)) + l;
-                const int xo = st * LANES + l;  // uint4 index within one x row
-                const uint4 wv = values8<BITS>(s, ost, slot);
+                for (int j = 0; j < 4; j++) {
+                    stj[j] = sj;
+                    sj = sj + 1 == spr ? 0 : sj + 1;
+                }
+                st = stj[0];
 #pragma unroll
-                for (int b = 0; b < BPAD; b++) {
-                    if (b < batch) {
-                        const int xi = b * (K >> 3) + xo;
-                        const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
-                        acc[b] = fma2_bf16(wv.x, xv.x, acc[b]);
-                        acc[b] = fma2_bf16(wv.y, xv.y, acc[b]);
-                        acc[b] = fma2_bf16(wv.z, xv.z, acc[b]);
-                        acc[b] = fma2_bf16(wv.w, xv.w, acc[b]);
+                for (int j = 0; j < 4; j++)
+                    if (j < n) st = st + 1 == spr ? 0 : st + 1;
+            }
+            float part[4][BPAD];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+#pragma unroll
+                for (int b = 0; b < BPAD; b++) part[j][b] = 0.f;
+                if (j < n) {
+#pragma unroll
+                    for (int k = 0; k < LPT; k++) {
+                        const int l = lane + kLanes * k;
+                        const uint4 wv = values8<BITS>(s, ost, LANES * ((t + j) & (kRing - 1)) + l);
+                        const int xo = stj[j] * LANES + l;
+#pragma unroll
+                        for (int b = 0; b < BPAD; b++) {
+                            if (b < batch) {
+                                const int xi = b * xrow + xo;
+                                const uint4 xv = x_in_smem ? xsm[xi] : __ldg(xg + xi);
+                                float p = part[j][b];
+                                p = fma2_bf16(wv.x, xv.x, p);
+                                p = fma2_bf16(wv.y, xv.y, p);
+                                p = fma2_bf16(wv.z, xv.z, p);
+                                p = fma2_bf16(wv.w, xv.w, p);
+                                part[j][b] = p;
+                            }
+                        }
                     }
                 }
             }
-            if (st == spr - 1) {
-                const long long row = row0 + t / spr;
 #pragma unroll
-                for (int b = 0; b < BPAD; b++) {
-                    if (b < batch) {
-                        const float v = warp_sum(acc[b]);
-                        if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row] = v;
+            for (int j = 0; j < 4; j++) {
+                if (j < n) {
+#pragma unroll
+                    for (int b = 0; b < BPAD; b++) acc[b] += part[j][b];
+                    if (stj[j] == spr - 1) {
+#pragma unroll
+                        for (int b = 0; b < BPAD; b++) {
+                            if (b < batch) {
+                                const float v = warp_sum(acc[b]);
+                                if (lane == 0) g.y[static_cast<long long>(b) * d.rows + row] = v;
+                            }
+                            acc[b] = 0.f;
+                        }
+                        row++;
                     }
-                    acc[b] = 0.f;
                 }
             }
         }
@@ -1046,22 +1093,38 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                 if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, a.status);
                 __syncthreads();  // the block's runs of every row are in the rings
                 const int col0 = (tb % spr) * (kRun * LANES);
-                for (int q = warp; q < groups; q += warps) {
-                    const int t = tb + q / kGroupsPerRun;
-                    const int slot = LANES * (t & (kRing - 1)) + 4 * (q % kGroupsPerRun) + tig;
-                    const int xo = ((col0 + 32 * q) >> 3) + tig;
-                    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-                    const uint4 xa = gid < batch ? __ldg(xg + gid * xrow + xo) : z4;
-                    const uint4 xb = gid + 8 < batch ? __ldg(xg + (gid + 8) * xrow + xo) : z4;
+                // two groups per pass: both groups' x loads (from L2) are in flight together
+                const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                for (int q0 = warp; q0 < groups; q0 += 2 * warps) {
+                    uint4 xa[2], xb[2], w[2][2];
+                    int slot[2];
 #pragma unroll
-                    for (int nt = 0; nt < 2; nt++) {
-                        if (8 * nt >= nrows) break;
-                        const int r = 8 * nt + gid;
-                        const uint4 w = r < nrows ? values8<BITS>(s, s.ostage + static_cast<size_t>(r) * a.out_words, slot)
-                                                  : z4;
-                        mma_16816_bf16(acc[nt], xa.x, xb.x, xa.y, xb.y, w.x, w.y);
-                        mma_16816_bf16(acc[nt], xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+                    for (int h = 0; h < 2; h++) {
+                        const int q = q0 + h * warps;
+                        const bool has = q < groups;
+                        const int t = tb + q / kGroupsPerRun;
+                        slot[h] = LANES * (t & (kRing - 1)) + 4 * (q % kGroupsPerRun) + tig;
+                        const int xo = ((col0 + 32 * q) >> 3) + tig;
+                        xa[h] = has && gid < batch ? __ldg(xg + gid * xrow + xo) : z4;
+                        xb[h] = has && gid + 8 < batch ? __ldg(xg + (gid + 8) * xrow + xo) : z4;
                     }
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+#pragma unroll
+                        for (int nt = 0; nt < 2; nt++) {
+                            const int r = 8 * nt + gid;
+                            w[h][nt] = q0 + h * warps < groups && r < nrows
+                                           ? values8<BITS>(s, s.ostage + static_cast<size_t>(r) * a.out_words, slot[h])
+                                           : z4;
+                        }
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+#pragma unroll
+                        for (int nt = 0; nt < 2; nt++) {
+                            if (8 * nt >= nrows) break;
+                            mma_16816_bf16(acc[nt], xa[h].x, xb[h].x, xa[h].y, xb[h].y, w[h][nt].x, w[h][nt].y);
+                            mma_16816_bf16(acc[nt], xa[h].z, xb[h].z, xa[h].w, xb[h].w, w[h][nt].z, w[h][nt].w);
+                        }
                 }
                 if (te % spr == 0) {
                     // row end: partial sums of every warp, added in warp order
