@@ -537,7 +537,8 @@ __device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int
 // thread `lane` serves the format lanes lane, lane + 32, ...
 template <int BITS, int OUT, int BPAD, int LANES>
 __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, const uint32_t *ost, long long first,
-                                          int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD]) {
+                                          int tb, int te, int batch, int x_in_smem, float (&acc)[BPAD],
+                                          int &st, long long &row) {
     constexpr int LPT = LANES / kLanes;
     const DevTensor &d = g.d;
     const int lane = threadIdx.x & 31;
@@ -576,13 +577,12 @@ __device__ __forceinline__ void emit_runs(const GroupEntry &g, const Smem &s, co
         // activations (fma.rn.f32.bf16) into a partial sum of its own, so the
         // passes' loads and FMA chains overlap; the partials are then added to
         // the lane's row sum in run order, and the warp reduces at the row end.
+        // `st` (run step within the row) and `row` carry over from block to block.
         const int K = static_cast<int>(d.cols);
         const int spr = K / (kRun * LANES);
         const int xrow = K >> 3;  // uint4 per row of x
         const uint4 *xg = reinterpret_cast<const uint4 *>(g.x);
         const uint4 *xsm = reinterpret_cast<const uint4 *>(s.xs);
-        int st = tb % spr;                       // run step within its row
-        long long row = first / K + tb / spr;    // the row run tb belongs to
         for (int t = tb; t < te; t += 4) {
             const int n = min(4, te - t);
             int stj[4];
@@ -751,11 +751,16 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
         float acc[BPAD];
 #pragma unroll
         for (int b = 0; b < BPAD; b++) acc[b] = 0.f;
+        // GEMV: run step within the row and the row of the chunk's first run (chunks are whole rows)
+        int gst = 0;
+        long long grow = OUT == OUT_GEMV ? c * static_cast<long long>(static_cast<int>(d.chunk_symbols) /
+                                                                      static_cast<int>(d.cols))
+                                         : 0;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
             decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, status);
             __syncwarp();
-            emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc);
+            emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc, gst, grow);
             __syncwarp();  // the ring slots just read are rewritten by the next block
         }
 #pragma unroll
