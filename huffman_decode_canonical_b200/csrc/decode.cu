@@ -940,21 +940,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 // lockstep on consecutive chunks (= consecutive rows, since its tensors have
 // whole-row chunks) and multiply with mma.sync m16n8k16 (bf16 operands, fp32
 // accumulation):
-//   A = x[16 batch rows (zero-padded), 16 columns]      straight from global
-//   B = W^T[16 columns, 8 rows of the CTA]              from the warps' run rings
-//   D = y partials [16 batch rows, 8 rows]              registers, per warp
+//   A = W[the CTA's 16 rows, 16 columns]                from the warps' run rings
+//   B = x^T[16 columns, 8 batch rows] (1 or 2 tiles)    from global memory (L2)
+//   D = y partials [16 rows, 8 batch rows]              registers, per warp
 // Each lockstep block covers E runs of every chunk (E divides the runs of a
 // row; E plus the kLookupsPerCheck - 1 slots a lane may write past it fit the
-// ring); after a CTA barrier the block's columns are split
-// among the warps in groups of 32 (4 format lanes x 8 weights).  The k order
-// inside an MMA is permuted so that each thread's B registers are the 8
-// weights of one ring slot and its A registers one 16-byte load of x:
+// ring); after a CTA barrier the block's columns are split among the warps in
+// groups of 32 (4 format lanes x 8 weights).  The k order inside an MMA is
+// permuted so that each thread's A registers are the 8 weights of one ring
+// slot and its B registers one 16-byte load of x:
 //   k-step 0: k = 2j + e <-> column 8j + e, k = 2j + 8 + e <-> column 8j + 2 + e
 //   k-step 1: the same with columns 8j + 4 + e and 8j + 6 + e  (j = lane % 4)
 // The partial sums of a row are added across warps in warp order at the row's
-// end (fixed order: the result does not depend on timing).  The tensor pipe is
-// not the bound: the MMAs replace 16 FMAs per weight with 1/8 of an MMA issue,
-// and x is read once per CTA instead of once per warp.
+// end (fixed order: the result does not depend on timing).  For a batch of up
+// to 8 one MMA covers 256 weights.
 
 constexpr int kTileMaxBlock = kRing - kLookupsPerCheck + 1;  // a block plus the slots a lane may write past it fit the ring
 constexpr int kTileBatch = 4;             // padded batch from which the tensor-core GEMV runs
@@ -981,14 +980,14 @@ __device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int BITS, bool SLOW, int LANES>
+template <int BITS, bool SLOW, int LANES, int NB>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     constexpr int LPT = LANES / kLanes;
     constexpr int kGroupsPerRun = LANES / 4;  // 32-column groups in one run step of a chunk
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
-    const Smem s = carve(smem_raw, warps, 0, a.stage_rows * LANES, a.out_words, static_cast<size_t>(warps) * 2 * 32 * 16);
+    const Smem s = carve(smem_raw, warps, 0, a.stage_rows * LANES, a.out_words, static_cast<size_t>(warps) * NB * 32 * 16);
     uint64_t *bar = s.bars + 2 * warp;
     const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
     uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
@@ -1092,67 +1091,82 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                     read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
                 }
             }
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float acc[NB][4];
+#pragma unroll
+            for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) acc[nb][i] = 0.f;
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
                 if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, a.status);
                 __syncthreads();  // the block's runs of every row are in the rings
                 const int col0 = (tb % spr) * (kRun * LANES);
-                // two groups per pass: both groups' x loads (from L2) are in flight together
+                // The warp's groups q = warp, warp + warps, ... two per pass; the x
+                // fragments of the next pass are loaded (from L2) while this pass
+                // multiplies.  A = rows gid and gid + 8 of the group (the code
+                // rings of those warps), B = x^T of batch rows 8 nb + gid.
                 const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t *ring_lo = s.ostage + static_cast<size_t>(gid) * a.out_words;
+                const uint32_t *ring_hi = s.ostage + static_cast<size_t>(gid + 8) * a.out_words;
+                const bool has_lo = gid < nrows, has_hi = gid + 8 < nrows;
+                auto xload = [&](int q, uint4(&xr)[NB]) {
+                    const int xo = ((col0 + 32 * q) >> 3) + tig;
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) {
+                        const int bb = 8 * nb + gid;
+                        xr[nb] = q < groups && bb < batch ? __ldg(xg + bb * xrow + xo) : z4;
+                    }
+                };
+                uint4 xc[2][NB];
+                xload(warp, xc[0]);
+                xload(warp + warps, xc[1]);
                 for (int q0 = warp; q0 < groups; q0 += 2 * warps) {
-                    uint4 xa[2], xb[2], w[2][2];
-                    int slot[2];
+                    uint4 xn[2][NB];
+                    xload(q0 + 2 * warps, xn[0]);
+                    xload(q0 + 3 * warps, xn[1]);
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
                         const int q = q0 + h * warps;
-                        const bool has = q < groups;
+                        if (q >= groups) break;
                         const int t = tb + q / kGroupsPerRun;
-                        slot[h] = LANES * (t & (kRing - 1)) + 4 * (q % kGroupsPerRun) + tig;
-                        const int xo = ((col0 + 32 * q) >> 3) + tig;
-                        xa[h] = has && gid < batch ? __ldg(xg + gid * xrow + xo) : z4;
-                        xb[h] = has && gid + 8 < batch ? __ldg(xg + (gid + 8) * xrow + xo) : z4;
+                        const int slot = LANES * (t & (kRing - 1)) + 4 * (q % kGroupsPerRun) + tig;
+                        const uint4 wlo = has_lo ? values8<BITS>(s, ring_lo, slot) : z4;
+                        const uint4 whi = has_hi ? values8<BITS>(s, ring_hi, slot) : z4;
+#pragma unroll
+                        for (int nb = 0; nb < NB; nb++) {
+                            mma_16816_bf16(acc[nb], wlo.x, whi.x, wlo.y, whi.y, xc[h][nb].x, xc[h][nb].y);
+                            mma_16816_bf16(acc[nb], wlo.z, whi.z, wlo.w, whi.w, xc[h][nb].z, xc[h][nb].w);
+                        }
                     }
 #pragma unroll
                     for (int h = 0; h < 2; h++)
 #pragma unroll
-                        for (int nt = 0; nt < 2; nt++) {
-                            const int r = 8 * nt + gid;
-                            w[h][nt] = q0 + h * warps < groups && r < nrows
-                                           ? values8<BITS>(s, s.ostage + static_cast<size_t>(r) * a.out_words, slot[h])
-                                           : z4;
-                        }
-#pragma unroll
-                    for (int h = 0; h < 2; h++)
-#pragma unroll
-                        for (int nt = 0; nt < 2; nt++) {
-                            if (8 * nt >= nrows) break;
-                            mma_16816_bf16(acc[nt], xa[h].x, xb[h].x, xa[h].y, xb[h].y, w[h][nt].x, w[h][nt].y);
-                            mma_16816_bf16(acc[nt], xa[h].z, xb[h].z, xa[h].w, xb[h].w, w[h][nt].z, w[h][nt].w);
-                        }
+                        for (int nb = 0; nb < NB; nb++) xc[h][nb] = xn[h][nb];
                 }
                 if (te % spr == 0) {
-                    // row end: partial sums of every warp, added in warp order
+                    // row end: partial sums of every warp, added in warp order.  Thread
+                    // 4 (r % 8) + n / 2 holds D[r][n] (element 2 (r >= 8) + n % 2).
                     float4 *rd = reinterpret_cast<float4 *>(s.red);
-                    rd[(2 * warp) * 32 + lane] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-                    rd[(2 * warp + 1) * 32 + lane] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++)
+                        rd[(NB * warp + nb) * 32 + lane] = make_float4(acc[nb][0], acc[nb][1], acc[nb][2], acc[nb][3]);
                     __syncthreads();
                     const long long row_in_chunk = tb / spr;
                     for (int o = threadIdx.x; o < 256; o += blockDim.x) {
                         const int bb = o >> 4, r = o & 15;
                         const long long row = (c0 + r) * rows_per_chunk + row_in_chunk;
                         if (bb < batch && r < nrows && row < d.rows) {
-                            const int nt = r >> 3, n = r & 7;
-                            const int src = ((4 * (bb & 7) + (n >> 1)) << 2) + ((bb >> 3) << 1) + (n & 1);
+                            const int nb = bb >> 3, n = bb & 7;
+                            const int src = ((4 * (r & 7) + (n >> 1)) << 2) + ((r >> 3) << 1) + (n & 1);
                             float v = 0.f;
-                            for (int w = 0; w < warps; w++) v += s.red[(2 * w + nt) * 128 + src];
+                            for (int w = 0; w < warps; w++) v += s.red[(NB * w + nb) * 128 + src];
                             g.y[static_cast<long long>(bb) * d.rows + row] = v;
                         }
                     }
 #pragma unroll
-                    for (int nt = 0; nt < 2; nt++)
+                    for (int nb = 0; nb < NB; nb++)
 #pragma unroll
-                        for (int i = 0; i < 4; i++) acc[nt][i] = 0.f;
+                        for (int i = 0; i < 4; i++) acc[nb][i] = 0.f;
                 }
                 __syncthreads();  // every warp is done reading the rings before they are rewritten
             }
@@ -1547,13 +1561,21 @@ static LanesFn pick_lanes(int bits, int out, bool slow, int bpad, int lanes) {
     return lanes == 64 ? pick_out<8, 64>(out, slow, bpad) : pick_out<8, 32>(out, slow, bpad);
 }
 
-static LanesFn pick_mma(int bits, bool slow, int lanes) {
+template <int NB>
+static LanesFn pick_mma_nb(int bits, bool slow, int lanes) {
     if (bits == 4) {
-        if (lanes == 64) return slow ? gemv_mma_kernel<4, true, 64> : gemv_mma_kernel<4, false, 64>;
-        return slow ? gemv_mma_kernel<4, true, 32> : gemv_mma_kernel<4, false, 32>;
+        if (lanes == 64) return slow ? gemv_mma_kernel<4, true, 64, NB> : gemv_mma_kernel<4, false, 64, NB>;
+        return slow ? gemv_mma_kernel<4, true, 32, NB> : gemv_mma_kernel<4, false, 32, NB>;
     }
-    if (lanes == 64) return slow ? gemv_mma_kernel<8, true, 64> : gemv_mma_kernel<8, false, 64>;
-    return slow ? gemv_mma_kernel<8, true, 32> : gemv_mma_kernel<8, false, 32>;
+    if (lanes == 64) return slow ? gemv_mma_kernel<8, true, 64, NB> : gemv_mma_kernel<8, false, 64, NB>;
+    return slow ? gemv_mma_kernel<8, true, 32, NB> : gemv_mma_kernel<8, false, 32, NB>;
+}
+
+// NB = 8-row tiles of the batch (B operand of the MMAs)
+static int mma_batch_tiles(int batch) { return batch > 8 ? 2 : 1; }
+
+static LanesFn pick_mma(int bits, bool slow, int lanes, int batch) {
+    return mma_batch_tiles(batch) == 2 ? pick_mma_nb<2>(bits, slow, lanes) : pick_mma_nb<1>(bits, slow, lanes);
 }
 
 // The tensor-core GEMV needs chunks of whole rows (every GEMV tensor has them).
@@ -1664,14 +1686,14 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     SmemOffsets so;
     for (;;) {
         so = smem_layout(warps, x_elems, stage_rows * lanes, out_words,
-                         mma ? static_cast<size_t>(warps) * 2 * 32 * 16 : 0);
+                         mma ? static_cast<size_t>(warps) * mma_batch_tiles(batch) * 32 * 16 : 0);
         if ((long long)so.total <= di.smem_optin) break;
         if (warps > 1) warps--;
         else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
         else return ENTRO_E_LIMIT;
     }
     const size_t bytes = so.total;
-    LanesFn fn = mma ? pick_mma(bits, slow, lanes) : pick_lanes(bits, out_kind, slow, bpad, lanes);
+    LanesFn fn = mma ? pick_mma(bits, slow, lanes, batch) : pick_lanes(bits, out_kind, slow, bpad, lanes);
     if (!fn) return ENTRO_E_INVAL;  // a batched GEMV whose chunks are not whole rows
     int per_sm = 0;
     if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, bytes, &per_sm) != ENTRO_OK)
