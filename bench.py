@@ -10,8 +10,10 @@ payload alone, against a 126 MB L2) and of its outputs rotate, each kernel on
 the next replica, so every kernel reads coded words that no recent kernel
 touched and writes outputs whose lines must first be evicted -- the steady
 state of decoding a model much larger than L2 (no flush kernel, so the decode
-code stays warm as it would in serving).  Kernel
-times come from CUDA events on the launching stream.
+code stays warm as it would in serving).  Times come from CUDA events on the
+launching stream: the K timed steps run back to back between one pair of
+events, and each kernel's own duration is the mean over K launches of it back
+to back (events between the calls would add gaps of their own, ~2.5 us each).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
@@ -272,14 +274,9 @@ def run_native(args, dist, rank, world, local_rank):
                ("bf16", lambda r: reps[r].decode_dequant_bf16(out=bf[r], status=status)),
                ("gemv", lambda r: reps[r].decode_gemv(x, y=y[r], status=status))]
 
-    def step(evs=None):
-        for i, (_, fn) in enumerate(kernels):
-            r = next_rep()
-            if evs is not None:
-                evs[2 * i].record(stream)
-            fn(r)
-            if evs is not None:
-                evs[2 * i + 1].record(stream)
+    def step():
+        for _, fn in kernels:
+            fn(next_rep())
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -291,24 +288,37 @@ def run_native(args, dist, rank, world, local_rank):
     while time.perf_counter() < t_end:
         step()
         torch.cuda.synchronize(device)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # The K steps run back to back between one pair of events (events between
+    # the calls would add their own gaps); the GPU is kept busy while the host
+    # enqueues them, so the events measure device time only.
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(dist, device)
     torch.cuda.synchronize(device)
     wall0 = time.perf_counter()
-    # keep the GPU busy while the host enqueues the timed steps, so that the
-    # kernels run back to back and the events measure device time only
     torch.cuda._sleep(int(args.steps * 300e-6 * 2.0e9))
+    ev0.record(stream)
     for s in range(args.steps):
-        step(events[s])
+        step()
+    ev1.record(stream)
     torch.cuda.synchronize(device)
     wall = time.perf_counter() - wall0
     _barrier(dist, device)
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+    # Each kernel's own duration: K launches of it back to back (rotating
+    # replicas), between one pair of events.
+    mean_ms = {}
+    for name, fn in kernels:
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(device)
+        torch.cuda._sleep(int(args.steps * 100e-6 * 2.0e9))
+        k0.record(stream)
+        for s in range(args.steps):
+            fn(next_rep())
+        k1.record(stream)
+        torch.cuda.synchronize(device)
+        mean_ms[name] = k0.elapsed_time(k1) / args.steps
     clk = clocks.stop()
     assert int(status.item()) == 0, f"device status {int(status.item())}"
-    per = {name: [events[s][2 * i].elapsed_time(events[s][2 * i + 1]) for s in range(args.steps)]
-           for i, (name, _) in enumerate(kernels)}
-    mean_ms = {k: sum(v) / len(v) for k, v in per.items()}
-    step_ms = sum(mean_ms.values())
     step_ms_max = _max_over_ranks(dist, step_ms, device)
     bf16_ms_max = _max_over_ranks(dist, mean_ms["bf16"], device)
 
@@ -340,7 +350,10 @@ def run_native(args, dist, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes -> bf16 / fp32 accumulate",
             "data": "synthetic", "config": _config(W, spec, chunk),
-            "value_definition": "symbols decoded per second over the step (3 passes of n = 16.8M symbols)",
+            "value_definition": "symbols decoded per second over the step (3 passes of n = 16.8M symbols); "
+                                "K steps back to back between one pair of CUDA events",
+            "kernels_timing": "each kernel alone: K launches back to back (rotating replicas) between one "
+                              "pair of CUDA events, per-launch mean",
             "kernels": kern,
             "bits_per_weight": {"coded": round(info["coded_bits"] / n, 4),
                                 "payload": round(8.0 * info["payload_bytes"] / n, 4),
