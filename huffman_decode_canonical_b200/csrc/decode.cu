@@ -1345,6 +1345,274 @@ __global__ void __launch_bounds__(256) single_kernel(const __grid_constant__ Lau
     }
 }
 
+// ------------------------------------------------------------------ single-stream format, CTA per chunk
+//
+// For chunks of up to kSegChunkSymbols codes: one CTA of kSegThreads threads
+// per chunk, the chunk's words staged in shared memory by one bulk copy.  The
+// chunk's bits [B0, B1) are cut into kSegThreads segments whose inner bounds
+// are multiples of 32 bits.
+//   1. Thread i decodes from the start of its segment until it crosses the
+//      end and marks, in a bitmap of the chunk's bits, where each of its codes
+//      began.  (Thread 0 starts on a code boundary; the others usually not.)
+//   2. A thread whose start differs from where its left neighbour stopped
+//      decodes again from there, but only until it reaches a position it
+//      marked: from a common code boundary the two decodings are the same, so
+//      the rest of its codes are the marked ones (a popcount) and its end
+//      stands.  Rounds repeat until no start changes; Huffman codes
+//      resynchronise within a few codes, so one round of a few codes is usual.
+//   3. A block-wide exclusive scan of the counts places every thread's codes;
+//      each thread decodes them once more into a shared-memory copy of the
+//      chunk's output, which the CTA writes out with coalesced stores.
+
+constexpr int kSegThreads = 256;
+constexpr int kSegChunkSymbols = 16384;
+
+struct SegLayout {
+    size_t words, bitmap, out, ends, counts, wsum, total;
+};
+
+// stage_words: staged words per chunk (a multiple of 4)
+__host__ __device__ inline SegLayout seg_layout(int stage_words, int chunk_symbols) {
+    SegLayout o;
+    size_t p = align_up(smem_layout(0, 0, 0, 0).total, 16);
+    o.words = p;
+    p += (size_t)stage_words * 4;
+    o.bitmap = p;
+    p += (size_t)stage_words * 4;
+    o.out = p;
+    p = align_up(p + (size_t)chunk_symbols, 16);
+    o.ends = p;
+    p += kSegThreads * 8;
+    o.counts = p;
+    p += kSegThreads * 4;
+    o.wsum = p;
+    p += (kSegThreads / 32) * 4;
+    o.total = align_up(p, 16);
+    return o;
+}
+
+struct SegReader {
+    uint32_t base;    // shared address of staged word 0
+    uint64_t bit0;    // stream position of staged word 0
+    uint32_t k;       // next staged word
+    uint32_t hi, lo;  // 64-bit window, MSB first
+    int nb;           // valid bits in the window
+
+    __device__ __forceinline__ uint32_t word(uint32_t i) const { return lds32(base + 4u * i); }
+    __device__ __forceinline__ void seek(uint64_t pos) {
+        const uint32_t rel = static_cast<uint32_t>(pos - bit0);
+        k = rel >> 5;
+        const uint32_t sh = rel & 31;
+        const uint32_t w0 = word(k), w1 = word(k + 1);
+        hi = __funnelshift_l(w1, w0, sh);
+        lo = w1 << sh;
+        nb = 64 - static_cast<int>(sh);
+        k += 2;
+    }
+    // one code; returns its table entry (length | symbol << 8)
+    template <bool SLOW>
+    __device__ __forceinline__ uint32_t next(const Smem &s, int max_len, int32_t *status) {
+        // branch-free refill: word k is always in the staged range (4 words of slack)
+        const bool need = nb <= 32;
+        const uint32_t wv = need ? word(k) : 0u, n = static_cast<uint32_t>(nb);
+        hi |= shr_clamp(wv, n);
+        lo |= shl_clamp(wv, 32u - n);
+        nb += need ? 32 : 0;
+        k += need ? 1u : 0u;
+        uint32_t e = lds32(smem_addr(s.lut) + ((hi >> (32 - kMaxLutBits)) << 2));
+        if (SLOW && (e & 31u) == 0)
+            e = slow_entry((static_cast<uint64_t>(hi) << 32) | lo, max_len, s.slim, s.soffs, s.ssyms, status);
+        const uint32_t len = e & 31u;
+        hi = __funnelshift_l(lo, hi, len);
+        lo <<= len;
+        nb -= static_cast<int>(len);
+        return e;
+    }
+};
+
+template <int BITS, int OUT, bool SLOW>
+__global__ void __launch_bounds__(kSegThreads) segment_kernel(const __grid_constant__ LaunchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const Smem s = carve(smem_raw, 0, 0, 0, 0);
+    const SegLayout L = seg_layout(a.stage_rows, static_cast<int>(a.one.d.chunk_symbols));
+    uint32_t *words = reinterpret_cast<uint32_t *>(smem_raw + L.words);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem_raw + L.bitmap);
+    uint8_t *ostage = smem_raw + L.out;
+    uint64_t *ends = reinterpret_cast<uint64_t *>(smem_raw + L.ends);
+    int *counts = reinterpret_cast<int *>(smem_raw + L.counts);
+    int *wsum = reinterpret_cast<int *>(smem_raw + L.wsum);
+    const GroupEntry &g = a.one;
+    const DevTensor &d = g.d;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long c = blockIdx.x;
+    const uint64_t B0 = d.index[2 * c], B1 = d.index[2 * c + 2];
+    const long long first = static_cast<long long>(d.index[2 * c + 1]);
+    const long long nc = static_cast<long long>(d.index[2 * c + 3]) - first;
+    const uint64_t w0 = (B0 >> 5) & ~3ull;                     // 16-byte aligned start of the copy
+    const uint64_t w1 = (((B1 + 31) >> 5) + 4 + 3) & ~3ull;    // past the chunk's last word, 4 words of slack
+    const bool sane = B1 >= B0 && (B1 + 31) / 32 <= static_cast<uint64_t>(d.payload_words) && nc >= 0 &&
+                      nc <= d.chunk_symbols && w1 - w0 <= static_cast<uint64_t>(a.stage_rows);
+    if (tid == 0) mbar_init(s.tbar, 1);
+    fence_mbar_init();
+    __syncthreads();
+    if (tid == 0) {
+        // tables and the chunk's words on one barrier
+        const uint32_t wbytes = sane ? static_cast<uint32_t>((w1 - w0) * 4) : 0u;
+        uint32_t bytes = kLutSize * 4 + wbytes;
+        if (SLOW) bytes += kSlowBytes;
+        mbar_arrive_expect_tx(s.tbar, bytes);
+        bulk_copy_g2s(s.lut, d.lut, kLutSize * 4, s.tbar);
+        if (SLOW) bulk_copy_g2s(s.slim, d.slow_limit, kSlowBytes, s.tbar);
+        if (wbytes) bulk_copy_g2s(words, d.payload + w0, wbytes, s.tbar);
+    }
+    for (int i = tid; i < a.stage_rows; i += kSegThreads) bitmap[i] = 0u;
+    if (!finish_tables<OUT, SLOW>(g, s, 0)) {
+        set_status(a.status, ENTRO_E_TIMEOUT);
+        return;
+    }
+    if (!sane) {
+        if (tid == 0) set_status(a.status, ENTRO_E_CORRUPT);
+        return;
+    }
+    SegReader rd{smem_addr(words), w0 * 32, 0, 0, 0};
+    const uint64_t span = B1 - B0;
+    auto bound = [&](int i) -> uint64_t {
+        if (i <= 0) return B0;
+        if (i >= kSegThreads) return B1;
+        const uint64_t b = (B0 + span * static_cast<uint64_t>(i) / kSegThreads + 31) & ~31ull;
+        return b < B1 ? b : B1;
+    };
+    const uint64_t seg0 = bound(tid), seg1 = bound(tid + 1);
+    // every code takes at least one bit: a segment never holds more codes than bits
+    const int cap = static_cast<int>(min(static_cast<long long>(seg1 - seg0) + 64, nc + 1));
+
+    // 1. scan from the segment start, marking code starts (bitmap words are this thread's own)
+    int n1 = 0;
+    uint64_t pos = seg0;
+    if (seg0 < seg1) {
+        rd.seek(seg0);
+        // the current bitmap word is stored after every code (no branch)
+        const uint32_t bm = smem_addr(bitmap);
+        uint32_t bwi = 0xFFFFFFFFu, bw = 0u;
+        while (pos < seg1 && n1 < cap) {
+            const uint32_t rel = static_cast<uint32_t>(pos - rd.bit0);
+            const uint32_t wi = rel >> 5;
+            bw = (wi == bwi ? bw : 0u) | (0x80000000u >> (rel & 31));
+            bwi = wi;
+            sts32(bm + 4u * wi, bw);
+            pos += rd.next<SLOW>(s, d.max_len, a.status) & 31u;
+            n1++;
+        }
+    }
+    const uint64_t end1 = pos;
+    uint64_t start = seg0, end = end1;
+    int n = n1;
+    ends[tid] = end1;
+    __syncthreads();
+
+    // 2. resynchronise with the left neighbour
+    bool bad = false;
+    for (int round = 0; round < kSegThreads; round++) {
+        const uint64_t prev = tid == 0 ? B0 : ends[tid - 1];
+        const bool redo = prev != start;
+        __syncthreads();
+        if (redo) {
+            start = prev;
+            if (prev >= seg1) {
+                n = 0;
+                end = prev;
+            } else {
+                rd.seek(prev);
+                uint64_t q = prev;
+                int m = 0;
+                for (;;) {
+                    if (q >= seg1) {
+                        n = m;
+                        end = q;
+                        break;
+                    }
+                    const uint32_t rel = static_cast<uint32_t>(q - rd.bit0);
+                    if ((bitmap[rel >> 5] << (rel & 31)) & 0x80000000u) {
+                        // a code this thread decoded in step 1 starts here: the rest is step 1's
+                        const uint32_t last = static_cast<uint32_t>(seg1 - 1 - rd.bit0) >> 5;
+                        int rest = __popc(bitmap[rel >> 5] & (0xFFFFFFFFu >> (rel & 31)));
+                        for (uint32_t wi = (rel >> 5) + 1; wi <= last; wi++) rest += __popc(bitmap[wi]);
+                        n = m + rest;
+                        end = end1;
+                        break;
+                    }
+                    if (m >= cap) {
+                        bad = true;
+                        n = 0;
+                        end = q;
+                        break;
+                    }
+                    q += rd.next<SLOW>(s, d.max_len, a.status) & 31u;
+                    m++;
+                }
+            }
+            ends[tid] = end;
+        }
+        if (!__syncthreads_or(redo)) break;
+    }
+
+    // 3. place: exclusive scan of the counts over the CTA
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    counts[tid] = n;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kSegThreads / 32; w++) {
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+    }
+    const int p0 = before + incl - n;
+    if (__syncthreads_or(bad) || total != nc || ends[kSegThreads - 1] != B1) {
+        if (tid == 0) set_status(a.status, ENTRO_E_CORRUPT);
+        return;
+    }
+    if (n > 0) {
+        rd.seek(start);
+        for (int j = 0; j < n; j++) ostage[p0 + j] = static_cast<uint8_t>(rd.next<SLOW>(s, d.max_len, a.status) >> 8);
+    }
+    __syncthreads();
+    const int ncodes = static_cast<int>(nc);
+    if (OUT == OUT_BF16) {
+        uint16_t *o16 = reinterpret_cast<uint16_t *>(g.out) + first;
+        if ((first & 1) == 0) {
+            uint32_t *o32 = reinterpret_cast<uint32_t *>(o16);
+            for (int j = tid; 2 * j + 1 < ncodes; j += kSegThreads)
+                o32[j] = (s.vtab[ostage[2 * j]] & 0xFFFFu) | (s.vtab[ostage[2 * j + 1]] << 16);
+            if ((ncodes & 1) && tid == 0) o16[ncodes - 1] = static_cast<uint16_t>(s.vtab[ostage[ncodes - 1]]);
+        } else {
+            for (int j = tid; j < ncodes; j += kSegThreads) o16[j] = static_cast<uint16_t>(s.vtab[ostage[j]]);
+        }
+    } else if (BITS == 8) {
+        uint8_t *o8 = reinterpret_cast<uint8_t *>(g.out) + first;
+        if ((first & 15) == 0) {
+            uint4 *o = reinterpret_cast<uint4 *>(o8);
+            const uint4 *src = reinterpret_cast<const uint4 *>(ostage);
+            for (int j = tid; j < ncodes / 16; j += kSegThreads) o[j] = src[j];
+            for (int j = (ncodes & ~15) + tid; j < ncodes; j += kSegThreads) o8[j] = ostage[j];
+        } else {
+            for (int j = tid; j < ncodes; j += kSegThreads) o8[j] = ostage[j];
+        }
+    } else {
+        // 4-bit: the chunk starts on an even code (checked on the host); code 2j in the low nibble
+        uint8_t *o8 = reinterpret_cast<uint8_t *>(g.out) + (first >> 1);
+        for (int j = tid; 2 * j < ncodes; j += kSegThreads) {
+            const uint32_t hi = 2 * j + 1 < ncodes ? ostage[2 * j + 1] : 0u;
+            o8[j] = static_cast<uint8_t>((ostage[2 * j] & 15u) | (hi << 4));
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 // Message of the last CUDA runtime error the library saw on this host thread.
@@ -1717,9 +1985,40 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
 }
 
+static LanesFn pick_segment(int bits, int out, bool slow) {
+    if (bits == 4) {
+        if (out == OUT_CODES) return slow ? segment_kernel<4, OUT_CODES, true> : segment_kernel<4, OUT_CODES, false>;
+        return slow ? segment_kernel<4, OUT_BF16, true> : segment_kernel<4, OUT_BF16, false>;
+    }
+    if (out == OUT_CODES) return slow ? segment_kernel<8, OUT_CODES, true> : segment_kernel<8, OUT_CODES, false>;
+    return slow ? segment_kernel<8, OUT_BF16, true> : segment_kernel<8, OUT_BF16, false>;
+}
+
 static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t *status, cudaStream_t st) {
     const DevTensor &d = t->d;
     if (d.n_chunks == 0) return ENTRO_OK;
+    DeviceInfo di;
+    if (device_info(t->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
+    // chunks of up to kSegChunkSymbols codes: a CTA per chunk, staged in shared memory
+    const int stage_words = ((d.max_chunk_words + 12) + 3) & ~3;
+    const SegLayout sl = seg_layout(stage_words, static_cast<int>(d.chunk_symbols));
+    if (d.chunk_symbols <= kSegChunkSymbols && (long long)sl.total <= di.smem_optin) {
+        LanesFn fn = pick_segment(d.bits, out_kind, t->slow);
+        int per_sm = 0;
+        if (kernel_config(reinterpret_cast<const void *>(fn), t->device, kSegThreads, sl.total, &per_sm) != ENTRO_OK)
+            return ENTRO_E_CUDA;
+        LaunchArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.one.d = d;
+        a.one.out = out;
+        a.count = 1;
+        a.batch = 1;
+        a.stage_rows = stage_words;
+        a.status = status;
+        fn<<<(unsigned)d.n_chunks, kSegThreads, sl.total, st>>>(a);
+        const cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "segment kernel launch");
+    }
     LanesFn fn = pick_single(d.bits, out_kind, t->slow);
     const size_t bytes = smem_layout(0, 0, 0, 0).total;
     const int threads = 64;  // two chunks per CTA: spreads small tensors over the SMs

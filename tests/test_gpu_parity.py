@@ -100,6 +100,11 @@ SMALL = [
     ("laplace", 4, 2, 12, 1, 4096, 100, 100),
     ("skew", 8, 2, 16, 1, 512, 50, 50),
     ("zeros", 4, 0, 12, 1, 50, 3, 33),
+    ("t4", 8, 2, 16, 1, 16384, 64, 512),      # single stream, chunks at the CTA-per-chunk limit
+    ("t4", 8, 2, 16, 1, 20000, 50, 500),      # single stream above it (warp per chunk), ragged
+    ("skew", 8, 2, 20, 1, 2048, 64, 100),     # single stream, codes longer than 16 bits
+    ("uniform", 8, 2, 16, 1, 4096, 32, 256),  # single stream, ~8 bits per code
+    ("laplace", 4, 2, 12, 1, 1024, 33, 97),   # single stream 4-bit, odd n
     ("laplace", 4, 2, 12, 2, -8192, 129, 64),  # 64 lanes (negative chunk marks them)
     ("laplace", 4, 2, 12, 2, -1024, 7, 333),   # 64 lanes, ragged
     ("t4", 8, 0, 16, 2, -2048, 100, 100),
