@@ -244,6 +244,7 @@ def _config(W, spec, chunk):
 
 def run_native(args, dist, rank, world, local_rank):
     import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -349,7 +350,7 @@ def run_native(args, dist, rank, world, local_rank):
     line = {"metric": METRIC, "value": round(value, 3), "unit": "Gsym/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes -> bf16 / fp32 accumulate",
-            "data": "synthetic", "config": _config(W, spec, chunk),
+            "data": "synthetic", "config": _config(W, spec, chunk), "launch_overlap": not args.no_overlap,
             "value_definition": "symbols decoded per second over the step (3 passes of n = 16.8M symbols); "
                                 "K steps back to back between one pair of CUDA events",
             "kernels_timing": "each kernel alone: K launches back to back (rotating replicas) between one "
@@ -433,6 +434,7 @@ def run_model(args, dist, rank, world, local_rank):
     """One step = one grouped launch over every tensor of a model-shaped workload:
     the fused GEMV of a whole decode step (tok/s) or a whole-model decode to bf16."""
     import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from model_helpers import encode_workload
 
@@ -489,7 +491,8 @@ def run_model(args, dist, rank, world, local_rank):
             "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": f"u{W.bits} codes -> bf16" + (" x bf16 -> fp32" if gemv else ""),
-            "data": "synthetic", "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
+            "data": "synthetic", "launch_overlap": not args.no_overlap,
+            "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
                                             "batch": args.batch if gemv else None,
                                             "l2": "working set larger than L2 (whole model)"},
             "gsym_s": round(n / (ms * 1e-3) / 1e9, 1),
@@ -509,6 +512,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch without overlap (programmatic dependent launch, on by default)")
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "smollm_1p7b_u8", "mistral_7b_u4",
                                                              "phi3_mini_u8"],
                     help="model-scale workloads time one grouped launch per step (not the default line)")

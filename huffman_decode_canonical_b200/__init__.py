@@ -61,7 +61,7 @@ EXPORTS = ["entro_encode", "entro_blob_from_bytes", "entro_blob_bytes", "entro_b
            "entro_device_bytes", "entro_upload", "entro_tensor_free", "entro_decode_codes",
            "entro_decode_dequant_bf16", "entro_decode_gemv", "entro_group_table_bytes", "entro_group_prepare",
            "entro_group_launch", "entro_group_free", "entro_strerror", "entro_version", "entro_last_cuda_error",
-           "entro_decode_gemv_group_static"]
+           "entro_decode_gemv_group_static", "entro_set_overlap"]
 
 
 def _load() -> ctypes.CDLL:
@@ -91,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "entro_version": ([], I32),
         "entro_last_cuda_error": ([], ctypes.c_char_p),
         "entro_decode_gemv_group_static": ([P, P, P, I32, I32, P, P], I32),
+        "entro_set_overlap": ([I32], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -314,7 +315,16 @@ def version() -> int:
     return int(_lib.entro_version())
 
 
-__all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "EXPORTS",
+def set_overlap(enable: bool) -> bool:
+    """Launch overlap (programmatic dependent launch) for every later decode call in this
+    process: a decode may start while the kernel before it on the stream finishes, reading
+    only the tensor's device image until that kernel has completed.  Enable only if no
+    kernel launched right before a decode call writes that tensor's device image.
+    Returns the previous setting."""
+    return bool(_lib.entro_set_overlap(1 if enable else 0))
+
+
+__all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "set_overlap", "EXPORTS",
            "decode_gemv_group_static", "STATIC_GROUP_MAX",
            "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES", "GROUP_GEMV",
            "GROUP_BF16", "SCHEME_UNSIGNED", "SCHEME_ASYM"]

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -99,6 +100,15 @@ struct TensorHandle {
 };
 
 // ------------------------------------------------------------------ device helpers
+
+// Programmatic dependent launch: a launch made with the overlap attribute may
+// start while the kernel before it on the stream is finishing.  A kernel lets
+// the next launch begin at once (it cannot take this kernel's SM resources
+// before they are freed), reads only the tensors' device images before
+// grid_wait_prior(), and touches activations, outputs and the status word only
+// after it.  Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void set_status(int32_t *st, int code) {
     if (st) atomicCAS(st, 0, code);
@@ -273,7 +283,14 @@ __device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int
     mbar_arrive_expect_tx(s.tbar, bytes);
     bulk_copy_g2s(s.lut, multi ? d.mlut : d.lut, kLutSize * 4, s.tbar);
     if (SLOW) bulk_copy_g2s(s.slim, d.slow_limit, kSlowBytes, s.tbar);
-    if (xbytes) bulk_copy_g2s(s.xs, g.x, xbytes, s.tbar);
+}
+
+// The activations' copy, counted on the same barrier by issue_tables; issued
+// after grid_wait_prior(), since the kernel before may be writing them.
+template <int OUT>
+__device__ void issue_x(const GroupEntry &g, const Smem &s, int batch, int x_in_smem) {
+    if (threadIdx.x != 0 || OUT != OUT_GEMV || !x_in_smem) return;
+    bulk_copy_g2s(s.xs, g.x, static_cast<uint32_t>(g.d.cols * batch * 2), s.tbar);
 }
 
 template <int OUT, bool SLOW>
@@ -845,6 +862,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
     }
     if (threadIdx.x == 0) mbar_init(s.tbar, 1);
     fence_mbar_init();
+    grid_launch_dependents();
     __syncthreads();
 
     // this CTA's share: chunks that start inside its symbol range
@@ -890,6 +908,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             pend0 = c < cb;
             pend1 = c + warps < cb;
         }
+        grid_wait_prior();
+        issue_x<OUT>(g, s, a.batch, a.x_in_smem);
         const bool tables_ok = finish_tables<OUT, SLOW>(g, s, tphase);
         tphase++;
         if (!tables_ok) {
@@ -998,6 +1018,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
     }
     if (threadIdx.x == 0) mbar_init(s.tbar, 1);
     fence_mbar_init();
+    grid_launch_dependents();
     __syncthreads();
 
     const long long s0 = a.total_syms * blockIdx.x / gridDim.x;
@@ -1040,6 +1061,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
             pend0 = c < cb;
             pend1 = c + warps < cb;
         }
+        grid_wait_prior();
         const bool tables_ok = finish_tables<OUT_GEMV, SLOW>(g, s, tphase);
         tphase++;
         if (!tables_ok) {
@@ -1266,8 +1288,10 @@ __global__ void __launch_bounds__(256) single_kernel(const __grid_constant__ Lau
     const DevTensor &d = g.d;
     if (threadIdx.x == 0) mbar_init(s.tbar, 1);
     fence_mbar_init();
+    grid_launch_dependents();
     __syncthreads();
     issue_tables<OUT, SLOW>(g, s, false, 1, 0);
+    grid_wait_prior();
     if (!finish_tables<OUT, SLOW>(g, s, 0)) {
         set_status(a.status, ENTRO_E_TIMEOUT);
         return;
@@ -1454,6 +1478,7 @@ __global__ void __launch_bounds__(kSegThreads) segment_kernel(const __grid_const
                       nc <= d.chunk_symbols && w1 - w0 <= static_cast<uint64_t>(a.stage_rows);
     if (tid == 0) mbar_init(s.tbar, 1);
     fence_mbar_init();
+    grid_launch_dependents();
     __syncthreads();
     if (tid == 0) {
         // tables and the chunk's words on one barrier
@@ -1466,6 +1491,7 @@ __global__ void __launch_bounds__(kSegThreads) segment_kernel(const __grid_const
         if (wbytes) bulk_copy_g2s(words, d.payload + w0, wbytes, s.tbar);
     }
     for (int i = tid; i < a.stage_rows; i += kSegThreads) bitmap[i] = 0u;
+    grid_wait_prior();
     if (!finish_tables<OUT, SLOW>(g, s, 0)) {
         set_status(a.status, ENTRO_E_TIMEOUT);
         return;
@@ -1912,6 +1938,29 @@ static int kernel_config(const void *fn, int device, int threads, size_t bytes, 
     return ENTRO_OK;
 }
 
+// Launch overlap (programmatic dependent launch), off unless the caller turns it on.
+static std::atomic<int> g_overlap{0};
+
+static cudaError_t launch(LanesFn fn, unsigned grid, unsigned threads, size_t smem, cudaStream_t st,
+                          const LaunchArgs &a) {
+    if (!g_overlap.load(std::memory_order_relaxed)) {
+        fn<<<grid, threads, smem, st>>>(a);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, a);
+}
+
 static int bpad_for(int batch) {
     int b = 1;
     while (b < batch) b <<= 1;
@@ -1980,8 +2029,7 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     a.x_elems = x_elems;
     a.total_syms = total;
     a.status = status;
-    fn<<<(unsigned)grid, warps * 32, bytes, st>>>(a);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch(fn, (unsigned)grid, warps * 32, bytes, st, a);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
 }
 
@@ -2015,8 +2063,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
         a.batch = 1;
         a.stage_rows = stage_words;
         a.status = status;
-        fn<<<(unsigned)d.n_chunks, kSegThreads, sl.total, st>>>(a);
-        const cudaError_t e = cudaGetLastError();
+        const cudaError_t e = launch(fn, (unsigned)d.n_chunks, kSegThreads, sl.total, st, a);
         return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "segment kernel launch");
     }
     LanesFn fn = pick_single(d.bits, out_kind, t->slow);
@@ -2033,8 +2080,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
     a.batch = 1;
     a.status = status;
     const long long grid = (d.n_chunks * 32 + threads - 1) / threads;
-    fn<<<(unsigned)grid, threads, bytes, st>>>(a);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch(fn, (unsigned)grid, threads, bytes, st, a);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "single kernel launch");
 }
 
@@ -2261,5 +2307,7 @@ extern "C" const char *entro_strerror(int code) {
 }
 
 extern "C" int entro_version(void) { return 100; }
+
+extern "C" ENTRO_API int entro_set_overlap(int enable) { return entro::g_overlap.exchange(enable ? 1 : 0); }
 
 extern "C" const char *entro_last_cuda_error(void) { return g_cuda_msg; }

@@ -203,6 +203,20 @@ ENTRO_API int entro_decode_gemv_group_static(const entro_tensor *const *tensors,
                                              float *const *ys, int32_t count, int32_t batch, int32_t *d_status,
                                              void *stream);
 
+/* Launch overlap (not in the pages: a B200 launch option).  When enabled,
+ * every decode launch (single tensor, group, static group) is made with
+ * programmatic dependent launch: it may start while the kernel launched just
+ * before it on the same stream is still finishing, and overlaps that kernel's
+ * tail with its own start-up (chunk index, tables and first coded words
+ * fetched from device memory).  Before the previous kernel has completed, a
+ * decode kernel reads only the tensor's device image (tables, index, coded
+ * words); activations, outputs and the status word are touched only after it
+ * has completed, as without overlap.  Enable it only if no kernel launched
+ * right before a decode call on the same stream writes that tensor's device
+ * image (copies, such as entro_upload's, are always waited for).  Process-
+ * wide; off by default.  Returns the previous setting. */
+ENTRO_API int entro_set_overlap(int enable);
+
 /* Text of the last CUDA runtime error behind an ENTRO_E_CUDA return on the
  * calling host thread ("" if none). */
 ENTRO_API const char *entro_last_cuda_error(void);
