@@ -1968,6 +1968,7 @@ static int bpad_for(int batch) {
 }
 
 static constexpr long long kXSmemElems = 48 * 1024;  // up to 96 KB of bf16 activations per CTA
+static constexpr long long kXL1Bytes = 16 * 1024;    // activations that grouped launches read through L1
 
 // Launch the lanes kernel over `count` entries (table on device, or `one`).
 static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
@@ -1991,7 +1992,16 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     const int bpad = out_kind == OUT_GEMV ? bpad_for(batch) : 1;
     bool mma = out_kind == OUT_GEMV && bpad >= kTileBatch;
     for (int i = 0; mma && i < count; i++) mma = mma_eligible(ts[i]->d);
-    long long x_elems = (out_kind == OUT_GEMV && !mma && max_kb <= kXSmemElems) ? max_kb : 0;
+    // Activations in shared memory (one bulk copy per tensor per CTA) for a
+    // single tensor, or when they are too large to stay in the L1 left beside
+    // the staging buffers (over 16 KB); a grouped launch over tensors with
+    // small activations reads them through L1 instead of copying them for
+    // every tensor a CTA touches (Phi-3-shaped step -3 %, one 4096-column
+    // tensor +7 % if read through L1).
+    long long x_elems = (out_kind == OUT_GEMV && !mma && max_kb <= kXSmemElems &&
+                         (count == 1 || max_kb * 2 > kXL1Bytes))
+                            ? max_kb
+                            : 0;
     const int stage_rows = max_words + kSlackRows;
     // the run ring: kRing runs of 8 codes per lane (padded for the tensor-core GEMV's cross-warp reads)
     const int out_words = mma ? tile_ring_words(bits, lanes) : kRing * lanes * bits / 4;
