@@ -44,6 +44,7 @@ import workloads  # noqa: E402
 METRIC = "decoded Gsym/s and % HBM roofline (Huffman decode+dequant); fused GEMV tok/s"
 WORKLOAD = "laplace_4096x4096_u4"
 REPLICAS = 40
+NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e, HGX figure (context beside the measured copy peak)
 
 
 def _peaks():
@@ -339,7 +340,8 @@ def run_native(args, dist, rank, world, local_rank):
     achieved = alg["bf16"] / (bf16_ms_max * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "lanes_kernel<4, bf16> (decode + dequant to bf16)",
                 "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": _traffic("bf16")}
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": _traffic("bf16"),
+                "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4)}
 
     e2e = _e2e(entro, blob, dt, device, stream, args, n, codes[0], bf[0], x, y[0], status)
     e2e["value"] = _max_over_ranks(dist, -e2e["value"], device) * -1 if dist is not None else e2e["value"]
