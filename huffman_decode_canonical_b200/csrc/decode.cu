@@ -1121,12 +1121,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
                 if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, a.status);
-                __syncthreads();  // the block's runs of every row are in the rings
                 const int col0 = (tb % spr) * (kRun * LANES);
                 // The warp's groups q = warp, warp + warps, ... two per pass; the x
-                // fragments of the next pass are loaded (from L2) while this pass
-                // multiplies.  A = rows gid and gid + 8 of the group (the code
-                // rings of those warps), B = x^T of batch rows 8 nb + gid.
+                // fragments of the first pass are loaded (from L2) before the
+                // barrier, those of the next pass while this pass multiplies.
+                // A = rows gid and gid + 8 of the group (the code rings of those
+                // warps), B = x^T of batch rows 8 nb + gid.
                 const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
                 const uint32_t *ring_lo = s.ostage + static_cast<size_t>(gid) * a.out_words;
                 const uint32_t *ring_hi = s.ostage + static_cast<size_t>(gid + 8) * a.out_words;
@@ -1142,6 +1142,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                 uint4 xc[2][NB];
                 xload(warp, xc[0]);
                 xload(warp + warps, xc[1]);
+                __syncthreads();  // the block's runs of every row are in the rings
                 for (int q0 = warp; q0 < groups; q0 += 2 * warps) {
                     uint4 xn[2][NB];
                     xload(q0 + 2 * warps, xn[0]);
