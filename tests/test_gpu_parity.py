@@ -241,6 +241,7 @@ def test_corrupt_device_data_sets_status_without_hanging(entro):
     info = dt.info
     payload_off = dt.mem.numel() - ((info["payload_bytes"] + 4 * 64 + 255) // 256) * 256
     dt.mem[payload_off: payload_off + info["payload_bytes"]] = 0xFF
+    torch.cuda.synchronize()  # a device image changes only between decode launches (launch overlap contract)
     st = _status()
     dt.decode_codes(status=st)
     torch.cuda.synchronize()
@@ -253,6 +254,7 @@ def test_corrupt_device_data_sets_status_without_hanging(entro):
     gen = torch.Generator(device="cuda").manual_seed(0)
     dt.mem[payload_off: payload_off + info["payload_bytes"]] = torch.randint(
         0, 256, (info["payload_bytes"],), dtype=torch.uint8, device="cuda", generator=gen)
+    torch.cuda.synchronize()
     st = _status()
     dt.decode_dequant_bf16(status=st)
     torch.cuda.synchronize()
