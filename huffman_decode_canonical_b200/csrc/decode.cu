@@ -339,13 +339,16 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
 }
 
 // Runs are staged in a ring of kRing slots per lane: a warp emits every
-// kEmitBlock runs, and a lane writes at most kLookupsPerCheck - 1 slots beyond
-// the block it is decoding, so kRing >= kEmitBlock + kLookupsPerCheck - 1
-// keeps the slots being emitted apart from the slots being written.
+// kEmitBlock runs; a lane may decode up to kLookahead runs into the next block
+// while the warp waits for its slowest lane, and writes at most
+// kLookupsPerCheck - 1 slots beyond where it stops, so kRing >= kEmitBlock +
+// kLookahead + kLookupsPerCheck - 1 keeps the slots being emitted apart from
+// the slots being written.
 constexpr int kEmitBlock = 8;
 constexpr int kRing = 16;
 constexpr int kLookupsPerCheck = 4;  // lanes kernel: table lookups between two checks of a lane's run count
-static_assert(kRing >= kEmitBlock + kLookupsPerCheck - 1, "ring too small for the decode overshoot");
+constexpr int kLookahead = 4;        // lanes kernel: runs a lane may decode ahead into the next block
+static_assert(kRing >= kEmitBlock + kLookahead + kLookupsPerCheck - 1, "ring too small for the decode overshoot");
 
 // Shifts that give 0 for a shift of 32 (PTX clamps the amount to the width).
 __device__ __forceinline__ uint32_t shl_clamp(uint32_t v, uint32_t n) {
@@ -706,19 +709,24 @@ __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, 
     }
 }
 
-// Advance every format lane the thread serves to run te (whole runs), STEPS
-// (2 or 4) lookups per check.  A lane may write up to STEPS - 1 slots past the
-// block before it stops (and reads past its last word by as many lookups,
-// which the staging slack covers).
+// Advance every format lane the thread serves to at least run te (whole
+// runs), STEPS (2 or 4) lookups per check, until every lane of the warp has
+// reached te.  Meanwhile a lane that is ahead keeps decoding up to run cap
+// (>= te): work of the next block instead of idling while the warp's slowest
+// lane finishes.  A lane may write up to STEPS - 1 slots past where it stops
+// (and read past its last word by as many lookups, which the staging slack
+// covers).
 template <int STEPS, int BITS, bool SLOW, int LANES, int LPT>
 __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[LPT], const Smem &s, int te,
-                                          int max_len, bool refill_each, int32_t *status) {
-    bool more = true;
-    while (more) {
-        more = false;
+                                          int cap, int max_len, bool refill_each, int32_t *status) {
+    for (;;) {
+        bool behind = false;
+#pragma unroll
+        for (int k = 0; k < LPT; k++) behind = behind || ld[k].t < te;
+        if (!__any_sync(0xffffffffu, behind)) break;
 #pragma unroll
         for (int k = 0; k < LPT; k++) {
-            if (ld[k].t < te) {
+            if (ld[k].t < cap) {
 #pragma unroll
                 for (int h = 0; h < STEPS / 2; h++) {
                     ld[k].refill();
@@ -726,7 +734,6 @@ __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[L
                     if (SLOW && refill_each) ld[k].refill();
                     ld[k].step(s, max_len, status);
                 }
-                more = more || ld[k].t < te;
             }
         }
     }
@@ -775,7 +782,8 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
                                          : 0;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
-            decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, status);
+            // a lane may run up to kLookahead runs into the next block, never past the chunk
+            decode_to<kLookupsPerCheck>(ld, s, te, te < runs ? te + kLookahead : te, d.max_len, refill_each, status);
             __syncwarp();
             emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc, gst, grow);
             __syncwarp();  // the ring slots just read are rewritten by the next block
@@ -1120,7 +1128,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                 for (int i = 0; i < 4; i++) acc[nb][i] = 0.f;
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
-                if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, d.max_len, refill_each, a.status);
+                if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, te, d.max_len, refill_each, a.status);
                 const int col0 = (tb % spr) * (kRun * LANES);
                 // The warp's groups q = warp, warp + warps, ... two per pass; the x
                 // fragments of the first pass are loaded (from L2) before the
