@@ -338,17 +338,21 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(lo), "r"(hi) : "memory");
 }
 
-// Runs are staged in a ring of kRing slots per lane: a warp emits every
-// kEmitBlock runs; a lane may decode up to kLookahead runs into the next block
-// while the warp waits for its slowest lane, and writes at most
-// kLookupsPerCheck - 1 slots beyond where it stops, so kRing >= kEmitBlock +
-// kLookahead + kLookupsPerCheck - 1 keeps the slots being emitted apart from
-// the slots being written.
+// Runs are staged in a ring of kRing slots per lane; the slot of run t is
+// written while run t is being assembled.  A check of a lane's progress is
+// followed by kLookupsPerCheck lookups of at most kMaxCodesPerLookup codes
+// each, which, with at most kRun - 1 codes pending, complete at most
+// kRunsPerCheck runs.  The lanes kernel emits every kEmitBlock runs and lets a
+// lane decode up to kLookahead runs into the next block, so the slots in use
+// while a block waits to be emitted are kEmitBlock + kLookahead +
+// kRunsPerCheck <= kRing.
 constexpr int kEmitBlock = 8;
 constexpr int kRing = 16;
-constexpr int kLookupsPerCheck = 4;  // lanes kernel: table lookups between two checks of a lane's run count
-constexpr int kLookahead = 4;        // lanes kernel: runs a lane may decode ahead into the next block
-static_assert(kRing >= kEmitBlock + kLookahead + kLookupsPerCheck - 1, "ring too small for the decode overshoot");
+constexpr int kLookupsPerCheck = 4;    // table lookups between two checks of a lane's run count
+constexpr int kMaxCodesPerLookup = 6;  // multi-symbol table: up to 6 4-bit or 3 8-bit codes per entry
+constexpr int kRunsPerCheck = (kRun - 1 + kLookupsPerCheck * kMaxCodesPerLookup) / kRun;
+constexpr int kLookahead = 4;          // lanes kernel: runs a lane may decode ahead into the next block
+static_assert(kRing >= kEmitBlock + kLookahead + kRunsPerCheck, "ring too small for the decode overshoot");
 
 // Shifts that give 0 for a shift of 32 (PTX clamps the amount to the width).
 __device__ __forceinline__ uint32_t shl_clamp(uint32_t v, uint32_t n) {
@@ -972,7 +976,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 //   B = x^T[16 columns, 8 batch rows] (1 or 2 tiles)    from global memory (L2)
 //   D = y partials [16 rows, 8 batch rows]              registers, per warp
 // Each lockstep block covers E runs of every chunk (E divides the runs of a
-// row; E plus the kLookupsPerCheck - 1 slots a lane may write past it fit the
+// row; E plus the kRunsPerCheck slots a lane may write past it fit the
 // ring); after a CTA barrier the block's columns are split among the warps in
 // groups of 32 (4 format lanes x 8 weights).  The k order inside an MMA is
 // permuted so that each thread's A registers are the 8 weights of one ring
@@ -983,7 +987,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 // end (fixed order: the result does not depend on timing).  For a batch of up
 // to 8 one MMA covers 256 weights.
 
-constexpr int kTileMaxBlock = kRing - kLookupsPerCheck + 1;  // a block plus the slots a lane may write past it fit the ring
+constexpr int kTileMaxBlock = kRing - kRunsPerCheck;  // a block plus the slots a lane may write past it fit the ring
 constexpr int kTileBatch = 4;             // padded batch from which the tensor-core GEMV runs
 
 // Runs per lockstep block: the largest divisor of the runs per row that fits the ring.
@@ -1706,7 +1710,7 @@ static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lu
         }
     }
     *n_codes = nz;
-    const int per = bits == 4 ? 6 : 3;
+    const int per = bits == 4 ? kMaxCodesPerLookup : kMaxCodesPerLookup / 2;
     for (uint32_t v = 0; v < (uint32_t)kLutSize; v++) {
         uint32_t used = 0, k = 0, packed = 0;
         while ((int)k < per) {
