@@ -368,11 +368,17 @@ def run_native(args, dist, rank, world, local_rank):
 
 
 def _kernel_source_hash() -> str:
+    """Hash of the kernel sources with comments and whitespace removed (a comment edit
+    does not change the kernels whose traffic profiles/traffic.json records)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in ("huffman_decode_canonical_b200/csrc/decode.cu", "huffman_decode_canonical_b200/csrc/blob_format.h"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

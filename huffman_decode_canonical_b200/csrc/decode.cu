@@ -410,7 +410,8 @@ struct LaneDecoder {
         if (need) wnext = lds32(min(bufa, bufcap));
     }
 
-    // one table lookup; appends its codes to the pending bit string
+    // One table lookup that only appends its codes to the pending bit string
+    // (no slot store): the tail of a partial last run, closed by close_run().
     __device__ __forceinline__ void lookup(const Smem &s, int max_len, int32_t *status) {
         const uint32_t e = lds32(lut + ((hi >> (32 - kMaxLutBits)) << 2));
         uint32_t syms = e >> 8, bits = e & 15u;
@@ -438,11 +439,11 @@ struct LaneDecoder {
         pb += add;
     }
 
-    // One table lookup and its run bookkeeping (the fast path of lookup() +
-    // emit()).  The window shift, the append of the entry's codes to the
-    // pending string, the slot store and the run completion are one block of
-    // hand-written PTX; a miss in the table (a code longer than 12 bits) goes
-    // through the canonical slow path and re-enters as a one-code entry.
+    // One table lookup and its run bookkeeping.  The window shift, the append
+    // of the entry's codes to the pending string, the slot store and the run
+    // completion are one block of hand-written PTX; a miss in the table (a
+    // code longer than 12 bits) goes through the canonical slow path and
+    // re-enters as a one-code entry.
     __device__ __forceinline__ void step(const Smem &s, int max_len, int32_t *status) {
         uint32_t e = lds32(lut + ((hi >> (32 - kMaxLutBits)) << 2));
         uint32_t bits = e & 15u;
