@@ -438,6 +438,70 @@ def _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status):
                     "three decodes, results copied to pinned host memory; wall clock per step"}
 
 
+def run_single_stream(args, dist, rank, world, local_rank):
+    """The 1024x1024 8-bit tensor in the one-bitstream-per-chunk format (4096-symbol
+    chunks): one step = decode to uint8 codes + decode to bf16, 40 rotating replicas."""
+    import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    W = workloads.get(args.workload)
+    spec = W.tensors[0]
+    w = workloads.weights(W, spec).numpy()
+    blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
+                             chunk_symbols=W.chunk_symbols(spec.cols), lanes=W.lanes)
+    info = blob.info()
+    reps = [entro.upload(blob, device=device) for _ in range(REPLICAS)]
+    codes = [r.empty_codes() for r in reps]
+    bf = [r.empty_bf16() for r in reps]
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    counter = [0]
+
+    def step():
+        for fn in (lambda r: reps[r].decode_codes(out=codes[r], status=status),
+                   lambda r: reps[r].decode_dequant_bf16(out=bf[r], status=status)):
+            fn(counter[0] % REPLICAS)
+            counter[0] += 1
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0  # burn-in so that clock samples cover a loaded GPU
+    while time.perf_counter() < t_end:
+        step()
+        torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(dist, device)
+    torch.cuda.synchronize(device)
+    torch.cuda._sleep(int(args.steps * 200e-6 * 2.0e9))
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    _barrier(dist, device)
+    clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    step_ms = _max_over_ranks(dist, ev0.elapsed_time(ev1) / args.steps, device)
+    if rank != 0:
+        return 0
+    n = info["n"]
+    line = {"metric": METRIC, "value": round(world * 2 * n / (step_ms * 1e-3) / 1e9, 3), "unit": "Gsym/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes -> bf16",
+            "data": "synthetic", "launch_overlap": not args.no_overlap,
+            "config": {"workload": W.name, "rows": spec.rows, "cols": spec.cols, "format": "single stream",
+                       "chunk_symbols": W.chunk_symbols(spec.cols), "replicas": REPLICAS},
+            "value_definition": "symbols decoded per second over the step (decode to codes + decode to bf16)",
+            "bits_per_weight": {"coded": round(info["coded_bits"] / n, 4)},
+            "gpu_launches": 2 * args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_model(args, dist, rank, world, local_rank):
     """One step = one grouped launch over every tensor of a model-shaped workload:
     the fused GEMV of a whole decode step (tok/s) or a whole-model decode to bf16."""
@@ -522,9 +586,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch without overlap (programmatic dependent launch, on by default)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "smollm_1p7b_u8", "mistral_7b_u4",
-                                                             "phi3_mini_u8"],
-                    help="model-scale workloads time one grouped launch per step (not the default line)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "t4_1024x1024_u8", "smollm_1p7b_u8",
+                                                             "mistral_7b_u4", "phi3_mini_u8"],
+                    help="other workloads (not the default line): the 1024x1024 single-stream tensor, or "
+                         "model-scale workloads timed as one grouped launch per step")
     ap.add_argument("--batch", type=int, default=1, help="GEMV batch for the model-scale GEMV workloads")
     ap.add_argument("--tensors", type=int, default=0, help="model-scale workloads: only the first N tensors")
     args = ap.parse_args(argv)
@@ -534,6 +599,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.workload == "t4_1024x1024_u8":
+            return run_single_stream(args, dist, rank, world, local_rank)
         if args.workload != WORKLOAD:
             return run_model(args, dist, rank, world, local_rank)
         return run_native(args, dist, rank, world, local_rank)
