@@ -65,7 +65,7 @@ extern "C" {
 /* Chunk formats (EntroLLM technical summary, parallel decoding over chunks;
  * LazyWeights abstract, interleaved lanes). */
 #define ENTRO_FORMAT_SINGLE 1 /* one bitstream per chunk, chunks bit-contiguous */
-#define ENTRO_FORMAT_LANES 2  /* 32 word-interleaved lane bitstreams per chunk */
+#define ENTRO_FORMAT_LANES 2  /* 32 (or 64) word-interleaved lane bitstreams per chunk */
 
 typedef struct entro_encode_opts {
     int32_t bits;          /* 4 or 8 */
@@ -150,8 +150,11 @@ ENTRO_API int entro_decode_dequant_bf16(const entro_tensor *t, void *d_out, int3
  * weights of entro_decode_dequant_bf16 (never written to memory), x bf16
  * [batch, cols], accumulation in fp32.  Needs the lanes format, cols a
  * multiple of 8 * lanes (256 or 512) and chunk_symbols a multiple of cols
- * (chunks of whole rows); batch in 1..16; d_x 16-byte aligned.  Rows are reduced in a fixed
- * order, so results are bit-reproducible. */
+ * (chunks of whole rows); batch in 1..16; d_x 16-byte aligned.  Batch 1-2:
+ * fp32 FMAs of the bf16 products in the decoding warp; batch 3-16: the
+ * tensor cores (mma.sync, bf16 operands, fp32 accumulation) with the warps of
+ * a block decoding consecutive rows.  Rows are reduced in a fixed order, so
+ * results are bit-reproducible. */
 ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t batch, float *d_y,
                       int32_t *d_status, void *stream);
 
@@ -164,7 +167,8 @@ ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t 
  * entro_group_launch then launches without any host-device traffic, as often
  * as wanted (for instance once per generated token).  d_table, the tensors'
  * device images and the x / y / output buffers must stay valid while the
- * handle is used; all tensors must share the bit width.  kind:
+ * handle is used; all tensors must share the bit width and the lane count.
+ * kind:
  *   ENTRO_GROUP_GEMV  xs[i] bf16 [batch, cols_i], ys[i] fp32 [batch, rows_i]
  *                     (the per-tensor rules of entro_decode_gemv apply)
  *   ENTRO_GROUP_BF16  outs[i] bf16 [rows_i, cols_i] (lanes format only) */
