@@ -48,10 +48,10 @@ constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
 constexpr int kSlackRows = 2;                 // staging rows past a chunk's longest lane (read-ahead)
 // A lane's window may run past its last word by the lookups made after its last
-// run completes (up to 3 of at most 24 bits, plus the word loaded one ahead):
+// run completes (up to 5 of at most 24 bits, plus the word loaded one ahead):
 // reads stay inside the staging buffer (clamped); a lane that moved more than
 // this many rows past its words has decoded a corrupt stream.
-constexpr int kOverrunRows = 5;
+constexpr int kOverrunRows = 7;
 
 enum OutKind { OUT_CODES = 0, OUT_BF16 = 1, OUT_GEMV = 2 };
 
@@ -348,11 +348,15 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t lo, uint32_t hi) {
 // kRunsPerCheck <= kRing.
 constexpr int kEmitBlock = 8;
 constexpr int kRing = 16;
-constexpr int kLookupsPerCheck = 4;    // table lookups between two checks of a lane's run count
 constexpr int kMaxCodesPerLookup = 6;  // multi-symbol table: up to 6 4-bit or 3 8-bit codes per entry
-constexpr int kRunsPerCheck = (kRun - 1 + kLookupsPerCheck * kMaxCodesPerLookup) / kRun;
-constexpr int kLookahead = 4;          // lanes kernel: runs a lane may decode ahead into the next block
+__host__ __device__ constexpr int runs_per_check(int lookups) {
+    return (kRun - 1 + lookups * kMaxCodesPerLookup) / kRun;
+}
+constexpr int kLookupsPerCheck = 6;    // lanes kernel: table lookups between two checks of a lane's run count
+constexpr int kRunsPerCheck = runs_per_check(kLookupsPerCheck);
+constexpr int kLookahead = 3;          // lanes kernel: runs a lane may decode ahead into the next block
 static_assert(kRing >= kEmitBlock + kLookahead + kRunsPerCheck, "ring too small for the decode overshoot");
+constexpr int kTileLookupsPerCheck = 4;  // tensor-core GEMV kernel (longer lockstep blocks fit the ring)
 
 // Shifts that give 0 for a shift of 32 (PTX clamps the amount to the width).
 __device__ __forceinline__ uint32_t shl_clamp(uint32_t v, uint32_t n) {
@@ -715,12 +719,12 @@ __device__ __forceinline__ void emit_ragged(const GroupEntry &g, const Smem &s, 
 }
 
 // Advance every format lane the thread serves to at least run te (whole
-// runs), STEPS (2 or 4) lookups per check, until every lane of the warp has
-// reached te.  Meanwhile a lane that is ahead keeps decoding up to run cap
-// (>= te): work of the next block instead of idling while the warp's slowest
-// lane finishes.  A lane may write up to STEPS - 1 slots past where it stops
-// (and read past its last word by as many lookups, which the staging slack
-// covers).
+// runs), STEPS lookups per check, until every lane of the warp has reached
+// te.  Meanwhile a lane that is ahead keeps decoding up to run cap (>= te):
+// work of the next block instead of idling while the warp's slowest lane
+// finishes.  A lane may complete up to runs_per_check(STEPS) runs past the
+// check that stops it, and read past its last word by up to STEPS - 1
+// lookups (clamped to the staging buffer).
 template <int STEPS, int BITS, bool SLOW, int LANES, int LPT>
 __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[LPT], const Smem &s, int te,
                                           int cap, int max_len, bool refill_each, int32_t *status) {
@@ -977,7 +981,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 //   B = x^T[16 columns, 8 batch rows] (1 or 2 tiles)    from global memory (L2)
 //   D = y partials [16 rows, 8 batch rows]              registers, per warp
 // Each lockstep block covers E runs of every chunk (E divides the runs of a
-// row; E plus the kRunsPerCheck slots a lane may write past it fit the
+// row; E plus the runs a lane may complete after its last check fit the
 // ring); after a CTA barrier the block's columns are split among the warps in
 // groups of 32 (4 format lanes x 8 weights).  The k order inside an MMA is
 // permuted so that each thread's A registers are the 8 weights of one ring
@@ -988,7 +992,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
 // end (fixed order: the result does not depend on timing).  For a batch of up
 // to 8 one MMA covers 256 weights.
 
-constexpr int kTileMaxBlock = kRing - kRunsPerCheck;  // a block plus the slots a lane may write past it fit the ring
+constexpr int kTileMaxBlock = kRing - runs_per_check(kTileLookupsPerCheck);  // a block plus the slots a lane may write past it fit the ring
 constexpr int kTileBatch = 4;             // padded batch from which the tensor-core GEMV runs
 
 // Runs per lockstep block: the largest divisor of the runs per row that fits the ring.
@@ -1133,7 +1137,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
                 for (int i = 0; i < 4; i++) acc[nb][i] = 0.f;
             for (int tb = 0; tb < runs; tb += E) {
                 const int te = tb + E;
-                if (active && tb < my_runs) decode_to<kLookupsPerCheck>(ld, s, te, te, d.max_len, refill_each, a.status);
+                if (active && tb < my_runs) decode_to<kTileLookupsPerCheck>(ld, s, te, te, d.max_len, refill_each, a.status);
                 const int col0 = (tb % spr) * (kRun * LANES);
                 // The warp's groups q = warp, warp + warps, ... two per pass; the x
                 // fragments of the first pass are loaded (from L2) before the
