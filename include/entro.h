@@ -208,8 +208,9 @@ ENTRO_API int entro_decode_gemv_group_static(const entro_tensor *const *tensors,
                                              void *stream);
 
 /* Launch overlap (not in the pages: a B200 launch option).  When enabled,
- * decode launches that fill each SM with one CTA (the lanes-format kernels on
- * tensors large enough for it) are made with programmatic dependent launch:
+ * decode launches that fill each SM with one or two large CTAs (the lanes-
+ * format kernels on tensors large enough for it) are made with programmatic
+ * dependent launch:
  * such a launch may start while the kernel launched just
  * before it on the same stream is still finishing, and overlaps that kernel's
  * tail with its own start-up (chunk index, tables and first coded words
