@@ -184,7 +184,9 @@ def cpu_baseline(seconds: float = 12.0):
     W = workloads.get(WORKLOAD)
     spec = W.tensors[0]
     w = workloads.weights(W, spec).numpy()
+    t_enc = time.perf_counter()
     blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols))
+    t_enc = time.perf_counter() - t_enc
     p = oracle.params(blob)
     x_bits = workloads.bf16_bits(workloads.activations(0, 1, spec.cols))
     threads = max(1, min(os.cpu_count() or 1, 64))
@@ -196,10 +198,23 @@ def cpu_baseline(seconds: float = 12.0):
         if time.perf_counter() - t0 >= seconds or reps >= 8:
             break
     dt = time.perf_counter() - t0
+    # one thread on a 1/32 sample of the chunks (the sequential decoder's rate)
+    sample1 = (0, max(1, n_chunks // 32))
+    total1, t1, reps1 = 0, time.perf_counter(), 0
+    while True:
+        total1 += _oracle_step(blob, sample1, 1, x_bits)
+        reps1 += 1
+        if time.perf_counter() - t1 >= seconds / 4 or reps1 >= 4:
+            break
+    dt1 = time.perf_counter() - t1
     return {"value": total / dt / 1e9, "unit": "Gsym/s", "cores": threads, "kind": "oracle",
             "sample": f"{reps} pass(es) of the whole {spec.rows}x{spec.cols} tensor "
                       f"({n_chunks} chunks; codes, bf16 and GEMV passes), chunk ranges over {threads} threads, "
-                      f"{dt:.1f} s"}
+                      f"{dt:.1f} s",
+            "single_thread": {"value": total1 / dt1 / 1e9, "unit": "Gsym/s", "cores": 1,
+                              "sample": f"{reps1} pass(es) of chunks {sample1[0]}..{sample1[1]} "
+                                        f"(codes, bf16 and GEMV passes), {dt1:.1f} s"},
+            "oracle_encode_s": round(t_enc, 3)}
 
 
 def run_reference(args, rank, world):
