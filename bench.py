@@ -345,18 +345,21 @@ def run_native(args, dist, rank, world, local_rank):
     alg = {"codes": coded + index + dt.codes_nbytes(), "bf16": coded + index + 2.0 * n,
            "gemv": coded + index + 2.0 * spec.cols + 4.0 * spec.rows}
     peak, peak_kind = _peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     kern = {}
     for k in mean_ms:
         us = 1e3 * mean_ms[k]
         gbs = alg[k] / (mean_ms[k] * 1e-3) / 1e9
         kern[k] = {"us": round(us, 3), "gsym_s": round(n / (mean_ms[k] * 1e-3) / 1e9, 2),
-                   "alg_bytes": int(alg[k]), "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4)}
+                   "alg_bytes": int(alg[k]), "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4),
+                   "issue_bound": _issue_ceiling(k, n, mean_ms[k], clk.get("sm_mhz"), sms)}
     kern["gemv"]["tok_s"] = round(1.0 / (mean_ms["gemv"] * 1e-3), 1)
     achieved = alg["bf16"] / (bf16_ms_max * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "lanes_kernel<4, bf16> (decode + dequant to bf16)",
                 "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": _traffic("bf16"),
-                "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4)}
+                "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                "issue_bound": kern["bf16"]["issue_bound"]}
 
     e2e = _e2e(entro, blob, dt, device, stream, args, n, codes[0], bf[0], x, y[0], status)
     e2e["value"] = _max_over_ranks(dist, -e2e["value"], device) * -1 if dist is not None else e2e["value"]
@@ -397,18 +400,40 @@ def _kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def _traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when the
-    summary was taken on other kernel sources (profiles/traffic.json records their hash)."""
+def _profile_record(key: str, kernel: str):
+    """A per-launch figure of `kernel` (`key`: "kernels" = DRAM bytes, "warp_inst" = warp
+    instructions) from the committed ncu summary, or None when the summary was taken on
+    other kernel sources (profiles/traffic.json records their hash)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
         if t.get("source_sha256_16") != _kernel_source_hash():
             return None
-        return t["kernels"].get(kernel)
+        return t[key].get(kernel)
     except Exception:
         return None
+
+
+def _traffic(kernel: str):
+    return _profile_record("kernels", kernel)
+
+
+def _issue_ceiling(kernel: str, n: int, ms: float, sm_mhz, sms: int):
+    """The instruction-issue bound of a decode kernel: every SM scheduler issues one warp
+    instruction per clock, so with I warp instructions per launch (ncu
+    smsp__inst_executed.sum) the launch takes at least I / (4 * SMs * clock).  Reported
+    as symbols/s at that bound and the fraction of it achieved; None without a record
+    for these kernel sources."""
+    inst = _profile_record("warp_inst", kernel)
+    if not inst or not sm_mhz:
+        return None
+    lane_inst_per_sym = 32.0 * inst / n
+    ceiling = 4 * 32 * sms * sm_mhz * 1e6 / lane_inst_per_sym
+    achieved = n / (ms * 1e-3)
+    return {"lane_inst_per_sym": round(lane_inst_per_sym, 2), "ceiling_gsym_s": round(ceiling / 1e9, 1),
+            "achieved_gsym_s": round(achieved / 1e9, 1), "frac": round(achieved / ceiling, 4),
+            "clock_mhz": sm_mhz, "sms": sms}
 
 
 def _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status):
