@@ -4,24 +4,32 @@
 // decoding" in the technical summary; LazyWeights, arXiv 2611.17108v1,
 // abstract: interleaved lanes, decode on demand so memory moves only coded
 // bytes):
-//   * lanes kernel: one warp per chunk of the 32-lane format.  The chunk's
-//     words are staged into shared memory with cp.async.bulk (one elected
-//     lane, mbarrier completion, double buffered per warp, no cluster
-//     multicast).  Each lane keeps a 64-bit MSB-first bit window, peeks 12
-//     bits into a shared-memory table of (length, symbol), and falls back to
-//     canonical length tables for longer codes.  Lane l emits runs of 8
-//     adjacent weights, so a warp writes 128/256/512 contiguous bytes per run
-//     (uint4 codes / uint8 codes / bf16) with one vector store per lane.
+//   * lanes kernel: one warp per chunk of the interleaved-lane format (32 or
+//     64 lanes; a thread serves one or two lanes).  The chunk's words are
+//     staged into shared memory with cp.async.bulk (one elected lane,
+//     mbarrier completion, double buffered per warp, a copy per CTA).  Each
+//     lane keeps an MSB-first bit window in two 32-bit registers, peeks 12
+//     bits into a shared-memory multi-symbol table (up to six 4-bit or three
+//     8-bit codes per entry), and falls back to canonical length tables for
+//     codes longer than 12 bits.  Lane l emits runs of 8 adjacent weights, so
+//     a warp writes 128/256/512 contiguous bytes per run (uint4 codes / uint8
+//     codes / bf16) with one vector store per lane.
 //   * the same kernel dequantizes, w = bf16_rne(float(q - zero) * scale), with
-//     the value of every code computed once per CTA in fp32 and carried in the
-//     high half of the table entry, or feeds the bf16 weights straight into an
-//     fp32 GEMV with a warp-shuffle reduction per row (weights never touch
-//     memory).
+//     the value of every code computed once per CTA in fp32 and looked up in
+//     a shared-memory table (for 4-bit codes, by byte: two values per entry),
+//     or feeds the bf16 weights straight into an fp32 GEMV with a
+//     warp-shuffle reduction per row (weights never touch memory).
 //   * gemv_mma kernel: the fused GEMV for batches of 3 to 16 activation rows.
 //     The warps of a CTA decode consecutive rows in lockstep and multiply the
 //     decoded weights with warp-level tensor-core MMAs (mma.sync m16n8k16,
-//     bf16 in, fp32 out), reading the B operand from the warps' code rings.
-//   * single kernel: the one-bitstream-per-chunk format, one thread per chunk.
+//     bf16 in, fp32 out), reading the A operand from the warps' code rings.
+//   * segment kernel: the one-bitstream-per-chunk format, one CTA per chunk
+//     of up to 16384 codes.  Its threads decode segments cut at 32-bit
+//     boundaries, re-decode from where the left neighbour stopped until they
+//     meet a code start they marked (Huffman codes resynchronise within a
+//     few codes), place their codes with a block-wide scan and write them
+//     through shared memory.
+//   * single kernel: the same format with larger chunks, one thread per chunk.
 // The decode itself is bit manipulation and streaming, not a dense
 // contraction; only the batched GEMV is MMA-shaped.  Errors are reported
 // through a status word, never by trapping; every wait on a copy is bounded.
