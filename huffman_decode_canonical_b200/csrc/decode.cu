@@ -190,7 +190,7 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
 // Canonical decode of a code longer than the table's 12 bits: the code length
 // is the first l with (top max_len bits) < limit[l].  Returns length | symbol
 // << 8, or a 1-bit entry after flagging corruption.
-__device__ __noinline__ uint32_t slow_entry(uint64_t win, int max_len, const uint32_t *limit,
+__device__ __forceinline__ uint32_t slow_entry(uint64_t win, int max_len, const uint32_t *limit,
                                             const int32_t *offs, const uint8_t *syms, int32_t *status) {
     const uint32_t v = static_cast<uint32_t>(win >> (64 - max_len));
     int l = kMaxLutBits + 1;
