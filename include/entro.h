@@ -167,7 +167,9 @@ ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t 
  * entro_group_launch then launches without any host-device traffic, as often
  * as wanted (for instance once per generated token).  d_table, the tensors'
  * device images and the x / y / output buffers must stay valid while the
- * handle is used; all tensors must share the bit width and the lane count.
+ * handle is used; all tensors must share the device, the bit width and the
+ * lane count (E_INVAL: entro_group_prepare checks the device and bit width,
+ * entro_group_launch the lane count).
  * kind:
  *   ENTRO_GROUP_GEMV  xs[i] bf16 [batch, cols_i], ys[i] fp32 [batch, rows_i]
  *                     (the per-tensor rules of entro_decode_gemv apply)
