@@ -30,7 +30,7 @@ _lock = threading.Lock()
 OK, EINVAL, ELIMIT, EFORMAT, ECORRUPT, ENOMEM = 0, -1, -2, -3, -4, -5
 MODE_AUTO, MODE_UNSIGNED, MODE_ASYM = 0, 1, 2
 SCHEME_UNSIGNED, SCHEME_ASYM = 0, 1
-FMT_SINGLE, FMT_LANES = 1, 2
+FMT_SINGLE, FMT_LANES, FMT_ROWS = 1, 2, 3
 
 
 class OracleError(RuntimeError):
@@ -162,14 +162,37 @@ def decode(blob: bytes) -> np.ndarray:
 
 
 def decode_chunks(blob: bytes, c0: int, c1: int) -> np.ndarray:
-    """Decode chunks [c0, c1) -> their codes (concatenated)."""
+    """Decode chunks [c0, c1) -> their codes (concatenated, each chunk in its own order:
+    row-major for the single-stream and lanes layouts, the tile's rows one after the other
+    for the row-tile layout)."""
     p = params(blob)
     b = np.frombuffer(blob, np.uint8)
-    first = c0 * p["chunk_symbols"]
-    last = min(p["n"], c1 * p["chunk_symbols"])
-    out = np.zeros(max(1, (c1 - c0) * p["chunk_symbols"]), np.uint8)
+    first, last = _chunk_first(p, c0), _chunk_first(p, c1)
+    out = np.zeros(max(1, p["n"] - first), np.uint8)        # room for anything a chunk may claim
     _check(_load().or_decode_chunks(_ptr(b), b.size, c0, c1, _ptr(out)), "decode_chunks")
     return out[: max(0, last - first)]
+
+
+def _chunk_first(p: Dict, c: int) -> int:
+    """Symbols in the chunks before chunk c, from the blob's geometry (chunk order)."""
+    if c >= p["n_chunks"]:
+        return p["n"]
+    if p["format"] != FMT_ROWS:
+        return min(p["n"], c * p["chunk_symbols"])
+    rows, cols, lanes = p["rows"], p["cols"], p["lanes"]
+    kc = p["chunk_symbols"] // lanes
+    tiles = -(-cols // kc)
+    g, j = divmod(c, tiles)
+    nrows = min(lanes, rows - g * lanes)
+    return g * lanes * cols + nrows * j * kc
+
+
+def tile(p: Dict, c: int) -> Tuple[int, int, int, int]:
+    """Row-tile layout: (first row, first column, rows, columns) of chunk c."""
+    lanes, kc = p["lanes"], p["chunk_symbols"] // p["lanes"]
+    tiles = -(-p["cols"] // kc)
+    g, j = divmod(c, tiles)
+    return g * lanes, j * kc, min(lanes, p["rows"] - g * lanes), min(kc, p["cols"] - j * kc)
 
 
 def dequant_bf16(q: np.ndarray, scale: float, zero: int) -> np.ndarray:

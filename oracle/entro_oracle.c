@@ -37,6 +37,13 @@
  *    of 8 consecutive symbols at chunk positions 8*L*t + 8*l + (0..7), each
  *    lane padded to the chunk's longest lane, word j of lane l stored at
  *    chunk_word_base + L*j + l.
+ *  - row-tile layout (a second reading of "interleaved lanes", for the fused
+ *    matrix-vector product): the tensor is cut into tiles of L rows by
+ *    Kc = chunk_symbols / L columns (row groups outer, column tiles inner);
+ *    lane l of a tile codes row l of the tile, its Kc (fewer in the last
+ *    column tile) codes in column order; a tile with fewer than L rows leaves
+ *    the remaining lanes empty.  Lanes are padded and word-interleaved as
+ *    above.  Columns and Kc must be multiples of 8.
  *
  * Numeric formulas checked elsewhere against independent pins (see tests).
  */
@@ -61,6 +68,7 @@
 
 #define OR_FMT_SINGLE 1
 #define OR_FMT_LANES 2
+#define OR_FMT_ROWS 3
 
 #define OR_RUN 8
 #define OR_HEADER_BYTES 128
@@ -383,20 +391,49 @@ static void put_code(bitw *bw, uint32_t code, int length) {
  *   payload   payload_words x u32
  */
 
+/* Row-tile layout: tiles of `lanes` rows by kc = chunk_symbols / lanes
+ * columns, row groups outer and column tiles inner; chunk c is one tile. */
+typedef struct {
+    int64_t row0, col0; /* first row and column of the tile */
+    int nrows;          /* rows in the tile (lanes that hold codes) */
+    int64_t width;      /* columns in the tile */
+    uint64_t first;     /* symbols in all earlier tiles */
+} tile;
+
+static uint64_t rows_tiles(int64_t rows, int64_t cols, int lanes, int64_t chunk_symbols) {
+    if (rows <= 0 || cols <= 0) return 0;
+    int64_t kc = chunk_symbols / lanes;
+    return (uint64_t)((rows + lanes - 1) / lanes) * (uint64_t)((cols + kc - 1) / kc);
+}
+
+static tile tile_of(int64_t rows, int64_t cols, int lanes, int64_t chunk_symbols, uint64_t c) {
+    int64_t kc = chunk_symbols / lanes;
+    int64_t tiles_per_group = (cols + kc - 1) / kc;
+    int64_t g = (int64_t)c / tiles_per_group, j = (int64_t)c % tiles_per_group;
+    tile t;
+    t.row0 = g * lanes;
+    t.col0 = j * kc;
+    t.nrows = (int)(rows - t.row0 < lanes ? rows - t.row0 : lanes);
+    t.width = cols - t.col0 < kc ? cols - t.col0 : kc;
+    t.first = (uint64_t)(t.row0 * cols + (int64_t)t.nrows * t.col0);
+    return t;
+}
+
 int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, int max_len,
               int format, int64_t chunk_symbols, int lanes, uint8_t *out, uint64_t cap, uint64_t *out_size) {
     if (rows < 0 || cols < 0 || (bits != 4 && bits != 8)) return OR_EINVAL;
-    if (format != OR_FMT_SINGLE && format != OR_FMT_LANES) return OR_EINVAL;
+    if (format != OR_FMT_SINGLE && format != OR_FMT_LANES && format != OR_FMT_ROWS) return OR_EINVAL;
     if (max_len == 0) max_len = (bits == 8) ? 16 : 12;
     if (max_len < 1 || max_len > 24) return OR_EINVAL;
     if (chunk_symbols == 0) chunk_symbols = (format == OR_FMT_SINGLE) ? 4096 : 8192;
     if (format == OR_FMT_SINGLE && (chunk_symbols < 1 || chunk_symbols > (1 << 20))) return OR_EINVAL;
-    if (format == OR_FMT_LANES && lanes == 0) lanes = 32;
-    if (format == OR_FMT_LANES && lanes != 32 && lanes != 64) return OR_EINVAL;
+    if (format != OR_FMT_SINGLE && lanes == 0) lanes = 32;
+    if (format != OR_FMT_SINGLE && lanes != 32 && lanes != 64) return OR_EINVAL;
     const int64_t step = (int64_t)OR_RUN * lanes; /* symbols per lane step */
-    if (format == OR_FMT_LANES &&
+    if (format != OR_FMT_SINGLE &&
         (chunk_symbols < step || chunk_symbols > 16384 || chunk_symbols % step != 0))
         return OR_EINVAL;
+    if (format == OR_FMT_ROWS && cols % OR_RUN != 0) return OR_EINVAL;
     int64_t n = rows * cols;
     int nsym = 1 << bits;
 
@@ -417,6 +454,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     or_canonical_codes(len, 256, code);
 
     uint64_t n_chunks = n > 0 ? (uint64_t)((n + chunk_symbols - 1) / chunk_symbols) : 0;
+    if (format == OR_FMT_ROWS) n_chunks = rows_tiles(rows, cols, lanes, chunk_symbols);
 
     /* pass 1: sizes.  Single stream: total bits.  Lanes: per-chunk word count. */
     uint64_t *start = (uint64_t *)calloc(n_chunks + 1, sizeof(uint64_t));
@@ -432,6 +470,22 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
         }
         start[n_chunks] = bitpos;
         payload_words = (bitpos + 31) / 32;
+    } else if (format == OR_FMT_ROWS) {
+        uint64_t wpos = 0;
+        for (uint64_t c = 0; c < n_chunks; c++) {
+            start[c] = wpos;
+            tile t = tile_of(rows, cols, lanes, chunk_symbols, c);
+            uint64_t wmax = 0;
+            for (int l = 0; l < t.nrows; l++) {
+                uint64_t lane_bits = 0;
+                for (int64_t k = 0; k < t.width; k++) lane_bits += len[q[(t.row0 + l) * cols + t.col0 + k]];
+                uint64_t wl = (lane_bits + 31) / 32;
+                if (wl > wmax) wmax = wl;
+            }
+            wpos += wmax * (uint64_t)lanes;
+        }
+        start[n_chunks] = wpos;
+        payload_words = wpos;
     } else {
         uint64_t wpos = 0;
         for (uint64_t c = 0; c < n_chunks; c++) {
@@ -464,7 +518,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     put_u32(out + 12, (uint32_t)scheme);
     put_u32(out + 16, (uint32_t)max_len);
     put_u32(out + 20, (uint32_t)format);
-    put_u32(out + 24, format == OR_FMT_SINGLE ? 1u : (uint32_t)lanes);
+    put_u32(out + 24, format == OR_FMT_SINGLE ? 1u : (uint32_t)lanes);  /* lanes or rows per tile */
     put_u32(out + 28, format == OR_FMT_SINGLE ? 1u : (uint32_t)OR_RUN);
     put_u64(out + 32, (uint64_t)rows);
     put_u64(out + 40, (uint64_t)cols);
@@ -480,6 +534,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     uint8_t *idx = out + OR_HEADER_BYTES + OR_LENGTHS_BYTES;
     for (uint64_t c = 0; c <= n_chunks; c++) {
         uint64_t first = c * (uint64_t)chunk_symbols;
+        if (format == OR_FMT_ROWS) first = c < n_chunks ? tile_of(rows, cols, lanes, chunk_symbols, c).first : (uint64_t)n;
         if (first > (uint64_t)n) first = (uint64_t)n;
         put_u64(idx + 16 * c, start[c]);
         put_u64(idx + 16 * c + 8, first);
@@ -491,6 +546,23 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     if (format == OR_FMT_SINGLE) {
         bitw bw = {payload, 0};
         for (int64_t i = 0; i < n; i++) put_code(&bw, code[q[i]], len[q[i]]);
+    } else if (format == OR_FMT_ROWS) {
+        for (uint64_t c = 0; c < n_chunks; c++) {
+            tile t = tile_of(rows, cols, lanes, chunk_symbols, c);
+            uint64_t wmax = (start[c + 1] - start[c]) / (uint64_t)lanes;
+            uint32_t *lane_words = (uint32_t *)calloc(wmax ? wmax : 1, sizeof(uint32_t));
+            if (!lane_words) { free(q); free(start); free(payload); return OR_ENOMEM; }
+            for (int l = 0; l < t.nrows; l++) {
+                memset(lane_words, 0, sizeof(uint32_t) * (wmax ? wmax : 1));
+                bitw bw = {lane_words, 0};
+                for (int64_t k = 0; k < t.width; k++) {
+                    uint8_t v = q[(t.row0 + l) * cols + t.col0 + k];
+                    put_code(&bw, code[v], len[v]);
+                }
+                for (uint64_t j = 0; j < wmax; j++) payload[start[c] + (uint64_t)lanes * j + l] = lane_words[j];
+            }
+            free(lane_words);
+        }
     } else {
         for (uint64_t c = 0; c < n_chunks; c++) {
             uint64_t a = c * (uint64_t)chunk_symbols, b = a + (uint64_t)chunk_symbols;
@@ -554,12 +626,18 @@ static int parse(const uint8_t *blob, uint64_t size, or_blob *b) {
     b->zero = (int32_t)get_u32(blob + 76);
     b->payload_words = get_u64(blob + 80);
     if (b->bits != 4 && b->bits != 8) return OR_EFORMAT;
-    if (b->format != OR_FMT_SINGLE && b->format != OR_FMT_LANES) return OR_EFORMAT;
-    if (b->format == OR_FMT_LANES && b->lanes != 32 && b->lanes != 64) return OR_EFORMAT;
+    if (b->format != OR_FMT_SINGLE && b->format != OR_FMT_LANES && b->format != OR_FMT_ROWS) return OR_EFORMAT;
+    if (b->format != OR_FMT_SINGLE && b->lanes != 32 && b->lanes != 64) return OR_EFORMAT;
     if (b->format == OR_FMT_SINGLE && b->lanes != 1) return OR_EFORMAT;
     if (b->max_len < 1 || b->max_len > 24) return OR_EFORMAT;
     if (b->chunk_symbols == 0 || b->n != b->rows * b->cols) return OR_EFORMAT;
-    if (b->n_chunks != (b->n + b->chunk_symbols - 1) / b->chunk_symbols) return OR_EFORMAT;
+    if (b->format == OR_FMT_ROWS) {
+        if (b->chunk_symbols % (OR_RUN * (uint64_t)b->lanes) || b->cols % OR_RUN) return OR_EFORMAT;
+        if (b->n_chunks != rows_tiles((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols))
+            return OR_EFORMAT;
+    } else if (b->n_chunks != (b->n + b->chunk_symbols - 1) / b->chunk_symbols) {
+        return OR_EFORMAT;
+    }
     uint64_t need = OR_HEADER_BYTES + OR_LENGTHS_BYTES + 16 * (b->n_chunks + 1) + 4 * b->payload_words;
     if (size < need) return OR_EFORMAT;
     memcpy(b->len, blob + OR_HEADER_BYTES, 256);
@@ -624,7 +702,30 @@ static int decode_symbol(const or_blob *b, bit_fn fn, const void *ctx, uint64_t 
     return OR_ECORRUPT;
 }
 
+/* Chunk c of the row-tile layout into out (the tile's rows one after the
+ * other, each in column order). */
+static int decode_tile(const or_blob *b, uint64_t c, uint8_t *out) {
+    uint64_t start = get_u64(b->index + 16 * c), next = get_u64(b->index + 16 * (c + 1));
+    uint64_t first = get_u64(b->index + 16 * c + 8), last = get_u64(b->index + 16 * (c + 1) + 8);
+    tile t = tile_of((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols, c);
+    if (first != t.first || last != first + (uint64_t)t.nrows * (uint64_t)t.width) return OR_ECORRUPT;
+    const uint64_t L = (uint64_t)b->lanes;
+    if (next < start || next > b->payload_words || (next - start) % L) return OR_ECORRUPT;
+    lane_ctx lc = {start, 0, b->lanes, (next - start) / L};
+    for (int l = 0; l < t.nrows; l++) {
+        lc.lane = l;
+        uint64_t pos = 0;
+        for (int64_t k = 0; k < t.width; k++) {
+            int s = decode_symbol(b, bit_lane, &lc, &pos);
+            if (s < 0) return s;
+            out[(uint64_t)l * (uint64_t)t.width + (uint64_t)k] = (uint8_t)s;
+        }
+    }
+    return OR_OK;
+}
+
 static int decode_chunk(const or_blob *b, uint64_t c, uint8_t *out /* chunk-local */) {
+    if (b->format == OR_FMT_ROWS) return decode_tile(b, c, out);
     uint64_t start = get_u64(b->index + 16 * c), next = get_u64(b->index + 16 * (c + 1));
     uint64_t first = get_u64(b->index + 16 * c + 8), last = get_u64(b->index + 16 * (c + 1) + 8);
     if (first != c * b->chunk_symbols || last < first || last > b->n) return OR_ECORRUPT;
@@ -674,26 +775,55 @@ int or_blob_params(const uint8_t *blob, uint64_t size, int64_t *out /* 14 entrie
     return r;
 }
 
-/* decode chunks [c0, c1) into out[first_symbol(c0) ...] */
+/* symbols in the chunks before chunk c (chunk order) */
+static uint64_t chunk_first(const or_blob *b, uint64_t c) {
+    if (b->format == OR_FMT_ROWS)
+        return c < b->n_chunks ? tile_of((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols, c).first
+                               : b->n;
+    uint64_t f = c * b->chunk_symbols;
+    return f < b->n ? f : b->n;
+}
+
+/* decode chunks [c0, c1) into out: each chunk's codes in its own order
+ * (row-major for the single-stream and lanes layouts; the tile's rows one
+ * after the other for the row-tile layout), chunk c at out + (symbols in the
+ * chunks c0 .. c-1) */
 int or_decode_chunks(const uint8_t *blob, uint64_t size, uint64_t c0, uint64_t c1, uint8_t *out) {
     or_blob *b = (or_blob *)malloc(sizeof(or_blob));
     if (!b) return OR_ENOMEM;
     int r = parse(blob, size, b);
     if (r == OR_OK && (c0 > c1 || c1 > b->n_chunks)) r = OR_EINVAL;
+    uint64_t base = r == OR_OK ? chunk_first(b, c0) : 0;
     for (uint64_t c = c0; r == OR_OK && c < c1; c++)
-        r = decode_chunk(b, c, out + (c - c0) * b->chunk_symbols);
+        r = decode_chunk(b, c, out + (chunk_first(b, c) - base));
     free(b);
     return r;
 }
 
+/* whole tensor, row-major */
 int or_decode(const uint8_t *blob, uint64_t size, uint8_t *out) {
     or_blob *b = (or_blob *)malloc(sizeof(or_blob));
     if (!b) return OR_ENOMEM;
     int r = parse(blob, size, b);
-    uint64_t nch = b->n_chunks;
+    if (r != OR_OK || b->format != OR_FMT_ROWS) {
+        uint64_t nch = b->n_chunks;
+        free(b);
+        if (r != OR_OK) return r;
+        return or_decode_chunks(blob, size, 0, nch, out);
+    }
+    /* row tiles: decode each tile, then place its rows */
+    uint8_t *tmp = (uint8_t *)malloc((size_t)b->chunk_symbols);
+    if (!tmp) { free(b); return OR_ENOMEM; }
+    for (uint64_t c = 0; r == OR_OK && c < b->n_chunks; c++) {
+        tile t = tile_of((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols, c);
+        r = decode_tile(b, c, tmp);
+        for (int l = 0; r == OR_OK && l < t.nrows; l++)
+            memcpy(out + (uint64_t)(t.row0 + l) * b->cols + (uint64_t)t.col0, tmp + (uint64_t)l * (uint64_t)t.width,
+                   (size_t)t.width);
+    }
+    free(tmp);
     free(b);
-    if (r != OR_OK) return r;
-    return or_decode_chunks(blob, size, 0, nch, out);
+    return r;
 }
 
 /* ------------------------------------------------------------------ */

@@ -313,6 +313,41 @@ def test_lane_layout_closed_form(lanes):
         assert int(words[lane]) == expect, lane
 
 
+@pytest.mark.parametrize("lanes", [32, 64])
+def test_row_tile_layout_closed_form(lanes):
+    """Row tiles of `lanes` rows by 40 columns (the last column tile 24 wide, the last row
+    group ragged): with one-bit codes, word i of lane l of a tile holds bits 32i .. 32i+31
+    of row l of the tile, MSB first, and lanes past the tile's last row stay zero."""
+    rows, cols, kc = 2 * lanes + 6, 104, 40
+    b = (((np.arange(rows)[:, None] * 5 + np.arange(cols)[None, :] * 3) % 7) < 3).astype(np.uint8)
+    blob = oracle.encode(_two_code_tensor(b), 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS, lanes * kc,
+                         lanes=lanes)
+    prm = oracle.params(blob)
+    assert prm["format"] == oracle.FMT_ROWS and prm["lanes"] == lanes
+    assert prm["lengths"][0] == 1 and prm["lengths"][15] == 1 and prm["lengths"].sum() == 2
+    tiles = [(g, j) for g in range(3) for j in range(3)]
+    assert prm["n_chunks"] == len(tiles)
+    idx = np.frombuffer(blob, np.uint64, 2 * (len(tiles) + 1), 384).reshape(-1, 2)
+    words = np.frombuffer(blob, np.uint32, prm["payload_words"], 384 + 16 * (len(tiles) + 1))
+    start = first = 0
+    for c, (g, j) in enumerate(tiles):
+        r0, c0 = g * lanes, j * kc
+        nr, wd = min(lanes, rows - r0), min(kc, cols - c0)
+        wc = -(-wd // 32)                                # one bit per code
+        assert (int(idx[c, 0]), int(idx[c, 1])) == (start, first), c
+        for lane in range(lanes):
+            for i in range(wc):
+                expect = 0
+                if lane < nr:
+                    for k in range(32):
+                        if 32 * i + k < wd:
+                            expect |= int(b[r0 + lane, c0 + 32 * i + k]) << (31 - k)
+                assert int(words[start + lanes * i + lane]) == expect, (c, lane, i)
+        start += wc * lanes
+        first += nr * wd
+    assert (int(idx[-1, 0]), int(idx[-1, 1])) == (start, rows * cols) and prm["payload_words"] == start
+
+
 def test_single_stream_layout_closed_form():
     n = 100
     b = ((np.arange(n) * 3) % 7 < 3).astype(np.uint8)
@@ -350,6 +385,10 @@ CASES = [
     ("t4", 4, oracle.MODE_ASYM, 4, oracle.FMT_LANES, 512, 9, 100),
     ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_LANES, -1024, 7, 333),    # 64 lanes
     ("t4", 8, oracle.MODE_AUTO, 16, oracle.FMT_LANES, -8192, 40, 300),        # 64 lanes
+    ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS, 8192, 100, 1000),   # row tiles, ragged both ways
+    ("t4", 8, oracle.MODE_AUTO, 16, oracle.FMT_ROWS, 4096, 70, 3072),
+    ("skew", 8, oracle.MODE_ASYM, 16, oracle.FMT_ROWS, 512, 33, 24),
+    ("laplace", 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS, -1024, 130, 520),   # 64-row tiles
 ]
 
 
@@ -373,7 +412,13 @@ def test_encode_decode_identity(case):
     if prm["n_chunks"] > 1:
         c0, c1 = 1, prm["n_chunks"]
         part = oracle.decode_chunks(blob, c0, c1)
-        assert (part == q[c0 * prm["chunk_symbols"]:]).all()
+        if fmt != oracle.FMT_ROWS:
+            assert (part == q[c0 * prm["chunk_symbols"]:]).all()
+        else:                                            # tiles, each row-major
+            Q = q.reshape(rows, cols)
+            tiles = [oracle.tile(prm, c) for c in range(c0, c1)]
+            want = np.concatenate([Q[r0:r0 + nr, k0:k0 + wd].reshape(-1) for r0, k0, nr, wd in tiles])
+            assert (part == want).all()
 
 
 def test_empty_tensor_blob():
