@@ -1,30 +1,33 @@
 """Benchmark of the Huffman weight-decoding hot path on B200.
 
-One step = one pass of the whole hot path over the 4096x4096 4-bit Laplace
-tensor (32 word-interleaved lanes per 8192-symbol chunk):
-    decode -> packed uint4 codes, decode -> dequantize -> bf16, and the fused
-    decode -> dequantize -> GEMV (batch 1),
-each through the C ABI of libentro.  Inputs are resident in HBM.  The working
-set is made larger than L2: 40 replicas of the encoded tensor (160 MB of coded
-payload alone, against a 126 MB L2) and of its outputs rotate, each kernel on
-the next replica, so every kernel reads coded words that no recent kernel
-touched and writes outputs whose lines must first be evicted -- the steady
-state of decoding a model much larger than L2 (no flush kernel, so the decode
-code stays warm as it would in serving).  Times come from CUDA events on the
-launching stream: the K timed steps run back to back between one pair of
-events, and each kernel's own duration is the mean over K launches of it back
-to back (events between the calls would add gaps of their own, ~2.5 us each).
+The line's headline is BASELINE's fused-GEMV metric on its Mistral-7B-shaped
+configuration: one simulated token-generation step = the fused decode ->
+dequantize -> GEMV of all 224 projection tensors (32 layers of q, k, v, o,
+gate, up, down; Laplace weights, tensor-level asymmetric 4-bit codes, one
+Huffman code per tensor, 6.98 G weights, ~1.42 GB of coded bytes) against bf16
+activations at batch 1, as ONE grouped launch through the C ABI of libentro.
+value = tokens/s = 1 / step time.  The coded model (1.4 GB) is far larger than
+L2, so every step streams its weights from HBM; no flush is needed.  Times come
+from CUDA events on the launching stream: K steps back to back between one pair
+of events (events between launches would add gaps of their own).
+
+Extra keys, each one grouped launch or a set of launches timed the same way:
+  * mistral batch 4 and 16 (the same model, the GEMV's batched path);
+  * smollm_bf16: the SmolLM-1.7B-shaped whole-model decode to bf16 (8-bit codes);
+  * laplace_4096x4096_u4: the 4096x4096 4-bit tensor decoded to codes, to bf16
+    and through the GEMV, 40 rotating replicas so that inputs exceed L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
-With N > 1 (torchrun) every rank decodes its own replica of the workload (the
-chunks are independent problems; no data-path collective), and the line
-reports the whole-job rate from the slowest rank ("weak" scaling).
---impl reference times the CPU oracle doing the same step on a bounded sample.
+With N > 1 (torchrun) every rank runs the step on its own GPU (tensors are
+independent problems; no data-path collective) and the line reports the
+whole-job rate from the slowest rank ("weak" scaling).  --impl reference times
+the CPU oracle doing the same step on a bounded sample and extrapolates.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -42,9 +45,12 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "decoded Gsym/s and % HBM roofline (Huffman decode+dequant); fused GEMV tok/s"
-WORKLOAD = "laplace_4096x4096_u4"
+WORKLOAD = "mistral_7b_u4"
+TENSOR_WORKLOAD = "laplace_4096x4096_u4"
 REPLICAS = 40
 NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e, HGX figure (context beside the measured copy peak)
+KERNEL_SOURCES = ("huffman_decode_canonical_b200/csrc/decode.cu", "huffman_decode_canonical_b200/csrc/rows.cuh",
+                  "huffman_decode_canonical_b200/csrc/blob_format.h")
 
 
 def _peaks():
@@ -151,238 +157,191 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle leg
 
-def _oracle_step(blob: bytes, chunks, threads: int, x_bits: np.ndarray):
-    """The oracle on host cores: decode the sample's chunks to codes, to bf16 weights,
-    and through the fp64 GEMV, chunk ranges split over threads (the EntroLLM
-    multi-threaded chunk decoder).  Returns symbols processed."""
+
+
+# ------------------------------------------------------------------ model-shaped workloads
+
+def encode_model(entro, W: workloads.Workload, device, limit=None, keep=0):
+    """Draw, encode (libentro's host encoder, all host cores) and upload every tensor of
+    W, one at a time.  Returns (device tensors, blob infos, seconds encoding, the
+    serialized blobs of the first `keep` tensors)."""
+    dts, infos, kept = [], [], []
+    t_enc = 0.0
+    specs = W.tensors if limit is None else W.tensors[:limit]
+    for i, spec in enumerate(specs):
+        w = workloads.weights(W, spec, device=device).cpu().numpy()
+        t0 = time.perf_counter()
+        blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
+                                 chunk_symbols=W.chunk_symbols(spec.cols), lanes=W.lanes)
+        t_enc += time.perf_counter() - t0
+        del w
+        dts.append(entro.upload(blob, device=device))
+        infos.append(blob.info())
+        if i < keep:
+            kept.append(blob.to_bytes())
+        del blob
+    return dts, infos, t_enc, kept
+
+
+def _override(W, args):
+    if not getattr(args, "fmt", ""):
+        return W
+    fmt = {"lanes": workloads.FORMAT_LANES, "rows": workloads.FORMAT_ROWS}[args.fmt]
+    lanes = args.lanes or W.lanes
+    rule = W.chunk_rule if fmt == workloads.FORMAT_LANES else "fixed:%d" % (args.chunk or 256 * lanes)
+    return dataclasses.replace(W, fmt=fmt, lanes=lanes, chunk_rule=rule)
+
+
+class GemvStep:
+    """The grouped fused GEMV over a model's tensors at one batch size.  Tensors with the
+    same number of columns read the same activations (as the projections of one layer
+    input do); every output row lands in one fp32 buffer, so a step's result comes back
+    with one copy."""
+
+    def __init__(self, entro, dts, seed, batch, device):
+        self.batch = batch
+        cols = sorted(set(d.cols for d in dts))
+        self.x = {K: workloads.activations(seed, batch, K).to(device) for K in cols}
+        self.rows = sum(d.rows for d in dts)
+        self.y = torch.empty((batch * self.rows,), dtype=torch.float32, device=device)
+        ys, off = [], 0
+        for d in dts:
+            ys.append(self.y[off: off + batch * d.rows].view(batch, d.rows))
+            off += batch * d.rows
+        self.ys = ys
+        self.group = entro.Group(dts, entro.GROUP_GEMV, xs=[self.x[d.cols] for d in dts], ys=ys, batch=batch)
+        self.x_bytes = sum(2 * x.numel() for x in self.x.values())        # distinct activation vectors
+        self.io_bytes = sum(2 * batch * d.cols for d in dts) + 4 * batch * self.rows
+
+    def launch(self, status):
+        self.group.launch(status=status)
+
+
+def _time_launches(fn, steps, stream, sleep_s=0.0):
+    """Mean ms of `steps` calls of fn() back to back between one pair of events; the GPU
+    is kept busy by a device sleep while the host enqueues them."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if sleep_s > 0:
+        torch.cuda._sleep(int(sleep_s * 2.0e9))
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _step_bytes(infos, step):
+    """Algorithmic bytes of one GEMV step: coded bits of every
+    tensor (lane padding excluded) / 8 + chunk index + one copy of each tensor's decode
+    tables + activations + outputs.  The bf16 weights are never written."""
+    table = 32768 + 512
+    return (sum(i["coded_bits"] for i in infos) / 8.0 + sum(i["index_bytes"] for i in infos)
+            + table * len(infos) + step.io_bytes)
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+def _oracle_sample(W, rows: int):
+    """The first `rows` rows of layer 0's seven tensors, encoded by the oracle itself in the
+    workload's format (the sample's own quantization parameters)."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
+    specs = W.tensors[:7]
 
-    p = oracle.params(blob)
-    C, K = p["chunk_symbols"], p["cols"]
-    c0, c1 = chunks
-    bounds = np.linspace(c0, c1, threads + 1).astype(int)
-
-    def work(i):
-        a, b = int(bounds[i]), int(bounds[i + 1])
-        if a >= b:
-            return 0
-        q = oracle.decode_chunks(blob, a, b)                     # pass 1: codes
-        q2 = oracle.decode_chunks(blob, a, b)                    # pass 2: codes -> bf16
-        wb = oracle.dequant_bf16(q2, p["scale"], p["zero"])
-        q3 = oracle.decode_chunks(blob, a, b)                    # pass 3: -> GEMV over the rows
-        wg = oracle.dequant_bf16(q3, p["scale"], p["zero"]).reshape(-1, K)
-        oracle.gemv(wg, x_bits)
-        return q.size + wb.size + wg.size
-
-    with ThreadPoolExecutor(threads) as ex:
-        return sum(ex.map(work, range(threads)))
+    def enc(spec):
+        w = workloads.weights(W, spec, device="cpu").numpy()[:rows]
+        blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols), lanes=W.lanes)
+        return blob, spec.cols
+    with ThreadPoolExecutor(len(specs)) as ex:
+        return list(ex.map(enc, specs))
 
 
-def cpu_baseline(seconds: float = 12.0):
+def _oracle_pass(sample, threads: int, seed: int):
+    """One pass of the oracle over the sample: decode every chunk bit by bit, dequantize to
+    bf16, fp64 GEMV of the chunk's weights with the matching activations; chunks spread
+    over threads (the EntroLLM multi-threaded chunk decoder).  Returns symbols processed."""
     import oracle
-    W = workloads.get(WORKLOAD)
-    spec = W.tensors[0]
-    w = workloads.weights(W, spec).numpy()
-    t_enc = time.perf_counter()
-    blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols))
-    t_enc = time.perf_counter() - t_enc
-    p = oracle.params(blob)
-    x_bits = workloads.bf16_bits(workloads.activations(0, 1, spec.cols))
-    threads = max(1, min(os.cpu_count() or 1, 64))
-    n_chunks = p["n_chunks"]
-    total, t0, reps = 0, time.perf_counter(), 0
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = []
+    for blob, cols in sample:
+        p = oracle.params(blob)
+        x = workloads.bf16_bits(workloads.activations(seed, 1, cols))
+        for c in range(p["n_chunks"]):
+            jobs.append((blob, p, x, c))
+
+    def work(job):
+        blob, p, x, c = job
+        q = oracle.decode_chunks(blob, c, c + 1)
+        wb = oracle.dequant_bf16(q, p["scale"], p["zero"])
+        if p["format"] == oracle.FMT_ROWS:
+            r0, k0, nr, wd = oracle.tile(p, c)
+            oracle.gemv(wb.reshape(nr, wd), np.ascontiguousarray(x[:, k0:k0 + wd]))
+        else:
+            oracle.gemv(wb.reshape(-1, p["cols"]), x)
+        return q.size
+    with ThreadPoolExecutor(threads) as ex:
+        return sum(ex.map(work, jobs))
+
+
+def _oracle_threads():
+    return max(1, min(os.cpu_count() or 1, 64))
+
+
+def cpu_baseline(W, seconds: float = 10.0, rows: int = 256):
+    """The oracle doing the step's work on a bounded sample, extrapolated to the whole step."""
+    t0 = time.perf_counter()
+    sample = _oracle_sample(W, rows)
+    t_enc = time.perf_counter() - t0
+    threads = _oracle_threads()
+    syms, passes, t0 = 0, 0, time.perf_counter()
     while True:
-        total += _oracle_step(blob, (0, n_chunks), threads, x_bits)
-        reps += 1
-        if time.perf_counter() - t0 >= seconds or reps >= 8:
+        syms += _oracle_pass(sample, threads, W.seed)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    # one thread on a 1/32 sample of the chunks (the sequential decoder's rate)
-    sample1 = (0, max(1, n_chunks // 32))
-    total1, t1, reps1 = 0, time.perf_counter(), 0
-    while True:
-        total1 += _oracle_step(blob, sample1, 1, x_bits)
-        reps1 += 1
-        if time.perf_counter() - t1 >= seconds / 4 or reps1 >= 4:
-            break
-    dt1 = time.perf_counter() - t1
-    return {"value": total / dt / 1e9, "unit": "Gsym/s", "cores": threads, "kind": "oracle",
-            "sample": f"{reps} pass(es) of the whole {spec.rows}x{spec.cols} tensor "
-                      f"({n_chunks} chunks; codes, bf16 and GEMV passes), chunk ranges over {threads} threads, "
-                      f"{dt:.1f} s",
-            "single_thread": {"value": total1 / dt1 / 1e9, "unit": "Gsym/s", "cores": 1,
-                              "sample": f"{reps1} pass(es) of chunks {sample1[0]}..{sample1[1]} "
-                                        f"(codes, bf16 and GEMV passes), {dt1:.1f} s"},
-            "oracle_encode_s": round(t_enc, 3)}
+    rate = syms / dt
+    return {"value": round(rate / W.n, 6), "unit": "tok/s (batch 1)", "cores": threads, "kind": "oracle",
+            "sample": f"{passes} pass(es) over the first {rows} rows of layer 0's 7 tensors "
+                      f"({syms // passes} weights: bit-by-bit decode, bf16 dequant, fp64 GEMV per chunk), "
+                      f"chunks over {threads} threads, {dt:.1f} s; tok/s = weights/s / {W.n} weights per step",
+            "gsym_s": round(rate / 1e9, 4), "oracle_encode_s": round(t_enc, 2)}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    import oracle
     W = workloads.get(WORKLOAD)
-    spec = W.tensors[0]
-    w = workloads.weights(W, spec).numpy()
-    blob = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, W.chunk_symbols(spec.cols))
-    p = oracle.params(blob)
-    x_bits = workloads.bf16_bits(workloads.activations(0, 1, spec.cols))
-    threads = max(1, min(os.cpu_count() or 1, 64))
-    sample = (0, min(p["n_chunks"], 256))                         # 1/8 of the tensor per step
+    sample = _oracle_sample(W, 256)
+    threads = _oracle_threads()
     for _ in range(args.warmup):
-        _oracle_step(blob, sample, threads, x_bits)
+        _oracle_pass(sample, threads, W.seed)
     t0 = time.perf_counter()
     syms = 0
     for _ in range(args.steps):
-        syms += _oracle_step(blob, sample, threads, x_bits)
+        syms += _oracle_pass(sample, threads, W.seed)
     dt = time.perf_counter() - t0
-    value = syms / dt / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Gsym/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+    value = syms / dt / W.n
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s (batch 1)", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u4->bf16/fp64",
-            "data": "synthetic", "config": _config(W, spec, p["chunk_symbols"]),
-            "cpu_baseline": {"value": value, "unit": "Gsym/s", "cores": threads, "kind": "oracle",
-                             "sample": f"chunks {sample[0]}..{sample[1]} of {p['n_chunks']} per step "
-                                       f"(codes, bf16 and GEMV passes) over {threads} threads"},
-            "e2e": {"value": value, "unit": "Gsym/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "data": "synthetic", "config": _step_config(W, 1),
+            "cpu_baseline": {"value": value, "unit": "tok/s (batch 1)", "cores": threads, "kind": "oracle",
+                             "sample": f"per step: the first 256 rows of layer 0's 7 tensors "
+                                       f"({syms // max(args.steps, 1)} weights), chunks over {threads} threads; "
+                                       f"tok/s extrapolated to the step's {W.n} weights"},
+            "e2e": {"value": value, "unit": "tok/s (batch 1)", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def _config(W, spec, chunk):
-    return {"workload": W.name, "shape": [spec.rows, spec.cols], "bits": W.bits, "quant": "asymmetric",
-            "max_code_len": W.max_len, "chunk_symbols": chunk, "lanes": 32, "gemv_batch": 1,
-            "l2": f"inputs larger than L2: {REPLICAS} rotating replicas (image + outputs), "
-                  "each kernel on a different replica; no flush"}
-
-
-# ------------------------------------------------------------------ native arm
-
-def run_native(args, dist, rank, world, local_rank):
-    import huffman_decode_canonical_b200 as entro
-    entro.set_overlap(not args.no_overlap)
-
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    stream = torch.cuda.current_stream(device)
-    W = workloads.get(WORKLOAD)
-    spec = W.tensors[0]
-    chunk = W.chunk_symbols(spec.cols)
-    w = workloads.weights(W, spec).numpy()
-    blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
-                             chunk_symbols=chunk)
-    info = blob.info()
-    reps = [entro.upload(blob, device=device) for _ in range(REPLICAS)]
-    dt = reps[0]
-    n = info["n"]
-    codes = [r.empty_codes() for r in reps]
-    bf = [r.empty_bf16() for r in reps]
-    x = workloads.activations(0, 1, spec.cols).to(device)
-    y = [torch.empty((1, spec.rows), dtype=torch.float32, device=device) for _ in reps]
-    status = torch.zeros(1, dtype=torch.int32, device=device)
-    counter = [0]
-
-    def next_rep():
-        r = counter[0] % REPLICAS
-        counter[0] += 1
-        return r
-
-    kernels = [("codes", lambda r: reps[r].decode_codes(out=codes[r], status=status)),
-               ("bf16", lambda r: reps[r].decode_dequant_bf16(out=bf[r], status=status)),
-               ("gemv", lambda r: reps[r].decode_gemv(x, y=y[r], status=status))]
-
-    def step():
-        for _, fn in kernels:
-            fn(next_rep())
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize(device)
-    clocks = ClockSampler(device)
-    clocks.start()
-    # untimed burn-in so that clock samples cover a loaded GPU even for short runs
-    t_end = time.perf_counter() + 1.0
-    while time.perf_counter() < t_end:
-        step()
-        torch.cuda.synchronize(device)
-    # The K steps run back to back between one pair of events (events between
-    # the calls would add their own gaps); the GPU is kept busy while the host
-    # enqueues them, so the events measure device time only.
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(dist, device)
-    torch.cuda.synchronize(device)
-    wall0 = time.perf_counter()
-    torch.cuda._sleep(int(args.steps * 300e-6 * 2.0e9))
-    ev0.record(stream)
-    for s in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize(device)
-    wall = time.perf_counter() - wall0
-    _barrier(dist, device)
-    step_ms = ev0.elapsed_time(ev1) / args.steps
-    # Each kernel's own duration: K launches of it back to back (rotating
-    # replicas), between one pair of events.
-    mean_ms = {}
-    for name, fn in kernels:
-        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(device)
-        torch.cuda._sleep(int(args.steps * 100e-6 * 2.0e9))
-        k0.record(stream)
-        for s in range(args.steps):
-            fn(next_rep())
-        k1.record(stream)
-        torch.cuda.synchronize(device)
-        mean_ms[name] = k0.elapsed_time(k1) / args.steps
-    clk = clocks.stop()
-    assert int(status.item()) == 0, f"device status {int(status.item())}"
-    step_ms_max = _max_over_ranks(dist, step_ms, device)
-    bf16_ms_max = _max_over_ranks(dist, mean_ms["bf16"], device)
-
-    # algorithmic bytes per launch: coded bits (no lane padding) + chunk index + output
-    coded = info["coded_bits"] / 8.0
-    index = info["index_bytes"]
-    alg = {"codes": coded + index + dt.codes_nbytes(), "bf16": coded + index + 2.0 * n,
-           "gemv": coded + index + 2.0 * spec.cols + 4.0 * spec.rows}
-    peak, peak_kind = _peaks()
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    kern = {}
-    for k in mean_ms:
-        us = 1e3 * mean_ms[k]
-        gbs = alg[k] / (mean_ms[k] * 1e-3) / 1e9
-        kern[k] = {"us": round(us, 3), "gsym_s": round(n / (mean_ms[k] * 1e-3) / 1e9, 2),
-                   "alg_bytes": int(alg[k]), "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4),
-                   "issue_bound": _issue_ceiling(k, n, mean_ms[k], clk.get("sm_mhz"), sms)}
-    kern["gemv"]["tok_s"] = round(1.0 / (mean_ms["gemv"] * 1e-3), 1)
-    achieved = alg["bf16"] / (bf16_ms_max * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "lanes_kernel<4, bf16> (decode + dequant to bf16)",
-                "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": _traffic("bf16"),
-                "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
-                "issue_bound": kern["bf16"]["issue_bound"]}
-
-    e2e = _e2e(entro, blob, dt, device, stream, args, n, codes[0], bf[0], x, y[0], status)
-    e2e["value"] = _max_over_ranks(dist, -e2e["value"], device) * -1 if dist is not None else e2e["value"]
-    if rank != 0:
-        return 0
-    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline()
-    value = world * 3 * n / (step_ms_max * 1e-3) / 1e9
-    line = {"metric": METRIC, "value": round(value, 3), "unit": "Gsym/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes -> bf16 / fp32 accumulate",
-            "data": "synthetic", "config": _config(W, spec, chunk), "launch_overlap": not args.no_overlap,
-            "value_definition": "symbols decoded per second over the step (3 passes of n = 16.8M symbols); "
-                                "K steps back to back between one pair of CUDA events",
-            "kernels_timing": "each kernel alone: K launches back to back (rotating replicas) between one "
-                              "pair of CUDA events, per-launch mean",
-            "kernels": kern,
-            "bits_per_weight": {"coded": round(info["coded_bits"] / n, 4),
-                                "payload": round(8.0 * info["payload_bytes"] / n, 4),
-                                "all_in": round(8.0 * (info["payload_bytes"] + info["index_bytes"] + 16384) / n, 4)},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps,
-            "clocks": clk, "wall_s_timed": round(wall, 4)}
-    print(json.dumps(line), flush=True)
-    return 0
+def _step_config(W, batch):
+    return {"workload": W.name, "tensors": len(W.tensors), "symbols": W.n, "bits": W.bits, "batch": batch,
+            "format": {workloads.FORMAT_LANES: "lanes", workloads.FORMAT_ROWS: "row tiles"}.get(W.fmt, "single"),
+            "lanes": W.lanes, "chunk_symbols": W.chunk_symbols(4096),
+            "l2": "inputs larger than L2: the step streams 1.4 GB of coded weights (L2 126 MB); no flush"}
 
 
 def _kernel_source_hash() -> str:
@@ -391,7 +350,7 @@ def _kernel_source_hash() -> str:
     import hashlib
     import re
     h = hashlib.sha256()
-    for rel in ("huffman_decode_canonical_b200/csrc/decode.cu", "huffman_decode_canonical_b200/csrc/blob_format.h"):
+    for rel in KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel)) as f:
             src = f.read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
@@ -436,60 +395,277 @@ def _issue_ceiling(kernel: str, n: int, ms: float, sm_mhz, sms: int):
             "clock_mhz": sm_mhz, "sms": sms}
 
 
-def _e2e(entro, blob, dt, device, stream, args, n, codes, bf, x, y, status):
-    """The same step through the public API with host buffers: upload the blob's device
-    image from host memory, decode the three ways, read every result back."""
-    import ctypes
-    host_codes = torch.empty(codes.numel(), dtype=torch.uint8, pin_memory=True)
-    host_bf = torch.empty(bf.shape, dtype=torch.bfloat16, pin_memory=True)
-    host_y = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
-    nbytes = blob.device_bytes()
-    mem = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    lib = entro.lib()
 
-    copy_stream = torch.cuda.Stream(device)
-    drained = torch.cuda.Event()  # the previous step's reads of codes / bf / y are done
-    drained.record(copy_stream)
+# ------------------------------------------------------------------ native arm: the GEMV step
+
+def _e2e_step(step, status, steps):
+    """The step through the public API with host buffers: the activations are copied from
+    pinned host memory, the grouped launch runs, and every output row is read back to
+    pinned host memory before the next step starts (a token's result is needed before the
+    next token's input exists).  Wall clock per step."""
+    host_x = {K: x.cpu().pin_memory() for K, x in step.x.items()}
+    host_y = torch.empty(step.y.shape, dtype=torch.float32, pin_memory=True)
+    cur = torch.cuda.current_stream()
 
     def one():
-        # results go back on a second stream as soon as each decode is done, so the
-        # transfers overlap the later decodes (and the next step's upload)
-        h = ctypes.c_void_p()
-        r = lib.entro_upload(blob._h, ctypes.c_void_p(mem.data_ptr()), nbytes, ctypes.c_void_p(stream.cuda_stream),
-                             ctypes.byref(h))
-        assert r == 0
-        st = ctypes.c_void_p(status.data_ptr())
-        s = ctypes.c_void_p(stream.cuda_stream)
-        stream.wait_event(drained)
-        done = [torch.cuda.Event() for _ in range(3)]
-        assert lib.entro_decode_codes(h, ctypes.c_void_p(codes.data_ptr()), st, s) == 0
-        done[0].record(stream)
-        assert lib.entro_decode_dequant_bf16(h, ctypes.c_void_p(bf.data_ptr()), st, s) == 0
-        done[1].record(stream)
-        assert lib.entro_decode_gemv(h, ctypes.c_void_p(x.data_ptr()), 1, ctypes.c_void_p(y.data_ptr()), st, s) == 0
-        done[2].record(stream)
-        with torch.cuda.stream(copy_stream):
-            for ev, dst, src in zip(done, (host_codes, host_bf, host_y), (codes, bf, y)):
-                copy_stream.wait_event(ev)
-                dst.copy_(src, non_blocking=True)
-            drained.record(copy_stream)
-        lib.entro_tensor_free(h)
+        for K, hx in host_x.items():
+            step.x[K].copy_(hx, non_blocking=True)
+        step.launch(status)
+        host_y.copy_(step.y, non_blocking=True)
+        cur.synchronize()
 
-    reps = max(3, min(args.steps, 20))
     for _ in range(2):
         one()
-    torch.cuda.synchronize(device)
+    reps = max(3, min(steps, 50))
     t0 = time.perf_counter()
     for _ in range(reps):
         one()
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(1.0 / dt, 2), "unit": f"tok/s (batch {step.batch})",
+            "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in host_x.values())),
+            "d2h_bytes_per_step": int(host_y.numel() * 4), "ms_per_step": round(1e3 * dt, 4),
+            "note": "per step: activations copied from pinned host memory, one grouped launch "
+                    "(entro_group_launch), all outputs copied back to pinned host memory, stream synchronised; "
+                    "wall clock"}
+
+
+def _smollm_bf16(entro, device, stream, steps, peak):
+    """SmolLM-1.7B-shaped whole-model decode to bf16 (169 tensors, 8-bit codes), one grouped launch."""
+    W = workloads.get("smollm_1p7b_u8")
+    dts, infos, t_enc, _ = encode_model(entro, W, device)
+    outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device=device) for d in dts]
+    g = entro.Group(dts, entro.GROUP_BF16, outs=outs)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    for _ in range(3):
+        g.launch(status=status)
+    ms = _time_launches(lambda: g.launch(status=status), max(5, min(steps, 20)), stream, 2e-4)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    n = sum(i["n"] for i in infos)
+    alg = sum(i["coded_bits"] for i in infos) / 8.0 + sum(i["index_bytes"] for i in infos) + 2.0 * n
+    gbs = alg / (ms * 1e-3) / 1e9
+    out = {"ms": round(ms, 4), "gsym_s": round(n / (ms * 1e-3) / 1e9, 1), "alg_bytes": int(alg),
+           "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4), "tensors": len(dts), "symbols": n,
+           "bits_per_weight": round(sum(i["coded_bits"] for i in infos) / n, 4), "host_encode_s": round(t_enc, 2)}
+    del outs, g, dts
+    torch.cuda.empty_cache()
+    return out
+
+
+def _tensor_kernels(entro, device, stream, steps, peak, clk_mhz, sms):
+    """The 4096x4096 4-bit tensor (32 interleaved lanes per 8192-symbol chunk): decode to
+    codes, to bf16 and the batch-1 GEMV, each K launches back to back over 40 rotating
+    replicas (160 MB of coded words, inputs larger than L2)."""
+    W = workloads.get(TENSOR_WORKLOAD)
+    spec = W.tensors[0]
+    w = workloads.weights(W, spec).numpy()
+    blob = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
+                             chunk_symbols=W.chunk_symbols(spec.cols))
+    info = blob.info()
+    reps = [entro.upload(blob, device=device) for _ in range(REPLICAS)]
+    n = info["n"]
+    codes = [r.empty_codes() for r in reps]
+    bf = [r.empty_bf16() for r in reps]
+    x = workloads.activations(0, 1, spec.cols).to(device)
+    y = [torch.empty((1, spec.rows), dtype=torch.float32, device=device) for _ in reps]
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    counter = [0]
+
+    def nxt():
+        counter[0] += 1
+        return counter[0] % REPLICAS
+
+    kernels = [("codes", lambda: (lambda r: reps[r].decode_codes(out=codes[r], status=status))(nxt())),
+               ("bf16", lambda: (lambda r: reps[r].decode_dequant_bf16(out=bf[r], status=status))(nxt())),
+               ("gemv", lambda: (lambda r: reps[r].decode_gemv(x, y=y[r], status=status))(nxt()))]
+    for _ in range(3):
+        for _, fn in kernels:
+            fn()
+    coded = info["coded_bits"] / 8.0
+    index = info["index_bytes"]
+    alg = {"codes": coded + index + reps[0].codes_nbytes(), "bf16": coded + index + 2.0 * n,
+           "gemv": coded + index + 2.0 * spec.cols + 4.0 * spec.rows}
+    out = {}
+    for name, fn in kernels:
+        ms = _time_launches(fn, max(steps, 20), stream, 1e-4)
+        gbs = alg[name] / (ms * 1e-3) / 1e9
+        out[name] = {"us": round(1e3 * ms, 3), "gsym_s": round(n / (ms * 1e-3) / 1e9, 2), "alg_bytes": int(alg[name]),
+                     "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4),
+                     "issue_bound": _issue_ceiling("tensor_" + name, n, ms, clk_mhz, sms)}
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    out["bits_per_weight"] = {"coded": round(info["coded_bits"] / n, 4),
+                              "payload": round(8.0 * info["payload_bytes"] / n, 4)}
+    out["note"] = ("one 4096x4096 tensor, 32 interleaved lanes per 8192-symbol chunk; each kernel K launches back "
+                   "to back between one pair of CUDA events over 40 rotating replicas; the gemv figure is one "
+                   "matrix, not a token")
+    del reps, codes, bf, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_step(args, dist, rank, world, local_rank):
+    import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    W = _override(workloads.get(WORKLOAD), args)
+    t_setup = time.perf_counter()
+    dts, infos, t_enc, _ = encode_model(entro, W, device)
+    t_setup = time.perf_counter() - t_setup
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    step = GemvStep(entro, dts, W.seed, 1, device)
+    for _ in range(max(3, args.warmup)):
+        step.launch(status)
     torch.cuda.synchronize(device)
-    dt_s = (time.perf_counter() - t0) / reps
-    d2h = host_codes.numel() + 2 * host_bf.numel() + 4 * host_y.numel()
-    return {"value": round(3 * n / dt_s / 1e9, 3), "unit": "Gsym/s", "h2d_bytes_per_step": int(nbytes),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(1e3 * dt_s, 4),
-            "note": "entro_upload from the blob's pageable host bytes (decode tables built on the host), "
-                    "three decodes, results copied to pinned host memory on a second stream as each decode "
-                    "finishes; wall clock per step"}
+    clocks = ClockSampler(device)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0  # burn-in, so that clock samples cover a loaded GPU
+    while time.perf_counter() < t_end:
+        step.launch(status)
+        torch.cuda.synchronize(device)
+    _barrier(dist, device)
+    wall0 = time.perf_counter()
+    ms = _time_launches(lambda: step.launch(status), args.steps, stream, 2e-4)
+    wall = time.perf_counter() - wall0
+    _barrier(dist, device)
+    clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    ms_max = _max_over_ranks(dist, ms, device)
+    peak, peak_kind = _peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    n = sum(i["n"] for i in infos)
+    alg = _step_bytes(infos, step)
+    achieved = alg / (ms_max * 1e-3) / 1e9
+    rec = _profile_record("kernels", "mistral_step")
+    roofline = {"bound": "hbm", "kernel": "rows_kernel<4, gemv> (one grouped launch = the whole step)",
+                "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": rec,
+                "alg_bytes": int(alg), "peak_nominal": NOMINAL_HBM_GBS,
+                "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                "issue_bound": _issue_ceiling("mistral_step", n, ms_max, clk.get("sm_mhz"), sms)}
+    e2e = _e2e_step(step, status, args.steps)
+    e2e["value"] = -_max_over_ranks(dist, -e2e["value"], device) if dist is not None else e2e["value"]
+    extras = {}
+    if not args.no_extras:
+        for b in (4, 16):
+            sb = GemvStep(entro, dts, W.seed, b, device)
+            for _ in range(3):
+                sb.launch(status)
+            mb = _time_launches(lambda: sb.launch(status), max(5, args.steps), stream, 2e-4)
+            assert int(status.item()) == 0, f"device status {int(status.item())}"
+            extras[f"mistral_batch{b}"] = {"ms": round(mb, 4), "tok_s": round(b / (mb * 1e-3), 1),
+                                          "steps_s": round(1.0 / (mb * 1e-3), 1)}
+            del sb
+        del step, dts
+        torch.cuda.empty_cache()
+        extras["smollm_bf16"] = _smollm_bf16(entro, device, stream, args.steps, peak)
+        extras[TENSOR_WORKLOAD] = _tensor_kernels(entro, device, stream, args.steps, peak, clk.get("sm_mhz"), sms)
+    if rank != 0:
+        return 0
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline(W)
+    value = world / (ms_max * 1e-3)
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "tok/s (batch 1)", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes -> bf16 x bf16 -> fp32 accumulate",
+            "data": "synthetic", "config": _step_config(W, 1), "launch_overlap": not args.no_overlap,
+            "value_definition": "tokens/s = n_gpus / step time; a step = the fused decode -> dequantize -> GEMV "
+                                "of all 224 tensors at batch 1 (one grouped launch); K steps back to back between "
+                                "one pair of CUDA events",
+            "gsym_s": round(n / (ms_max * 1e-3) / 1e9, 1),
+            "bits_per_weight": {"coded": round(sum(i["coded_bits"] for i in infos) / n, 4),
+                                "payload": round(8.0 * sum(i["payload_bytes"] for i in infos) / n, 4)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clk, "host_encode_s": round(t_enc, 2), "setup_s": round(t_setup, 2),
+            "wall_s_timed": round(wall, 4), "extras": extras}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ other workloads (not the default line)
+
+def run_model(args, dist, rank, world, local_rank):
+    """One step = one grouped launch over every tensor of a model-shaped workload: the
+    fused GEMV of a whole decode step (tok/s) or a whole-model decode to bf16."""
+    import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    W = _override(workloads.get(args.workload), args)
+    dts, infos, t_enc, _ = encode_model(entro, W, device, limit=args.tensors or None)
+    n = sum(i["n"] for i in infos)
+    coded = sum(i["coded_bits"] for i in infos) / 8.0
+    payload = sum(i["payload_bytes"] for i in infos)
+    index = sum(i["index_bytes"] for i in infos)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    gemv = args.workload != "smollm_1p7b_u8"
+    if gemv:
+        step = GemvStep(entro, dts, W.seed, args.batch, device)
+        launch = lambda: step.launch(status)  # noqa: E731
+        out_bytes = step.io_bytes
+    else:
+        outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device=device) for d in dts]
+        g = entro.Group(dts, entro.GROUP_BF16, outs=outs)
+        launch = lambda: g.launch(status=status)  # noqa: E731
+        out_bytes = 2 * n
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    clocks.start()
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        launch()
+        torch.cuda.synchronize(device)
+    _barrier(dist, device)
+    ms = _time_launches(launch, args.steps, stream, 2e-4)
+    clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    ms = _max_over_ranks(dist, ms, device)
+    if rank != 0:
+        return 0
+    peak, peak_kind = _peaks()
+    alg = coded + index + out_bytes
+    achieved = alg / (ms * 1e-3) / 1e9
+    partial = " (first %d tensors)" % len(dts) if args.tensors else ""
+    line = {"metric": METRIC,
+            "value": round(world / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
+            "unit": (f"tok/s (batch {args.batch})" if gemv else "Gsym/s") + partial, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": f"u{W.bits} codes -> bf16" + (" x bf16 -> fp32" if gemv else ""),
+            "data": "synthetic", "launch_overlap": not args.no_overlap,
+            "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
+                       "batch": args.batch if gemv else None, "format": W.fmt, "lanes": W.lanes,
+                       "l2": "working set larger than L2 (whole model)"},
+            "gsym_s": round(n / (ms * 1e-3) / 1e9, 1),
+            "bits_per_weight": {"coded": round(8 * coded / n, 4), "payload": round(8 * payload / n, 4)},
+            "roofline": {"bound": "hbm", "kernel": "grouped launch", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None},
+            "host_encode_s": round(t_enc, 2), "gpu_launches": args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tensor(args, dist, rank, world, local_rank):
+    """The 4096x4096 4-bit tensor's three kernels alone (the round-robin lanes format)."""
+    import huffman_decode_canonical_b200 as entro
+    entro.set_overlap(not args.no_overlap)
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peak, _ = _peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    clocks = ClockSampler(device)
+    clocks.start()
+    out = _tensor_kernels(entro, device, stream, args.steps, peak, None, sms)
+    clk = clocks.stop()
+    if rank == 0:
+        print(json.dumps({"workload": TENSOR_WORKLOAD, "kernels": out, "clocks": clk}), flush=True)
+    return 0
+
+
 
 
 def run_single_stream(args, dist, rank, world, local_rank):
@@ -556,80 +732,6 @@ def run_single_stream(args, dist, rank, world, local_rank):
     return 0
 
 
-def run_model(args, dist, rank, world, local_rank):
-    """One step = one grouped launch over every tensor of a model-shaped workload:
-    the fused GEMV of a whole decode step (tok/s) or a whole-model decode to bf16."""
-    import huffman_decode_canonical_b200 as entro
-    entro.set_overlap(not args.no_overlap)
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from model_helpers import encode_workload
-
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    stream = torch.cuda.current_stream(device)
-    W = workloads.get(args.workload)
-    dts, infos, t_enc = encode_workload(entro, W, device=device, limit=args.tensors or None)
-    n = sum(i["n"] for i in infos)
-    coded = sum(i["coded_bits"] for i in infos) / 8.0
-    payload = sum(i["payload_bytes"] for i in infos)
-    index = sum(i["index_bytes"] for i in infos)
-    status = torch.zeros(1, dtype=torch.int32, device=device)
-    gemv = args.workload != "smollm_1p7b_u8"
-    if gemv:
-        xs = [workloads.activations(W.seed, args.batch, d.cols).to(device) for d in dts]
-        ys = [torch.empty((args.batch, d.rows), dtype=torch.float32, device=device) for d in dts]
-        g = entro.Group(dts, entro.GROUP_GEMV, xs=xs, ys=ys, batch=args.batch)
-        out_bytes = sum(2 * x.numel() for x in xs) + sum(4 * y.numel() for y in ys)
-    else:
-        outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device=device) for d in dts]
-        g = entro.Group(dts, entro.GROUP_BF16, outs=outs)
-        out_bytes = 2 * n
-    for _ in range(args.warmup):
-        g.launch(status=status)
-    torch.cuda.synchronize(device)
-    clocks = ClockSampler(device)
-    clocks.start()
-    t_end = time.perf_counter() + 1.0
-    while time.perf_counter() < t_end:
-        g.launch(status=status)
-        torch.cuda.synchronize(device)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    _barrier(dist, device)
-    torch.cuda.synchronize(device)
-    torch.cuda._sleep(int(args.steps * 100e-6 * 2.0e9))
-    for s_ in range(args.steps):
-        ev[s_].record(stream)
-        g.launch(status=status)
-    ev[args.steps].record(stream)
-    torch.cuda.synchronize(device)
-    clk = clocks.stop()
-    assert int(status.item()) == 0, f"device status {int(status.item())}"
-    ms = sum(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)) / args.steps
-    ms = _max_over_ranks(dist, ms, device)
-    if rank != 0:
-        return 0
-    peak, peak_kind = _peaks()
-    alg = coded + index + out_bytes
-    achieved = alg / (ms * 1e-3) / 1e9
-    partial = " (first %d tensors)" % len(dts) if args.tensors else ""
-    line = {"metric": METRIC, "value": round(world / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
-            "unit": (f"tok/s (batch {args.batch})" if gemv else "Gsym/s") + partial, "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": f"u{W.bits} codes -> bf16" + (" x bf16 -> fp32" if gemv else ""),
-            "data": "synthetic", "launch_overlap": not args.no_overlap,
-            "config": {"workload": W.name, "tensors": len(dts), "symbols": n, "bits": W.bits,
-                                            "batch": args.batch if gemv else None,
-                                            "l2": "working set larger than L2 (whole model)"},
-            "gsym_s": round(n / (ms * 1e-3) / 1e9, 1),
-            "bits_per_weight": {"coded": round(8 * coded / n, 4), "payload": round(8 * payload / n, 4)},
-            "roofline": {"bound": "hbm", "kernel": "lanes_kernel grouped launch", "achieved": round(achieved, 1),
-                         "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None},
-            "host_encode_s": round(t_enc, 2), "gpu_launches": args.steps, "clocks": clk}
-    print(json.dumps(line), flush=True)
-    return 0
-
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
@@ -638,14 +740,19 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="default line without its extra workloads")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch without overlap (programmatic dependent launch, on by default)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "t4_1024x1024_u8", "smollm_1p7b_u8",
-                                                             "mistral_7b_u4", "phi3_mini_u8"],
-                    help="other workloads (not the default line): the 1024x1024 single-stream tensor, or "
-                         "model-scale workloads timed as one grouped launch per step")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, TENSOR_WORKLOAD, "t4_1024x1024_u8", "smollm_1p7b_u8", "phi3_mini_u8"],
+                    help="other workloads (not the default line): the 4096x4096 tensor's kernels, the "
+                         "1024x1024 single-stream tensor, or model-scale workloads timed as one grouped launch per "
+                         "step")
     ap.add_argument("--batch", type=int, default=1, help="GEMV batch for the model-scale GEMV workloads")
     ap.add_argument("--tensors", type=int, default=0, help="model-scale workloads: only the first N tensors")
+    ap.add_argument("--fmt", choices=["lanes", "rows"], default="", help="model-scale workloads: chunk format")
+    ap.add_argument("--lanes", type=int, default=0, help="model-scale workloads: lanes (rows per tile) per chunk")
+    ap.add_argument("--chunk", type=int, default=0, help="model-scale workloads, row tiles: symbols per chunk")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -655,9 +762,11 @@ def main(argv=None):
             return run_reference(args, rank, world)
         if args.workload == "t4_1024x1024_u8":
             return run_single_stream(args, dist, rank, world, local_rank)
-        if args.workload != WORKLOAD:
-            return run_model(args, dist, rank, world, local_rank)
-        return run_native(args, dist, rank, world, local_rank)
+        if args.workload == TENSOR_WORKLOAD:
+            return run_tensor(args, dist, rank, world, local_rank)
+        if args.workload == WORKLOAD and not args.tensors and args.batch == 1:
+            return run_step(args, dist, rank, world, local_rank)
+        return run_model(args, dist, rank, world, local_rank)
     finally:
         if dist is not None:
             dist.destroy_process_group()

@@ -30,7 +30,7 @@ OK = 0
 E_INVAL, E_LIMIT, E_FORMAT, E_CORRUPT, E_OVERRUN, E_NOMEM, E_CUDA, E_TIMEOUT = -1, -2, -3, -4, -5, -6, -7, -8
 QUANT_AUTO, QUANT_UNSIGNED, QUANT_ASYM = 0, 1, 2
 SCHEME_UNSIGNED, SCHEME_ASYM = 0, 1
-FORMAT_SINGLE, FORMAT_LANES = 1, 2
+FORMAT_SINGLE, FORMAT_LANES, FORMAT_ROWS = 1, 2, 3
 GROUP_GEMV, GROUP_BF16 = 1, 2
 
 
@@ -61,7 +61,7 @@ EXPORTS = ["entro_encode", "entro_blob_from_bytes", "entro_blob_bytes", "entro_b
            "entro_device_bytes", "entro_upload", "entro_tensor_free", "entro_decode_codes",
            "entro_decode_dequant_bf16", "entro_decode_gemv", "entro_group_table_bytes", "entro_group_prepare",
            "entro_group_launch", "entro_group_free", "entro_strerror", "entro_version", "entro_last_cuda_error",
-           "entro_decode_gemv_group_static", "entro_set_overlap"]
+           "entro_decode_gemv_group_static", "entro_set_overlap", "entro_test_stall_tables"]
 
 
 def _load() -> ctypes.CDLL:
@@ -92,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "entro_last_cuda_error": ([], ctypes.c_char_p),
         "entro_decode_gemv_group_static": ([P, P, P, I32, I32, P, P], I32),
         "entro_set_overlap": ([I32], I32),
+        "entro_test_stall_tables": ([ctypes.c_uint32], ctypes.c_uint32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -198,6 +199,8 @@ class DeviceTensor:
     def __init__(self, blob: Blob, device: Optional[torch.device] = None,
                  stream: Optional[torch.cuda.Stream] = None):
         device = torch.device(device if device is not None else "cuda")
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
         info = blob.info()
         self.rows, self.cols, self.n = info["rows"], info["cols"], info["n"]
         self.bits, self.format = info["bits"], info["format"]
@@ -305,10 +308,26 @@ def decode_gemv_group_static(tensors: Sequence[DeviceTensor], xs: Sequence[torch
                              stream: Optional[torch.cuda.Stream] = None) -> None:
     """Grouped fused GEMV whose work table lives inside the library (no device allocation)."""
     count = len(tensors)
+    if count < 1 or len(xs) != count or len(ys) != count:
+        raise ValueError("need one x and one y per tensor")
+    for t, x, y in zip(tensors, xs, ys):
+        if (x.dtype != torch.bfloat16 or not x.is_contiguous() or x.dim() != 2 or x.shape != (batch, t.cols)
+                or x.device != t.device):
+            raise ValueError("each x must be a contiguous bf16 [batch, cols] tensor on the tensors' device")
+        if (y.dtype != torch.float32 or not y.is_contiguous() or y.dim() != 2 or y.shape != (batch, t.rows)
+                or y.device != t.device):
+            raise ValueError("each y must be a contiguous fp32 [batch, rows] tensor on the tensors' device")
     arr = ctypes.c_void_p * count
     _check(_lib.entro_decode_gemv_group_static(arr(*[t._h for t in tensors]), arr(*[x.data_ptr() for x in xs]),
                                                arr(*[y.data_ptr() for y in ys]), count, batch, _dptr(status),
                                                _stream_ptr(stream)), "entro_decode_gemv_group_static")
+
+
+def test_stall_tables(extra_bytes: int) -> int:
+    """Test hook for the bounded waits: later launches wait for `extra_bytes` of table copy that
+    never arrive, so each gives up after about a second with E_TIMEOUT in the status word.
+    0 turns it off.  Returns the previous value."""
+    return int(_lib.entro_test_stall_tables(int(extra_bytes)))
 
 
 def version() -> int:
@@ -326,5 +345,6 @@ def set_overlap(enable: bool) -> bool:
 
 __all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "set_overlap", "EXPORTS",
            "decode_gemv_group_static", "STATIC_GROUP_MAX",
-           "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES", "GROUP_GEMV",
+           "test_stall_tables", "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES",
+           "FORMAT_ROWS", "GROUP_GEMV",
            "GROUP_BF16", "SCHEME_UNSIGNED", "SCHEME_ASYM"]

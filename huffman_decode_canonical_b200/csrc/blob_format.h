@@ -15,6 +15,15 @@
 // payload[chunk_start + L*j + l], so one row of 4L bytes holds word j of all
 // lanes (the interleaved lanes of the LazyWeights abstract; the run of 8
 // makes each lane's output 8 adjacent weights).
+//
+// Row-tile format (a second reading of the interleaved lanes, made for the
+// fused matrix-vector product): the [rows, cols] tensor is cut into tiles of
+// L rows by Kc = chunk_symbols / L columns, row groups outer and column tiles
+// inner, one tile per chunk.  Lane l of a tile codes row l of the tile, its Kc
+// codes (fewer in the last column tile) in column order; lanes past the last
+// row of a ragged row group are empty.  Padding and word interleave as in the
+// lanes format.  cols and Kc are multiples of 8.  The index's first_symbol is
+// the number of symbols in earlier tiles.
 #pragma once
 #include <stdint.h>
 
@@ -45,6 +54,31 @@ struct BlobHeader {
 };
 #pragma pack(pop)
 static_assert(sizeof(BlobHeader) == kHeaderBytes, "header size");
+
+// Row-tile geometry of chunk c.
+struct TileGeom {
+    int64_t row0, col0, width;  // first row, first column, columns
+    int nrows;                  // rows (lanes that hold codes)
+    uint64_t first;             // symbols in all earlier tiles
+};
+
+inline uint64_t tile_count(uint64_t rows, uint64_t cols, uint64_t lanes, uint64_t chunk_symbols) {
+    if (rows == 0 || cols == 0) return 0;
+    const uint64_t kc = chunk_symbols / lanes;
+    return ((rows + lanes - 1) / lanes) * ((cols + kc - 1) / kc);
+}
+
+inline TileGeom tile_geom(uint64_t rows, uint64_t cols, uint64_t lanes, uint64_t chunk_symbols, uint64_t c) {
+    const uint64_t kc = chunk_symbols / lanes, per_group = (cols + kc - 1) / kc;
+    const uint64_t g = c / per_group, j = c % per_group;
+    TileGeom t;
+    t.row0 = (int64_t)(g * lanes);
+    t.col0 = (int64_t)(j * kc);
+    t.nrows = (int)(rows - g * lanes < lanes ? rows - g * lanes : lanes);
+    t.width = (int64_t)(cols - j * kc < kc ? cols - j * kc : kc);
+    t.first = g * lanes * cols + (uint64_t)t.nrows * j * kc;
+    return t;
+}
 
 inline uint64_t index_offset() { return kHeaderBytes + kLengthsBytes; }
 inline uint64_t payload_offset(uint64_t n_chunks) { return index_offset() + 16 * (n_chunks + 1); }

@@ -69,6 +69,7 @@ struct DevTensor {
     const uint32_t *slow_limit;  // [32]  (first[l] + count[l]) << (max_len - l)
     const int32_t *slow_offs;    // [32]  rank of the first code of length l minus first[l]
     const uint8_t *slow_syms;    // [256] symbols sorted by (length, symbol)
+    const uint2 *wlut;           // [4096] {codes, meta}: up to 8 (4-bit) or 4 (8-bit) codes per entry
     const uint64_t *index;       // (n_chunks + 1) x {start, first_symbol}
     const uint32_t *payload;
     long long n, rows, cols, chunk_symbols, n_chunks, payload_words;
@@ -85,7 +86,7 @@ struct GroupEntry {
     long long sym_begin;     // prefix over entries, in symbols
 };
 
-static_assert(sizeof(GroupEntry) == 176, "the fixed group table is documented as 176-byte entries");
+static_assert(sizeof(GroupEntry) == 184, "the fixed group table is documented as 184-byte entries");
 
 struct LaunchArgs {
     const GroupEntry *table;  // device array, or nullptr: use `one`
@@ -98,6 +99,7 @@ struct LaunchArgs {
     long long x_elems;    // bf16 activations held in shared memory
     long long total_syms;
     int32_t *status;
+    uint32_t tx_extra;    // bytes added to the table barrier that never arrive (bounded-wait test; 0)
 };
 
 struct TensorHandle {
@@ -281,10 +283,11 @@ __device__ __forceinline__ uint32_t dequant_bf16_bits(int q, int zero, float sca
 // the canonical tables and (GEMV) the activations arrive by bulk copies on the
 // CTA barrier; thread 0 issues them at phase `tphase`.
 template <int OUT, bool SLOW>
-__device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int batch, int x_in_smem) {
+__device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int batch, int x_in_smem,
+                             uint32_t tx_extra) {
     if (threadIdx.x != 0) return;
     const DevTensor &d = g.d;
-    uint32_t bytes = kLutSize * 4;
+    uint32_t bytes = kLutSize * 4 + tx_extra;
     if (SLOW) bytes += kSlowBytes;
     const uint32_t xbytes = (OUT == OUT_GEMV && x_in_smem) ? static_cast<uint32_t>(d.cols * batch * 2) : 0u;
     bytes += xbytes;
@@ -914,7 +917,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
         long long cb = (s1 - g.sym_begin + C - 1) / C;
         if (cb > g.d.n_chunks) cb = g.d.n_chunks;
         if (ca >= cb) continue;
-        issue_tables<OUT, SLOW>(g, s, true, a.batch, a.x_in_smem);
+        issue_tables<OUT, SLOW>(g, s, true, a.batch, a.x_in_smem, a.tx_extra);
         // warp w takes chunks ca + w, ca + w + warps, ...  double buffered.  The
         // index entries of the first two are read by four lanes at once, and
         // both copies fly while the tables arrive.
@@ -938,8 +941,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
         const bool tables_ok = finish_tables<OUT, SLOW>(g, s, tphase);
         tphase++;
         if (!tables_ok) {
+            // the table barrier may never complete: give up on every later entry, let this
+            // entry's copies land (bounded waits) and leave
             set_status(a.status, ENTRO_E_TIMEOUT);
-            dead = true;
+            if (pend0) mbar_wait(bar, phase0 & 1);
+            if (pend1) mbar_wait(bar + 1, phase1 & 1);
+            if (threadIdx.x == 0) mbar_wait(s.tbar, (tphase - 1) & 1);
+            __syncthreads();
+            return;
         }
         if (!dead) {
             for (int k = 0; c < cb; c += warps, k++) {
@@ -1070,7 +1079,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
         long long cb = (s1 - g.sym_begin + C - 1) / C;
         if (cb > d.n_chunks) cb = d.n_chunks;
         if (ca >= cb) continue;
-        issue_tables<OUT_GEMV, SLOW>(g, s, true, batch, 0);
+        issue_tables<OUT_GEMV, SLOW>(g, s, true, batch, 0, a.tx_extra);
         bool pend0 = false, pend1 = false;
         if (!dead) {
             const long long c = ca + warp;
@@ -1091,7 +1100,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
         tphase++;
         if (!tables_ok) {
             set_status(a.status, ENTRO_E_TIMEOUT);
-            dead = true;
+            if (pend0) mbar_wait(bar, phase0 & 1);
+            if (pend1) mbar_wait(bar + 1, phase1 & 1);
+            if (threadIdx.x == 0) mbar_wait(s.tbar, (tphase - 1) & 1);
+            __syncthreads();
+            return;
         }
         const int K = static_cast<int>(d.cols);
         const int spr = K / (kRun * LANES);                      // runs per row
@@ -1241,6 +1254,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
     }
 }
 
+#include "rows.cuh"
+
 // ------------------------------------------------------------------ single-stream format
 //
 // One warp per chunk of the one-bitstream format (EntroLLM technical summary:
@@ -1316,10 +1331,12 @@ __global__ void __launch_bounds__(256) single_kernel(const __grid_constant__ Lau
     fence_mbar_init();
     grid_launch_dependents();
     __syncthreads();
-    issue_tables<OUT, SLOW>(g, s, false, 1, 0);
+    issue_tables<OUT, SLOW>(g, s, false, 1, 0, a.tx_extra);
     grid_wait_prior();
     if (!finish_tables<OUT, SLOW>(g, s, 0)) {
         set_status(a.status, ENTRO_E_TIMEOUT);
+        if (threadIdx.x == 0) mbar_wait(s.tbar, 0);  // bounded: let the table copy land before leaving
+        __syncthreads();
         return;
     }
     const int lane = threadIdx.x & 31;
@@ -1509,7 +1526,7 @@ __global__ void __launch_bounds__(kSegThreads) segment_kernel(const __grid_const
     if (tid == 0) {
         // tables and the chunk's words on one barrier
         const uint32_t wbytes = sane ? static_cast<uint32_t>((w1 - w0) * 4) : 0u;
-        uint32_t bytes = kLutSize * 4 + wbytes;
+        uint32_t bytes = kLutSize * 4 + wbytes + a.tx_extra;
         if (SLOW) bytes += kSlowBytes;
         mbar_arrive_expect_tx(s.tbar, bytes);
         bulk_copy_g2s(s.lut, d.lut, kLutSize * 4, s.tbar);
@@ -1520,6 +1537,8 @@ __global__ void __launch_bounds__(kSegThreads) segment_kernel(const __grid_const
     grid_wait_prior();
     if (!finish_tables<OUT, SLOW>(g, s, 0)) {
         set_status(a.status, ENTRO_E_TIMEOUT);
+        if (tid == 0) mbar_wait(s.tbar, 0);  // bounded: let the copies land before leaving
+        __syncthreads();
         return;
     }
     if (!sane) {
@@ -1705,7 +1724,9 @@ static int device_info(int dev, DeviceInfo *out) {
 //   mlut: 12-bit peek -> every whole code inside the 12 bits, up to 6 (4-bit)
 //         or 3 (8-bit): bits used | count << 4 | symbols << 8
 //   limit / offs / syms: canonical description for codes longer than 12 bits
-static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lut, uint32_t *mlut,
+//   wlut: 12-bit peek -> {every whole code inside the 12 bits, up to 8 (4-bit)
+//         or 4 (8-bit), first code in the low bits; bits used | count * bits << 8}
+static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lut, uint32_t *mlut, uint32_t *wlut,
                          uint32_t *limit, int32_t *offs, uint8_t *syms, int *n_codes) {
     uint32_t code[256];
     canonical_codes(len, code);
@@ -1736,6 +1757,20 @@ static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lu
         }
         mlut[v] = used | (k << 4) | (packed << 8);
     }
+    const int wide = wide_max_codes(bits);
+    for (uint32_t v = 0; v < (uint32_t)kLutSize; v++) {
+        uint32_t used = 0, k = 0, packed = 0;
+        while ((int)k < wide) {
+            const uint32_t e = lut[(v << used) & (kLutSize - 1)];
+            const uint32_t l = e & 31u;
+            if (l == 0 || used + l > (uint32_t)kMaxLutBits) break;
+            packed |= ((e >> 8) & 0xFFu) << (bits * k);
+            used += l;
+            k++;
+        }
+        wlut[2 * v] = packed;
+        wlut[2 * v + 1] = used | ((k * (uint32_t)bits) << kPbShift);
+    }
     uint32_t first[33] = {0};
     int base[33] = {0};
     uint32_t c = 0;
@@ -1762,14 +1797,15 @@ static void build_tables(const uint8_t *len, int max_len, int bits, uint32_t *lu
 }
 
 struct ImageLayout {
-    uint64_t lut, mlut, slow, index, payload, total;
+    uint64_t lut, mlut, wlut, slow, index, payload, total;
 };
 
 static ImageLayout image_layout(const Blob &b) {
     ImageLayout L;
     L.lut = 0;
     L.mlut = align256(L.lut + kLutSize * 4);
-    L.slow = align256(L.mlut + kLutSize * 4);
+    L.wlut = align256(L.mlut + kLutSize * 4);
+    L.slow = align256(L.wlut + kWideLutBytes);
     L.index = align256(L.slow + kSlowBytes);
     L.payload = align256(L.index + 16 * (b.header.n_chunks + 1));
     L.total = align256(L.payload + 4 * (b.header.payload_words + kPadWords));
@@ -1793,7 +1829,7 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     const Blob &b = *reinterpret_cast<const Blob *>(blob);
     const ImageLayout L = image_layout(b);
     if (d_bytes < L.total || (reinterpret_cast<uintptr_t>(d_mem) & 255)) return ENTRO_E_INVAL;
-    if (b.header.format == ENTRO_FORMAT_LANES && b.max_chunk_words > 16384) return ENTRO_E_LIMIT;
+    if (b.header.format != ENTRO_FORMAT_SINGLE && b.max_chunk_words > 16384) return ENTRO_E_LIMIT;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ENTRO_E_CUDA;
     TensorHandle *t = new (std::nothrow) TensorHandle();
@@ -1801,11 +1837,13 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     std::vector<uint8_t> host(L.index - L.lut, 0);
     uint32_t *lut = reinterpret_cast<uint32_t *>(host.data());
     uint32_t *mlut = reinterpret_cast<uint32_t *>(host.data() + L.mlut);
+    uint32_t *wlut = reinterpret_cast<uint32_t *>(host.data() + L.wlut);
     uint32_t *limit = reinterpret_cast<uint32_t *>(host.data() + L.slow);
     int32_t *offs = reinterpret_cast<int32_t *>(host.data() + L.slow + 128);
     uint8_t *syms = host.data() + L.slow + 256;
     int n_codes = 0;
-    build_tables(b.lengths, (int)b.header.max_len, (int)b.header.bits, lut, mlut, limit, offs, syms, &n_codes);
+    build_tables(b.lengths, (int)b.header.max_len, (int)b.header.bits, lut, mlut, wlut, limit, offs, syms,
+                 &n_codes);
     uint8_t *base = static_cast<uint8_t *>(d_mem);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint8_t *src = b.bytes.data();
@@ -1827,6 +1865,7 @@ extern "C" int entro_upload(const entro_blob *blob, void *d_mem, uint64_t d_byte
     DevTensor &d = t->d;
     d.lut = reinterpret_cast<const uint32_t *>(base + L.lut);
     d.mlut = reinterpret_cast<const uint32_t *>(base + L.mlut);
+    d.wlut = reinterpret_cast<const uint2 *>(base + L.wlut);
     d.slow_limit = reinterpret_cast<const uint32_t *>(base + L.slow);
     d.slow_offs = reinterpret_cast<const int32_t *>(base + L.slow + 128);
     d.slow_syms = base + L.slow + 256;
@@ -1966,6 +2005,8 @@ static int kernel_config(const void *fn, int device, int threads, size_t bytes, 
 
 // Launch overlap (programmatic dependent launch), off unless the caller turns it on.
 static std::atomic<int> g_overlap{0};
+// Bounded-wait test hook: bytes every launch adds to its table barrier that never arrive.
+static std::atomic<uint32_t> g_tx_extra{0};
 
 // overlap_ok: the kernel fills each SM with one CTA (the next launch's CTAs
 // cannot move in before this one's leave).  Kernels with several CTAs per SM
@@ -2084,8 +2125,90 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     a.x_elems = x_elems;
     a.total_syms = total;
     a.status = status;
+    a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
     const cudaError_t e = launch(fn, (unsigned)grid, warps * 32, bytes, st, a, overlap_ok);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
+}
+
+template <int BITS, int OUT, int LANES>
+static LanesFn pick_rows3(bool slow, int nb) {
+    if (OUT != OUT_GEMV) return slow ? rows_kernel<BITS, OUT, true, LANES, 1> : rows_kernel<BITS, OUT, false, LANES, 1>;
+    if (nb == 2) return slow ? rows_kernel<BITS, OUT, true, LANES, 2> : rows_kernel<BITS, OUT, false, LANES, 2>;
+    return slow ? rows_kernel<BITS, OUT, true, LANES, 1> : rows_kernel<BITS, OUT, false, LANES, 1>;
+}
+
+template <int BITS, int LANES>
+static LanesFn pick_rows2(int out, bool slow, int nb) {
+    if (out == OUT_CODES) return pick_rows3<BITS, OUT_CODES, LANES>(slow, nb);
+    if (out == OUT_BF16) return pick_rows3<BITS, OUT_BF16, LANES>(slow, nb);
+    return pick_rows3<BITS, OUT_GEMV, LANES>(slow, nb);
+}
+
+static LanesFn pick_rows(int bits, int out, bool slow, int nb, int lanes) {
+    if (bits == 4) return lanes == 64 ? pick_rows2<4, 64>(out, slow, nb) : pick_rows2<4, 32>(out, slow, nb);
+    return lanes == 64 ? pick_rows2<8, 64>(out, slow, nb) : pick_rows2<8, 32>(out, slow, nb);
+}
+
+// Launch the row-tile kernel over `count` entries (table on device, or `one`).
+static int launch_rows(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
+                       const GroupEntry &one, int32_t *status, cudaStream_t st) {
+    bool slow = false;
+    const int bits = ts[0]->d.bits, lanes = ts[0]->d.lanes;
+    int max_words = 0;
+    long long max_runs = 0, total = 0, units = 0;
+    for (int i = 0; i < count; i++) {
+        const DevTensor &d = ts[i]->d;
+        if (d.format != ENTRO_FORMAT_ROWS || d.bits != bits || d.lanes != lanes) return ENTRO_E_INVAL;
+        slow = slow || ts[i]->slow;
+        max_words = std::max(max_words, d.max_chunk_words);
+        max_runs = std::max(max_runs, d.chunk_symbols / lanes / kRun);
+        total += d.n;
+        units += d.n_chunks;  // tiles
+    }
+    if (total == 0) return ENTRO_OK;
+    DeviceInfo di;
+    if (device_info(ts[0]->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
+    const int nb = out_kind == OUT_GEMV && batch > 8 ? 2 : 1;
+    LanesFn fn = pick_rows(bits, out_kind, slow, nb, lanes);
+    const int stage_rows = max_words + kSlackRows;
+    // a run slot for every run of a chunk, plus the runs a lane may complete past its last check
+    int run_buf_bytes = static_cast<int>(max_runs + wide_runs_per_check(bits, 6)) * rows_run_bytes(bits, lanes);
+    // the GEMV parks two sets of partial sums (fp32 D fragments) in a warp's run buffer
+    if (out_kind == OUT_GEMV) run_buf_bytes = std::max(run_buf_bytes, 2 * (lanes / 16) * nb * 4 * 32 * 4);
+    int warps = (int)std::min<long long>(kMaxWarps, std::max<long long>(1, (units + di.sms - 1) / di.sms));
+    RowsLayout rl;
+    for (;;) {
+        rl = rows_layout(warps, stage_rows * lanes, run_buf_bytes);
+        if ((long long)rl.total <= di.smem_optin) break;
+        if (warps > 1) warps--;
+        else return ENTRO_E_LIMIT;
+    }
+    int per_sm = 0;
+    if (kernel_config(reinterpret_cast<const void *>(fn), ts[0]->device, warps * 32, rl.total, &per_sm) != ENTRO_OK)
+        return ENTRO_E_CUDA;
+    long long grid = std::min<long long>((units + warps - 1) / warps, (long long)per_sm * di.sms);
+    grid = std::max<long long>(grid, 1);
+    LaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.table = d_table;
+    a.one = one;
+    a.count = count;
+    a.batch = batch;
+    a.stage_rows = stage_rows;
+    a.out_words = run_buf_bytes / 4;
+    a.total_syms = total;
+    a.status = status;
+    a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
+    const cudaError_t e = launch(fn, (unsigned)grid, warps * 32, rl.total, st, a, per_sm <= 2);
+    return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "row-tile kernel launch");
+}
+
+// A grouped launch of tensors of one format.
+static int launch_group(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
+                        const GroupEntry &one, int32_t *status, cudaStream_t st) {
+    if (ts[0]->d.format == ENTRO_FORMAT_ROWS)
+        return launch_rows(ts, count, out_kind, batch, d_table, one, status, st);
+    return launch_lanes(ts, count, out_kind, batch, d_table, one, status, st);
 }
 
 static LanesFn pick_segment(int bits, int out, bool slow) {
@@ -2118,6 +2241,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
         a.batch = 1;
         a.stage_rows = stage_words;
         a.status = status;
+        a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
         const cudaError_t e = launch(fn, (unsigned)d.n_chunks, kSegThreads, sl.total, st, a, false);
         return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "segment kernel launch");
     }
@@ -2134,6 +2258,7 @@ static int launch_single(const TensorHandle *t, int out_kind, void *out, int32_t
     a.count = 1;
     a.batch = 1;
     a.status = status;
+    a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
     const long long grid = (d.n_chunks * 32 + threads - 1) / threads;
     const cudaError_t e = launch(fn, (unsigned)grid, threads, bytes, st, a, false);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "single kernel launch");
@@ -2154,13 +2279,14 @@ static int decode_one(const entro_tensor *tensor, int out_kind, void *out, int32
     std::memset(&one, 0, sizeof(one));
     one.d = t->d;
     one.out = out;
-    return launch_lanes(&t, 1, out_kind, 1, nullptr, one, status, st);
+    return launch_group(&t, 1, out_kind, 1, nullptr, one, status, st);
 }
 
 static int gemv_check(const TensorHandle *t, const void *x, int batch, const float *y) {
     if (!t || !x || !y || batch < 1 || batch > kMaxBatch) return ENTRO_E_INVAL;
     if (reinterpret_cast<uintptr_t>(x) & 15) return ENTRO_E_INVAL;
     const DevTensor &d = t->d;
+    if (d.format == ENTRO_FORMAT_ROWS) return ENTRO_OK;  // any shape of the format (cols a multiple of 8)
     if (d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
     if (d.cols <= 0 || d.cols % (kRun * d.lanes) || d.chunk_symbols % d.cols) return ENTRO_E_INVAL;
     return ENTRO_OK;
@@ -2186,7 +2312,7 @@ extern "C" int entro_decode_gemv(const entro_tensor *tensor, const void *d_x, in
     one.d = t->d;
     one.x = static_cast<const __nv_bfloat16 *>(d_x);
     one.y = d_y;
-    return launch_lanes(&t, 1, OUT_GEMV, batch, nullptr, one, d_status, static_cast<cudaStream_t>(stream));
+    return launch_group(&t, 1, OUT_GEMV, batch, nullptr, one, d_status, static_cast<cudaStream_t>(stream));
 }
 
 namespace entro {
@@ -2222,10 +2348,12 @@ extern "C" int entro_group_prepare(const entro_tensor *const *tensors, int32_t c
     for (int i = 0; i < count; i++) {
         const TensorHandle *t = reinterpret_cast<const TensorHandle *>(tensors[i]);
         int r = ENTRO_OK;
-        if (!t || t->d.format != ENTRO_FORMAT_LANES) r = ENTRO_E_INVAL;
+        if (!t || t->d.format == ENTRO_FORMAT_SINGLE) r = ENTRO_E_INVAL;
         else if (out_kind == OUT_GEMV) r = gemv_check(t, xs[i], batch, ys[i]);
         else if (!outs[i] || (reinterpret_cast<uintptr_t>(outs[i]) & 15)) r = ENTRO_E_INVAL;
-        if (r == ENTRO_OK && i > 0 && (t->device != h->ts[0]->device || t->d.bits != h->ts[0]->d.bits))
+        if (r == ENTRO_OK && i > 0 &&
+            (t->device != h->ts[0]->device || t->d.bits != h->ts[0]->d.bits || t->d.format != h->ts[0]->d.format ||
+             t->d.lanes != h->ts[0]->d.lanes))
             r = ENTRO_E_INVAL;
         if (r != ENTRO_OK) {
             delete h;
@@ -2264,7 +2392,7 @@ extern "C" int entro_group_prepare(const entro_tensor *const *tensors, int32_t c
 extern "C" int entro_group_launch(const entro_group *group, int32_t *d_status, void *stream) {
     if (!group) return ENTRO_E_INVAL;
     const GroupHandle *h = reinterpret_cast<const GroupHandle *>(group);
-    return launch_lanes(h->ts.data(), (int)h->ts.size(), h->kind, h->batch, h->d_table, h->first, d_status,
+    return launch_group(h->ts.data(), (int)h->ts.size(), h->kind, h->batch, h->d_table, h->first, d_status,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -2300,10 +2428,12 @@ extern "C" int entro_decode_gemv_group_static(const entro_tensor *const *tensors
     const TensorHandle *const *ts = reinterpret_cast<const TensorHandle *const *>(tensors);
     for (int i = 0; i < count; i++) {
         const TensorHandle *t = ts[i];
-        if (!t || t->d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
+        if (!t || t->d.format == ENTRO_FORMAT_SINGLE) return ENTRO_E_INVAL;
         const int r = gemv_check(t, xs[i], batch, ys[i]);
         if (r != ENTRO_OK) return r;
-        if (t->device != ts[0]->device || t->d.bits != ts[0]->d.bits) return ENTRO_E_INVAL;
+        if (t->device != ts[0]->device || t->d.bits != ts[0]->d.bits || t->d.format != ts[0]->d.format ||
+            t->d.lanes != ts[0]->d.lanes)
+            return ENTRO_E_INVAL;
     }
     const int dev = ts[0]->device;
     int cur = -1;
@@ -2343,7 +2473,7 @@ extern "C" int entro_decode_gemv_group_static(const entro_tensor *const *tensors
                                               cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (static group table)");
     }
-    return launch_lanes(ts, count, OUT_GEMV, batch, static_cast<const GroupEntry *>(table), first, d_status, st);
+    return launch_group(ts, count, OUT_GEMV, batch, static_cast<const GroupEntry *>(table), first, d_status, st);
 }
 
 extern "C" const char *entro_strerror(int code) {
@@ -2364,5 +2494,9 @@ extern "C" const char *entro_strerror(int code) {
 extern "C" int entro_version(void) { return 100; }
 
 extern "C" ENTRO_API int entro_set_overlap(int enable) { return entro::g_overlap.exchange(enable ? 1 : 0); }
+
+extern "C" ENTRO_API uint32_t entro_test_stall_tables(uint32_t extra_bytes) {
+    return entro::g_tx_extra.exchange(extra_bytes);
+}
 
 extern "C" const char *entro_last_cuda_error(void) { return g_cuda_msg; }

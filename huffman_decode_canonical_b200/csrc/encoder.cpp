@@ -319,18 +319,21 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     if ((rows * cols > 0) && !w) return ENTRO_E_INVAL;
     if (o->bits != 4 && o->bits != 8) return ENTRO_E_INVAL;
     if (o->quant_mode < 0 || o->quant_mode > 2) return ENTRO_E_INVAL;
-    if (o->format != ENTRO_FORMAT_SINGLE && o->format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
+    if (o->format != ENTRO_FORMAT_SINGLE && o->format != ENTRO_FORMAT_LANES && o->format != ENTRO_FORMAT_ROWS)
+        return ENTRO_E_INVAL;
     if (o->threads < 0) return ENTRO_E_INVAL;
     const int bits = o->bits, nsym = 1 << bits;
     const int max_len = o->max_len ? o->max_len : (bits == 8 ? 16 : 12);
     if (max_len < 1 || max_len > kMaxLenLimit) return ENTRO_E_INVAL;
-    const bool lanes = o->format == ENTRO_FORMAT_LANES;
+    const bool tiles = o->format == ENTRO_FORMAT_ROWS;
+    const bool lanes = o->format == ENTRO_FORMAT_LANES || tiles;  // word-interleaved lanes
     const int L = lanes ? (o->lanes ? o->lanes : kLanes) : 1;
     if (lanes && L != 32 && L != 64) return ENTRO_E_INVAL;
     const int64_t step = (int64_t)kRun * L;
     int64_t C = o->chunk_symbols ? o->chunk_symbols : (lanes ? 8192 : 4096);
     if (lanes && (C < step || C > kMaxLanesChunk || C % step)) return ENTRO_E_INVAL;
     if (!lanes && (C < 1 || C > kMaxSingleChunk)) return ENTRO_E_INVAL;
+    if (tiles && cols % kRun) return ENTRO_E_INVAL;
     const int64_t n = rows * cols;
     const int threads = pick_threads(o->threads, n);
 
@@ -361,7 +364,8 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     uint32_t code[256];
     canonical_codes(len, code);
 
-    const uint64_t n_chunks = n > 0 ? (uint64_t)((n + C - 1) / C) : 0;
+    const uint64_t n_chunks = tiles ? tile_count((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C)
+                                    : n > 0 ? (uint64_t)((n + C - 1) / C) : 0;
     std::vector<uint64_t> start(n_chunks + 1, 0);
 
     // pass 1: per-chunk size (bits for single stream, words for lanes)
@@ -369,7 +373,17 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     parallel_for(threads, (int64_t)n_chunks, [&](int64_t c0, int64_t c1, int) {
         for (int64_t c = c0; c < c1; c++) {
             const int64_t a = c * C, b = std::min<int64_t>(n, a + C);
-            if (!lanes) {
+            if (tiles) {
+                const TileGeom t = tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, (uint64_t)c);
+                uint64_t wmax = 0;
+                for (int l = 0; l < t.nrows; l++) {
+                    const uint8_t *row = q.data() + (t.row0 + l) * cols + t.col0;
+                    uint64_t s = 0;
+                    for (int64_t k = 0; k < t.width; k++) s += len[row[k]];
+                    wmax = std::max<uint64_t>(wmax, (s + 31) / 32);
+                }
+                csize[c] = wmax * (uint64_t)L;
+            } else if (!lanes) {
                 uint64_t s = 0;
                 for (int64_t i = a; i < b; i++) s += len[q[i]];
                 csize[c] = s;
@@ -419,6 +433,9 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     for (uint64_t c = 0; c <= n_chunks; c++) {
         idx[2 * c] = start[c];
         idx[2 * c + 1] = std::min<uint64_t>((uint64_t)n, c * (uint64_t)C);
+        if (tiles)
+            idx[2 * c + 1] = c < n_chunks ? tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, c).first
+                                          : (uint64_t)n;
     }
     uint32_t *payload = reinterpret_cast<uint32_t *>(base + payload_offset(n_chunks));
 
@@ -427,7 +444,16 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
         std::vector<uint32_t> tmp;
         for (int64_t c = c0; c < c1; c++) {
             const int64_t a = c * C, b = std::min<int64_t>(n, a + C);
-            if (!lanes) {
+            if (tiles) {
+                const TileGeom t = tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, (uint64_t)c);
+                uint32_t *cbase = payload + start[c];
+                for (int l = 0; l < t.nrows; l++) {
+                    BitSink s{cbase + l, L};
+                    const uint8_t *row = q.data() + (t.row0 + l) * cols + t.col0;
+                    for (int64_t k = 0; k < t.width; k++) s.put(code[row[k]], len[row[k]]);
+                    s.flush();
+                }
+            } else if (!lanes) {
                 // chunks are bit-contiguous: write this chunk's bits into a
                 // private word buffer aligned like the payload, then OR the
                 // edge words (shared with neighbours) atomically.
@@ -483,7 +509,8 @@ int Blob::finalize_info() {
     if (h.bits != 4 && h.bits != 8) return ENTRO_E_FORMAT;
     if (h.scheme > 1) return ENTRO_E_FORMAT;
     if (h.max_len < 1 || h.max_len > (uint32_t)kMaxLenLimit) return ENTRO_E_FORMAT;
-    const bool lanes = h.format == ENTRO_FORMAT_LANES;
+    const bool tiles = h.format == ENTRO_FORMAT_ROWS;
+    const bool lanes = h.format == ENTRO_FORMAT_LANES || tiles;
     if (!lanes && h.format != ENTRO_FORMAT_SINGLE) return ENTRO_E_FORMAT;
     if (lanes ? (h.lanes != 32 && h.lanes != 64) : h.lanes != 1) return ENTRO_E_FORMAT;
     if (h.run != (lanes ? (uint32_t)kRun : 1u)) return ENTRO_E_FORMAT;
@@ -493,7 +520,10 @@ int Blob::finalize_info() {
     if (!lanes && h.chunk_symbols > (uint64_t)kMaxSingleChunk) return ENTRO_E_FORMAT;
     if (h.cols != 0 && h.rows > UINT64_MAX / h.cols) return ENTRO_E_FORMAT;
     if (h.n != h.rows * h.cols) return ENTRO_E_FORMAT;
-    if (h.n_chunks != (h.n + h.chunk_symbols - 1) / h.chunk_symbols) return ENTRO_E_FORMAT;
+    if (tiles && h.cols % kRun) return ENTRO_E_FORMAT;
+    if (h.n_chunks != (tiles ? tile_count(h.rows, h.cols, h.lanes, h.chunk_symbols)
+                             : (h.n + h.chunk_symbols - 1) / h.chunk_symbols))
+        return ENTRO_E_FORMAT;
     if (h.n_chunks > (uint64_t(1) << 40) || h.payload_words > (uint64_t(1) << 40)) return ENTRO_E_FORMAT;
     if (bytes.size() != (size_t)(payload_offset(h.n_chunks) + 4 * h.payload_words)) return ENTRO_E_FORMAT;
     int nz = 0;
@@ -517,7 +547,10 @@ int Blob::finalize_info() {
     uint64_t maxw = 0, prev = 0;
     for (uint64_t c = 0; c <= h.n_chunks; c++) {
         const uint64_t st = idx[2 * c], first = idx[2 * c + 1];
-        if (first != std::min<uint64_t>(h.n, c * h.chunk_symbols)) return ENTRO_E_FORMAT;
+        const uint64_t want = !tiles ? std::min<uint64_t>(h.n, c * h.chunk_symbols)
+                              : c < h.n_chunks ? tile_geom(h.rows, h.cols, h.lanes, h.chunk_symbols, c).first
+                                               : h.n;
+        if (first != want) return ENTRO_E_FORMAT;
         if (c == 0 ? st != 0 : st < prev) return ENTRO_E_FORMAT;
         if (c > 0 && lanes) {
             const uint64_t wc = st - prev;

@@ -66,17 +66,20 @@ extern "C" {
  * LazyWeights abstract, interleaved lanes). */
 #define ENTRO_FORMAT_SINGLE 1 /* one bitstream per chunk, chunks bit-contiguous */
 #define ENTRO_FORMAT_LANES 2  /* 32 (or 64) word-interleaved lane bitstreams per chunk */
+#define ENTRO_FORMAT_ROWS 3   /* row tiles: a chunk is L = 32 (or 64) rows by chunk_symbols / L columns,
+                                 lane l holding row l of the tile; word-interleaved like LANES.  Made for
+                                 the fused GEMV; cols must be a multiple of 8 */
 
 typedef struct entro_encode_opts {
     int32_t bits;          /* 4 or 8 */
     int32_t quant_mode;    /* ENTRO_QUANT_* */
     int32_t max_len;       /* code length limit, 1..24; 0 = 16 for 8-bit, 12 for 4-bit */
     int32_t format;        /* ENTRO_FORMAT_* */
-    int64_t chunk_symbols; /* 0 = 4096 (single) / 8192 (lanes).  Lanes: a multiple of 8 * lanes
-                              in [8 * lanes, 16384].  Single: 1 .. 2^20. */
+    int64_t chunk_symbols; /* 0 = 4096 (single) / 8192 (lanes, rows).  Lanes and rows: a multiple of
+                              8 * lanes in [8 * lanes, 16384].  Single: 1 .. 2^20. */
     int32_t threads;       /* host threads for encoding; 0 = all hardware threads */
-    int32_t lanes;         /* lanes format: 32 (also 0) or 64 interleaved lanes per chunk; a chunk
-                              must then hold a multiple of 8 * lanes symbols */
+    int32_t lanes;         /* lanes / rows formats: 32 (also 0) or 64 interleaved lanes per chunk; a
+                              chunk must then hold a multiple of 8 * lanes symbols */
 } entro_encode_opts;
 
 typedef struct entro_blob entro_blob;     /* host copy of one encoded tensor (serialized bytes) */
@@ -148,13 +151,15 @@ ENTRO_API int entro_decode_dequant_bf16(const entro_tensor *t, void *d_out, int3
 /* Fused decode -> dequantize -> GEMV for token generation: for b < batch and
  * r < rows, d_y[b*rows + r] = sum_k w[r,k] * x[b*cols + k], w the bf16
  * weights of entro_decode_dequant_bf16 (never written to memory), x bf16
- * [batch, cols], accumulation in fp32.  Needs the lanes format, cols a
- * multiple of 8 * lanes (256 or 512) and chunk_symbols a multiple of cols
- * (chunks of whole rows); batch in 1..16; d_x 16-byte aligned.  Batch 1-2:
- * fp32 FMAs of the bf16 products in the decoding warp; batch 3-16: the
- * tensor cores (mma.sync, bf16 operands, fp32 accumulation) with the warps of
- * a block decoding consecutive rows.  Rows are reduced in a fixed order, so
- * results are bit-reproducible. */
+ * [batch, cols], accumulation in fp32; batch in 1..16; d_x 16-byte aligned.
+ * Row-tile format (any shape of it): a warp decodes a tile's 32 (64) rows and
+ * multiplies them on the tensor cores (mma.sync m16n8k16, bf16 operands,
+ * fp32 accumulation) for every batch size.  Lanes format: cols a multiple of
+ * 8 * lanes (256 or 512) and chunk_symbols a multiple of cols (chunks of
+ * whole rows); batch 1-2 use fp32 FMAs of the bf16 products in the decoding
+ * warp, batch 3-16 the tensor cores with the warps of a block decoding
+ * consecutive rows.  Every sum is taken in a fixed order, so results are
+ * bit-reproducible. */
 ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t batch, float *d_y,
                       int32_t *d_status, void *stream);
 
@@ -167,13 +172,13 @@ ENTRO_API int entro_decode_gemv(const entro_tensor *t, const void *d_x, int32_t 
  * entro_group_launch then launches without any host-device traffic, as often
  * as wanted (for instance once per generated token).  d_table, the tensors'
  * device images and the x / y / output buffers must stay valid while the
- * handle is used; all tensors must share the device, the bit width and the
- * lane count (E_INVAL: entro_group_prepare checks the device and bit width,
- * entro_group_launch the lane count).
+ * handle is used; all tensors must share the device, the bit width, the
+ * format (lanes or row tiles) and the lane count (E_INVAL from
+ * entro_group_prepare otherwise).
  * kind:
  *   ENTRO_GROUP_GEMV  xs[i] bf16 [batch, cols_i], ys[i] fp32 [batch, rows_i]
  *                     (the per-tensor rules of entro_decode_gemv apply)
- *   ENTRO_GROUP_BF16  outs[i] bf16 [rows_i, cols_i] (lanes format only) */
+ *   ENTRO_GROUP_BF16  outs[i] bf16 [rows_i, cols_i] (lanes or row-tile format) */
 #define ENTRO_GROUP_GEMV 1
 #define ENTRO_GROUP_BF16 2
 typedef struct entro_group entro_group;
@@ -191,7 +196,7 @@ ENTRO_API const char *entro_strerror(int code);
  * that reserves the whole device up front and allows no cudaMalloc later.  No
  * counterpart on the EntroLLM or LazyWeights pages: it only changes where the
  * launch's work table lives.  The table is a fixed array inside the library
- * (ENTRO_STATIC_GROUP_MAX entries of 176 bytes, about 88 KB, held on every
+ * (ENTRO_STATIC_GROUP_MAX entries of 184 bytes, about 92 KB, held on every
  * GPU that loads the library until the process exits); the caller still
  * passes the uploaded tensors, the activations xs[i] (bf16 [batch, cols_i])
  * and the outputs ys[i] (fp32 [batch, rows_i]), with the rules of
@@ -224,6 +229,15 @@ ENTRO_API int entro_decode_gemv_group_static(const entro_tensor *const *tensors,
  * image (copies, such as entro_upload's, are always waited for).  Process-
  * wide; off by default.  Returns the previous setting. */
 ENTRO_API int entro_set_overlap(int enable);
+
+/* Test hook for the bounded waits (no counterpart on the pages).  With
+ * extra_bytes > 0, every later launch declares extra_bytes more on the
+ * barrier of its decode-table copy than the copy delivers, so that barrier
+ * never completes: the kernel's bounded wait gives up after about a second,
+ * writes ENTRO_E_TIMEOUT to the status word, lets its copies in flight land
+ * (again a bounded wait) and returns; outputs are then incomplete.  0 (the
+ * default) turns it off.  Process-wide; returns the previous value. */
+ENTRO_API uint32_t entro_test_stall_tables(uint32_t extra_bytes);
 
 /* Text of the last CUDA runtime error behind an ENTRO_E_CUDA return on the
  * calling host thread ("" if none). */

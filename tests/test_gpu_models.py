@@ -1,22 +1,31 @@
-"""Full-size parity on the model-shaped workloads, in the launch configuration the
-grouped kernels use (one launch over every tensor).
+"""Full-size parity on the model-shaped workloads, every tensor of every model.
 
-Whole-model outputs are too large for the oracle to recompute in full; sampled
-tensors are checked completely (codes via bf16 bit patterns, every GEMV row),
-and properties that hold at any size (status word, finiteness) are checked
-everywhere.
+* Codes and bf16 weights: the GPU's decode of every tensor is compared bit for bit
+  with the oracle's quantization (codes) and dequantization (bf16) of the same
+  seeded tensor.  SmolLM-shaped: the whole model in one grouped bf16 launch (the
+  benchmark's launch); Mistral- and Phi-3-shaped: codes and bf16 of every tensor.
+* Fused GEMV: one grouped launch over every tensor of the model (the benchmark's
+  decode step), at each batch size of the configuration; sampled rows of every
+  tensor (first, last and evenly spaced) against the oracle's fp64 product of the
+  oracle's bf16 weights, within 2e-3 of sum |w x|.
+
+The oracle's work for a tensor (quantize, dequantize, compare) runs on worker
+threads while the GPU decodes the next tensor.
 """
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads
-from model_helpers import encode_workload, sample_indices
+from model_helpers import encode_workload
 
 pytestmark = pytest.mark.gpu
 
 GEMV_TOL = 2e-3
+SAMPLE_ROWS = 16
 
 
 @pytest.fixture(scope="module")
@@ -31,82 +40,115 @@ def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
 
 
-def _oracle_weights(W, spec):
-    w = workloads.weights(W, spec, device="cuda").cpu().numpy()
+def _pack4(q):
+    return (q[0::2] | (q[1::2] << 4)).astype(np.uint8)
+
+
+def _sample_rows(rows):
+    return np.unique(np.linspace(0, rows - 1, min(rows, SAMPLE_ROWS)).round().astype(np.int64))
+
+
+def _check_tensor(W, spec, w, info, got_bf, got_codes):
     q, s, z, scheme = oracle.quantize(w, W.bits, W.quant_mode)
-    return q, s, z, scheme
+    assert (info["scheme"], info["scale"], info["zero"]) == (scheme, s, z), spec.name
+    ref = oracle.dequant_bf16(q, s, z)
+    assert np.array_equal(got_bf, ref), spec.name
+    if got_codes is not None:
+        assert np.array_equal(got_codes, q if W.bits == 8 else _pack4(q)), spec.name
+    rows = _sample_rows(spec.rows)
+    return rows, ref.reshape(spec.rows, spec.cols)[rows]
+
+
+def _decode_and_check(entro, W, dts, infos, codes=True, bf16_group=False):
+    """Decode every tensor on the GPU and check it against the oracle; returns the sampled
+    rows of every tensor for the GEMV checks."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = None
+    if bf16_group:
+        outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device="cuda") for d in dts]
+        entro.Group(dts, entro.GROUP_BF16, outs=outs).launch(status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+    samples = [None] * len(dts)
+    pending = []
+    with ThreadPoolExecutor(8) as pool:
+        for i, (spec, dt) in enumerate(zip(W.tensors, dts)):
+            w = workloads.weights(W, spec, device="cuda").cpu().numpy()
+            if outs is not None:
+                got_bf = _bits(outs[i])
+                outs[i] = None
+            else:
+                got_bf = _bits(dt.decode_dequant_bf16(status=st))
+            got_codes = dt.decode_codes(status=st).cpu().numpy()[: dt.codes_nbytes()] if codes else None
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0, spec.name
+            pending.append((i, pool.submit(_check_tensor, W, spec, w, infos[i], got_bf, got_codes)))
+            del w, got_bf, got_codes
+            while len(pending) > 8:
+                j, f = pending.pop(0)
+                samples[j] = f.result()
+        for j, f in pending:
+            samples[j] = f.result()
+    return samples
+
+
+def _gemv_check(entro, W, dts, samples, batch):
+    """One grouped launch over every tensor (the benchmark's step); sampled rows of every
+    tensor against the oracle.  Tensors with the same column count share activations."""
+    xs = {K: workloads.activations(W.seed + batch, batch, K).cuda() for K in set(d.cols for d in dts)}
+    ys = [torch.full((batch, d.rows), float("nan"), device="cuda") for d in dts]
+    g = entro.Group(dts, entro.GROUP_GEMV, xs=[xs[d.cols] for d in dts], ys=ys, batch=batch)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.launch(status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    xbits = {K: workloads.bf16_bits(x.cpu()) for K, x in xs.items()}
+    worst = 0.0
+    for spec, d, y, (rows, wb) in zip(W.tensors, dts, ys, samples):
+        assert torch.isfinite(y).all(), spec.name
+        y_ref, mag = oracle.gemv(wb, xbits[d.cols])
+        got = y[:, torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
+        err = float((np.abs(got - y_ref) / np.where(mag > 0, mag, 1.0)).max())
+        assert err <= GEMV_TOL, (spec.name, batch, err)
+        worst = max(worst, err)
+    return worst
 
 
 def test_smollm_whole_model_decode_to_bf16(entro):
-    """SmolLM-1.7B shapes, mixed unsigned/asymmetric 8-bit: one grouped launch decodes all 169 tensors."""
+    """SmolLM-1.7B shapes, mixed unsigned/asymmetric 8-bit: one grouped launch decodes all
+    169 tensors to bf16; every tensor bit-exact."""
     W = workloads.get("smollm_1p7b_u8")
     dts, infos, _ = encode_workload(entro, W)
-    outs = [torch.empty((d.rows, d.cols), dtype=torch.bfloat16, device="cuda") for d in dts]
-    g = entro.Group(dts, entro.GROUP_BF16, outs=outs)
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    g.launch(status=st)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0
-    shifted = [i for i, s in enumerate(W.tensors) if s.shifted]
-    picks = sorted(set(sample_indices(len(W.tensors), 4) + shifted[:2]))
-    for i in picks:
-        spec = W.tensors[i]
-        q, s, z, scheme = _oracle_weights(W, spec)
-        assert infos[i]["scheme"] == scheme and infos[i]["scale"] == s and infos[i]["zero"] == z, spec.name
-        assert np.array_equal(_bits(outs[i]), oracle.dequant_bf16(q, s, z)), spec.name
+    _decode_and_check(entro, W, dts, infos, codes=False, bf16_group=True)
 
 
-def test_mistral_decode_step_gemv(entro):
-    """Mistral-7B shapes, asymmetric 4-bit, row-aligned chunks: the 224 GEMVs of one decode step in one launch."""
+def test_mistral_every_tensor_and_decode_step(entro):
+    """Mistral-7B shapes, asymmetric 4-bit: codes and bf16 of all 224 tensors bit-exact, and the
+    decode step's fused GEMV (one launch over every tensor) at batch 1, 4 and 16."""
     W = workloads.get("mistral_7b_u4")
     dts, infos, _ = encode_workload(entro, W)
-    xs = [workloads.activations(W.seed, 1, d.cols).cuda() for d in dts]
-    ys = [torch.full((1, d.rows), float("nan"), device="cuda") for d in dts]
-    g = entro.Group(dts, entro.GROUP_GEMV, xs=xs, ys=ys, batch=1)
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    g.launch(status=st)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0
-    assert all(torch.isfinite(y).all() for y in ys)
-    for i in sample_indices(len(W.tensors), 5):
-        spec = W.tensors[i]
-        q, s, z, _ = _oracle_weights(W, spec)
-        wb = oracle.dequant_bf16(q, s, z).reshape(spec.rows, spec.cols)
-        y_ref, mag = oracle.gemv(wb, workloads.bf16_bits(xs[i].cpu()))
-        err = np.abs(ys[i].cpu().numpy().astype(np.float64) - y_ref) / np.where(mag > 0, mag, 1.0)
-        assert float(err.max()) <= GEMV_TOL, (spec.name, float(err.max()))
+    samples = _decode_and_check(entro, W, dts, infos)
+    for batch in (1, 4, 16):
+        _gemv_check(entro, W, dts, samples, batch)
 
 
-@pytest.mark.parametrize("batch", [1, 4, 16])
-def test_phi3_gemv_batches(entro, batch):
-    """Phi-3-mini shapes, mixed 8-bit, fused GEMV at batch 1, 4 and 16 over the first 8 layers."""
+def test_phi3_every_tensor_and_gemv_batches(entro):
+    """Phi-3-mini shapes, mixed 8-bit: codes and bf16 of all 128 tensors bit-exact, and the fused
+    GEMV over every tensor at batch 1, 4 and 16."""
     W = workloads.get("phi3_mini_u8")
-    dts, infos, _ = encode_workload(entro, W, limit=32)
-    xs = [workloads.activations(W.seed + batch, batch, d.cols).cuda() for d in dts]
-    ys = [torch.full((batch, d.rows), float("nan"), device="cuda") for d in dts]
-    g = entro.Group(dts, entro.GROUP_GEMV, xs=xs, ys=ys, batch=batch)
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    g.launch(status=st)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0
-    for i in sample_indices(len(dts), 4):
-        spec = W.tensors[i]
-        q, s, z, _ = _oracle_weights(W, spec)
-        wb = oracle.dequant_bf16(q, s, z).reshape(spec.rows, spec.cols)
-        rows = slice(0, min(spec.rows, 512))
-        y_ref, mag = oracle.gemv(wb[rows], workloads.bf16_bits(xs[i].cpu()))
-        got = ys[i][:, rows].cpu().numpy().astype(np.float64)
-        err = np.abs(got - y_ref) / np.where(mag > 0, mag, 1.0)
-        assert float(err.max()) <= GEMV_TOL, (spec.name, batch, float(err.max()))
+    dts, infos, _ = encode_workload(entro, W)
+    samples = _decode_and_check(entro, W, dts, infos)
+    for batch in (1, 4, 16):
+        _gemv_check(entro, W, dts, samples, batch)
 
 
 def test_stress_tensors(entro):
-    """8192x8192 near-uniform codes (entropy ~7.99 bits) and p(mode)=0.9 skew (the 16-bit limit binds)."""
+    """8192x8192 near-uniform codes (entropy ~7.99 bits) and p(mode)=0.9 skew (the 16-bit limit
+    binds): codes and bf16 bit-exact, GEMV on sampled rows."""
     W = workloads.get("stress_8192_u8")
     dts, infos, _ = encode_workload(entro, W)
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
     for i, spec in enumerate(W.tensors):
-        q, s, z, _ = _oracle_weights(W, spec)
+        q, s, z, _ = oracle.quantize(workloads.weights(W, spec, device="cuda").cpu().numpy(), W.bits, W.quant_mode)
         hist = np.bincount(q, minlength=256)
         if spec.law == "skew":
             assert abs(hist.max() / hist.sum() - 0.9) < 5e-4            # p(mode) = 0.9 by construction
@@ -114,16 +156,5 @@ def test_stress_tensors(entro):
         else:
             p = hist[hist > 0] / hist.sum()
             assert float(-(p * np.log2(p)).sum()) > 7.9
-        out = dts[i].decode_dequant_bf16(status=st)
-        codes = dts[i].decode_codes(status=st)
-        x = workloads.activations(7, 1, spec.cols).cuda()
-        y = dts[i].decode_gemv(x, status=st)
-        torch.cuda.synchronize()
-        assert int(st.item()) == 0
-        wb = oracle.dequant_bf16(q, s, z)
-        assert np.array_equal(_bits(out), wb)
-        assert np.array_equal(codes.cpu().numpy()[: q.size], q)
-        rows = slice(0, 256)
-        y_ref, mag = oracle.gemv(wb.reshape(spec.rows, spec.cols)[rows], workloads.bf16_bits(x.cpu()))
-        err = np.abs(y[:, rows].cpu().numpy().astype(np.float64) - y_ref) / np.where(mag > 0, mag, 1.0)
-        assert float(err.max()) <= GEMV_TOL
+    samples = _decode_and_check(entro, W, dts, infos)
+    _gemv_check(entro, W, dts, samples, 1)

@@ -57,6 +57,11 @@ CASES = [
     ("laplace", 4, oracle.MODE_ASYM, 12, 2, -1024, 7, 333),     # 64 lanes (negative chunk marks them)
     ("t4", 8, oracle.MODE_AUTO, 16, 2, -6144, 20, 3072),
     ("skew", 8, oracle.MODE_ASYM, 16, 2, -14336, 3, 14336),
+    ("laplace", 4, oracle.MODE_ASYM, 12, 3, 8192, 100, 1000),     # row tiles, ragged both ways
+    ("t4", 8, oracle.MODE_AUTO, 16, 3, 4096, 70, 3072),
+    ("skew", 8, oracle.MODE_ASYM, 16, 3, 512, 33, 24),
+    ("laplace", 4, oracle.MODE_ASYM, 12, 3, -1024, 130, 520),    # 64-row tiles
+    ("t4", 8, oracle.MODE_ASYM, 16, 3, 256, 0, 16),
 ]
 
 
@@ -126,10 +131,17 @@ def test_encoder_errors_match_oracle():
     assert e.value.code == entro.E_LIMIT
     with pytest.raises(oracle.OracleError):
         oracle.encode(many, 8, oracle.MODE_ASYM, 7, 2, 256)
-    for kw in ({"bits": 5}, {"fmt": 3}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25},
-               {"lanes": 48}, {"lanes": 64, "chunk_symbols": 768}):
+    for kw in ({"bits": 5}, {"fmt": 4}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25},
+               {"lanes": 48}, {"lanes": 64, "chunk_symbols": 768}, {"fmt": 3, "chunk_symbols": 300}):
         with pytest.raises(entro.EntroError):
             entro.Blob.encode(many, **kw)
+    # row tiles need whole runs of 8 columns
+    odd = workloads.small_tensor("t4", 8, 12, seed=3)
+    with pytest.raises(entro.EntroError) as e:
+        entro.Blob.encode(odd, bits=8, fmt=entro.FORMAT_ROWS, chunk_symbols=256)
+    assert e.value.code == entro.E_INVAL
+    with pytest.raises(oracle.OracleError):
+        oracle.encode(odd, 8, oracle.MODE_ASYM, 16, oracle.FMT_ROWS, 256)
 
 
 def test_blob_bytes_roundtrip_and_validation():

@@ -52,5 +52,5 @@ def test_reference_arm_under_torchrun_two_ranks():
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1, r.stdout
     d = json.loads(lines[0])
-    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "Gsym/s" and d["value"] > 0
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"].startswith("tok/s") and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"

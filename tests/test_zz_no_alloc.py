@@ -52,3 +52,40 @@ def test_static_group_gemv_matches_group_launch():
         entro.decode_gemv_group_static(too_many, [xs[0]] * len(too_many), [ys_new[0]] * len(too_many),
                                        batch=batch)
     assert e.value.code == entro.E_LIMIT
+
+
+@pytest.mark.parametrize("fmt", ["lanes", "rows"])
+def test_static_group_gemv_many_tensors_against_oracle(fmt):
+    """70 small tensors: the fixed table is filled in three host-to-device copies of up to
+    32 entries, so the later copies' offsets and running chunk and symbol counts are used.
+    Checked against the oracle's fp64 product and against the grouped launch, twice."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import oracle
+    import huffman_decode_canonical_b200 as entro
+
+    f = entro.FORMAT_ROWS if fmt == "rows" else entro.FORMAT_LANES
+    batch = 2
+    dts, xs, refs = [], [], []
+    for i in range(70):
+        r, c = 8 + 8 * (i % 5), 256 * (1 + i % 3)
+        w = workloads.small_tensor("laplace", r, c, seed=200 + i)
+        q, s, z, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
+        dt = entro.upload(entro.Blob.encode(w, bits=4, quant_mode=entro.QUANT_ASYM, fmt=f,
+                                            chunk_symbols=8192 if fmt == "rows" else max(1, 8192 // c) * c))
+        x = workloads.activations(300 + i, batch, c)
+        refs.append(oracle.gemv(oracle.dequant_bf16(q, s, z).reshape(r, c), workloads.bf16_bits(x)))
+        dts.append(dt)
+        xs.append(x.cuda())
+    ys_group = [torch.empty((batch, d.rows), dtype=torch.float32, device="cuda") for d in dts]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    entro.Group(dts, entro.GROUP_GEMV, xs=xs, ys=ys_group, batch=batch).launch(status=st)
+    for call in range(2):
+        ys = [torch.full((batch, d.rows), float("nan"), dtype=torch.float32, device="cuda") for d in dts]
+        entro.decode_gemv_group_static(dts, xs, ys, batch=batch, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        for y, yg, (y_ref, mag) in zip(ys, ys_group, refs):
+            err = np.abs(y.cpu().numpy().astype(np.float64) - y_ref) / np.where(mag > 0, mag, 1.0)
+            assert np.isfinite(err).all() and float(err.max()) <= GEMV_TOL, (call, float(err.max()))
+            assert torch.equal(y, yg)                 # the same kernel on the same table contents

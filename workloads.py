@@ -40,6 +40,7 @@ QUANT_ASYM = 2
 
 FORMAT_SINGLE = 1      # one bitstream per chunk
 FORMAT_LANES = 2       # 32 word-interleaved lane bitstreams per chunk
+FORMAT_ROWS = 3        # row tiles: lane l of a chunk is row l of a 32- or 64-row tile
 
 
 @dataclasses.dataclass(frozen=True)
