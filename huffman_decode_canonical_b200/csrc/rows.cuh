@@ -481,6 +481,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
         long long head_g = -1, tail_g = -1;  // row groups of this warp's partial sums (hacc, acc)
         bool began = false;               // the current row group began in this warp
         long long k = 0;
+        // GEMV: the warp's tiles are consecutive, so their (row group, column tile) advance by one
+        long long ggrp = OUT == OUT_GEMV ? wa / sh.T : 0, gj = OUT == OUT_GEMV ? wa % sh.T : 0;
         for (long long c = chunk_of(0); c >= 0 && !dead; c = chunk_of(++k)) {
             const int b = static_cast<int>(k & 1);
             const uint32_t phase = b ? phase1 : phase0;
@@ -491,7 +493,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
             }
             if (b) { phase1++; pend1 = false; }
             else { phase0++; pend0 = false; }
-            const long long grp = c / sh.T, j = c % sh.T;
+            long long grp, j;
+            if (OUT == OUT_GEMV) {
+                grp = ggrp;
+                j = gj;
+                if (++gj == sh.T) {
+                    gj = 0;
+                    ggrp++;
+                }
+            } else {
+                grp = c / sh.T;
+                j = c - grp * sh.T;
+            }
             const long long row0 = grp * LANES, col0 = j * sh.Kc;
             const int nrows = static_cast<int>(min(static_cast<long long>(LANES), d.rows - row0));
             const int runs = static_cast<int>(min(sh.Kc, sh.K - col0) / kRun);
@@ -504,9 +517,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
 #pragma unroll
                         for (int i = 0; i < 4; i++) acc[m][nb][i] = 0.f;
             }
-            if (chunk_words_ok(d, c, a.stage_rows, LANES)) {
+            const uint64_t wst = d.index[2 * c], wnx = d.index[2 * c + 2];
+            if (wnx >= wst && wnx <= static_cast<uint64_t>(d.payload_words) && (wnx - wst) % LANES == 0 &&
+                (wnx - wst) / LANES + kSlackRows <= static_cast<uint64_t>(a.stage_rows)) {
                 const uint32_t *buf = stage + b * buf_words;
-                const int words = static_cast<int>((d.index[2 * c + 2] - d.index[2 * c]) / LANES);
+                const int words = static_cast<int>((wnx - wst) / LANES);
                 WideDecoder<BITS, SLOW, LANES> ld[LPT];
                 uint32_t read_limit[LPT];
 #pragma unroll
@@ -516,6 +531,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                                l < nrows);
                     read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
                 }
+                // GEMV: this thread's row of x (batch row 8 nb + gid) at the tile's first column
+                const __nv_bfloat16 *xrow[NB];
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++)
+                    xrow[nb] = OUT == OUT_GEMV ? g.x + min(8 * nb + gid, a.batch - 1) * sh.K + col0 : nullptr;
                 for (int tb = 0; tb < runs; tb += kRowsBlock) {
                     const int te = min(tb + kRowsBlock, runs);
                     wide_decode_to<kStepsPerCheck>(ld, slim, soffs, ssyms, te, runs, d.max_len, refill_each,
@@ -525,16 +545,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                     if (OUT == OUT_GEMV) {
                         // groups of 4 runs = 32 columns: thread (gid, tig) supplies run t0 + tig of
                         // rows gid and gid + 8 of each 16-row tile (A) and of batch row 8 nb + gid (B)
-                        const __nv_bfloat16 *xb = g.x + col0;
                         for (int t0 = tb; t0 < te; t0 += 4) {
                             const int t = t0 + tig;
                             uint4 xv[NB];
 #pragma unroll
-                            for (int nb = 0; nb < NB; nb++) {
-                                const int br = 8 * nb + gid;
-                                xv[nb] = (t < te && br < a.batch) ? ldg_nc_v4(xb + br * sh.K + kRun * t)
-                                                                  : make_uint4(0u, 0u, 0u, 0u);
-                            }
+                            for (int nb = 0; nb < NB; nb++)
+                                xv[nb] = (t < te && 8 * nb + gid < a.batch) ? ldg_nc_v4(xrow[nb] + kRun * t)
+                                                                            : make_uint4(0u, 0u, 0u, 0u);
                             const uint32_t sl = runbuf + static_cast<uint32_t>(t) * RB + gid * LB;
 #pragma unroll
                             for (int m = 0; m < kMT; m++) {

@@ -140,10 +140,10 @@ WORKLOADS = {
         "SmolLM-1.7B-shaped (24 layers + 49152x2048 embedding), t(4) with per-tensor std "
         "U(0.01, 0.04), 10% shifted non-negative, mixed unsigned/asymmetric 8-bit"),
     "mistral_7b_u4": Workload(
-        "mistral_7b_u4", 3, 4, QUANT_ASYM, 12, FORMAT_LANES, "rows",
+        "mistral_7b_u4", 3, 4, QUANT_ASYM, 12, FORMAT_ROWS, "fixed:8192",
         _mistral_7b(),
         "Mistral-7B-shaped (32 layers), Laplace with std 0.02, asymmetric 4-bit, "
-        "row-aligned chunks, 64 lanes per chunk, fused GEMV at batch 1", 64),
+        "row tiles of 32 rows x 256 columns, fused GEMV at batch 1", 32),
     "phi3_mini_u8": Workload(
         "phi3_mini_u8", 4, 8, QUANT_AUTO, 16, FORMAT_LANES, "rows",
         _phi3_mini(4),
