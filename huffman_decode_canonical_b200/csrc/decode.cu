@@ -100,6 +100,7 @@ struct LaunchArgs {
     long long total_syms;
     int32_t *status;
     uint32_t tx_extra;    // bytes added to the table barrier that never arrive (bounded-wait test; 0)
+    uint32_t k_one;       // 1, a value the compiler cannot see (moves integer work to the FMA pipe)
 };
 
 struct TensorHandle {
@@ -2199,6 +2200,7 @@ static int launch_rows(const TensorHandle *const *ts, int count, int out_kind, i
     a.total_syms = total;
     a.status = status;
     a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
+    a.k_one = 1;
     const cudaError_t e = launch(fn, (unsigned)grid, warps * 32, rl.total, st, a, per_sm <= 2);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "row-tile kernel launch");
 }

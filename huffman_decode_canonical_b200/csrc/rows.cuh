@@ -92,6 +92,29 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     return v;
 }
 
+// Integer constants the compiler cannot see (kernel arguments: 1 and powers of
+// two).  A shift or an addition written as a multiply-add with one of them
+// runs on the FMA pipe (IMAD) instead of the ALU pipe, which the lookups would
+// otherwise saturate: the decode and its emission split their integer work
+// over both pipes.
+struct Pipes {
+    uint32_t one, four, eight, two8, two12, two24;
+};
+
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {  // a * b + c
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t imulhi(uint32_t a, uint32_t b) {  // (a * b) >> 32
+    uint32_t d;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t byte_of(uint32_t v, uint32_t sel) {  // byte sel of v, zero-extended
+    return __byte_perm(v, 0u, 0x4440u | sel);
+}
+
 template <int BITS, bool SLOW, int LANES>
 struct WideDecoder {
     static constexpr uint32_t kRowBytes = 4 * LANES;                      // one staged word of every lane
@@ -102,7 +125,7 @@ struct WideDecoder {
     uint32_t hi, lo;      // 64-bit window, MSB first
     uint32_t wnext;       // next word, loaded one refill ahead
     uint32_t C;           // consumed window bits | pending bits << 8 | runs << 16
-    uint32_t p0, p1, p2;  // pending codes as one bit string, first code at bit 0 of p0
+    uint32_t p0, p1;      // pending codes as one bit string, first code at bit 0 of p0 (p1: 8-bit only)
     uint32_t osta;        // shared address of the current run's slot
 
     // b: shared address of this lane's word 0 (word j at b + kRowBytes j);
@@ -115,7 +138,7 @@ struct WideDecoder {
         bufa = b + 2 * kRowBytes;
         wnext = lds32(min(bufa, bufcap));
         C = active ? 0u : 0xFFFF0000u;  // an empty lane counts as done
-        p0 = p1 = p2 = 0;
+        p0 = p1 = 0;
         osta = slot0;
     }
 
@@ -123,7 +146,7 @@ struct WideDecoder {
 
     // When 32 or more window bits are consumed (the valid bits then all sit in
     // hi and lo is zero), the next word lands right below them.
-    __device__ __forceinline__ void refill() {
+    __device__ __forceinline__ void refill(const Pipes &k) {
         asm volatile(
             "{\n\t"
             ".reg .pred p;\n\t"
@@ -131,37 +154,41 @@ struct WideDecoder {
             "and.b32 x, %2, 32;\n\t"
             "setp.ne.u32 p, x, 0;\n\t"
             "@p shf.l.wrap.b32 x, %3, 0, %2;\n\t"  // wnext >> (32 - s), s = consumed - 32
-            "@p or.b32 %0, %0, x;\n\t"
+            "@p mad.lo.u32 %0, x, %6, %0;\n\t"     // hi |= x (x lands on hi's zero bits)
             "@p shf.l.wrap.b32 %1, 0, %3, %2;\n\t"  // wnext << s
-            "@p sub.u32 %2, %2, 32;\n\t"
-            "@p add.u32 %4, %4, %6;\n\t"
+            "@p mad.lo.u32 %2, %6, %7, %2;\n\t"    // consumed - 32
+            "@p mad.lo.u32 %4, %6, %8, %4;\n\t"    // next word
             "@p min.u32 a, %4, %5;\n\t"
             "@p ld.shared.u32 %3, [a];\n\t"
             "}"
             : "+r"(hi), "+r"(lo), "+r"(C), "+r"(wnext), "+r"(bufa)
-            : "r"(bufcap), "n"(kRowBytes)
+            : "r"(bufcap), "r"(k.one), "r"(0xFFFFFFE0u), "r"(kRowBytes)
             : "memory");
+    }
+
+    __device__ __forceinline__ uint2 entry(const Pipes &k) const {
+        return lds64(imad(imulhi(hi, k.two12), k.eight, tab));  // table[window >> 52]
     }
 
     // One table lookup: the entry of the window's top 12 bits, or, for a code
     // longer than 12 bits, the canonical slow path's single code.
-    __device__ __forceinline__ void step(const uint32_t *slim, const int32_t *soffs, const uint8_t *ssyms,
-                                         int max_len, int32_t *status) {
-        uint2 e = lds64(tab + ((hi >> (32 - kMaxLutBits)) << 3));
+    __device__ __forceinline__ void step(const Pipes &k, const uint32_t *slim, const int32_t *soffs,
+                                         const uint8_t *ssyms, int max_len, int32_t *status) {
+        uint2 e = entry(k);
         if (SLOW && (e.y & 31u) == 0) {
             const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
             const uint32_t se = slow_entry(win, max_len, slim, soffs, ssyms, status);
             e.x = (se >> 8) & 0xFFu;
             e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
         }
-        advance(e.x, e.y);
+        advance(k, e.x, e.y);
     }
 
     // The same lookup, made a no-op (no bits consumed, no codes appended) for a
     // lane that is done: lets the streams of a thread run in one basic block.
-    __device__ __forceinline__ void step_if(bool live, const uint32_t *slim, const int32_t *soffs,
+    __device__ __forceinline__ void step_if(bool live, const Pipes &k, const uint32_t *slim, const int32_t *soffs,
                                             const uint8_t *ssyms, int max_len, int32_t *status) {
-        uint2 e = lds64(tab + ((hi >> (32 - kMaxLutBits)) << 3));
+        uint2 e = entry(k);
         e.x = live ? e.x : 0u;
         e.y = live ? e.y : 0u;
         if (SLOW && live && (e.y & 31u) == 0) {
@@ -170,67 +197,65 @@ struct WideDecoder {
             e.x = (se >> 8) & 0xFFu;
             e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
         }
-        advance(e.x, e.y);
+        advance(k, e.x, e.y);
     }
 
     // Consume meta's bits, append the codes to the pending string, store the
     // current run's slot, and move to the next slot when a run is whole.
-    __device__ __forceinline__ void advance(uint32_t codes, uint32_t meta) {
+    // Appends land on zero bits of the string, so they are additions.
+    __device__ __forceinline__ void advance(const Pipes &k, uint32_t codes, uint32_t meta) {
         if (BITS == 4) {
-            // pending bits < 32 before the append
+            // pending bits < 32 before the append; what passes bit 32 (phi) starts the next run
             asm volatile(
                 "{\n\t"
                 ".reg .u32 q, plo, phi, x;\n\t"
                 ".reg .pred dn;\n\t"
-                "shf.l.wrap.b32 %0, %1, %0, %8;\n\t"
-                "shf.l.wrap.b32 %1, 0, %1, %8;\n\t"
-                "shr.u32 q, %2, 8;\n\t"
-                "shf.l.wrap.b32 plo, 0, %7, q;\n\t"
-                "shf.l.wrap.b32 phi, %7, 0, q;\n\t"
-                "or.b32 %3, %3, plo;\n\t"
-                "or.b32 %4, %4, phi;\n\t"
-                "add.u32 %2, %2, %8;\n\t"
-                "st.shared.u32 [%5], %3;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %7;\n\t"
+                "shf.l.wrap.b32 %1, 0, %1, %7;\n\t"
+                "mul.hi.u32 q, %2, %9;\n\t"           // pending bits (C >> 8; the shifts use q mod 32)
+                "shf.l.wrap.b32 plo, 0, %6, q;\n\t"
+                "shf.l.wrap.b32 phi, %6, 0, q;\n\t"
+                "mad.lo.u32 %3, plo, %8, %3;\n\t"
+                "mad.lo.u32 %2, %7, %8, %2;\n\t"      // C += meta
+                "st.shared.u32 [%4], %3;\n\t"
                 "and.b32 x, %2, 0x2000;\n\t"
                 "setp.ne.u32 dn, x, 0;\n\t"
-                "selp.b32 %3, %4, %3, dn;\n\t"
-                "selp.b32 %4, 0, %4, dn;\n\t"
-                "@dn add.u32 %2, %2, 0xE000;\n\t"  // runs + 1, pending - 32
-                "@dn add.u32 %5, %5, %6;\n\t"
+                "selp.b32 %3, phi, %3, dn;\n\t"
+                "@dn mad.lo.u32 %2, %8, %10, %2;\n\t"  // runs + 1, pending - 32
+                "@dn mad.lo.u32 %4, %8, %5, %4;\n\t"
                 "}"
-                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(p1), "+r"(osta)
-                : "n"(kRunBytes), "r"(codes), "r"(meta)
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xE000u)
                 : "memory");
         } else {
-            // pending bits < 64 before the append: codes go to p0:p1 below bit
-            // 32 of the string, to p1:p2 above
+            // pending bits < 64 before the append: below bit 32 of the string the codes
+            // go to p0 and what passes bit 32 to p1 (then zero); above, to p1 and past bit 64
+            // (phi) to the next run
             asm volatile(
                 "{\n\t"
                 ".reg .u32 q, plo, phi, x;\n\t"
                 ".reg .pred hs, dn;\n\t"
-                "shf.l.wrap.b32 %0, %1, %0, %9;\n\t"
-                "shf.l.wrap.b32 %1, 0, %1, %9;\n\t"
-                "shr.u32 q, %2, 8;\n\t"
-                "shf.l.wrap.b32 plo, 0, %8, q;\n\t"
-                "shf.l.wrap.b32 phi, %8, 0, q;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %8;\n\t"
+                "shf.l.wrap.b32 %1, 0, %1, %8;\n\t"
+                "mul.hi.u32 q, %2, %10;\n\t"
+                "shf.l.wrap.b32 plo, 0, %7, q;\n\t"
+                "shf.l.wrap.b32 phi, %7, 0, q;\n\t"
                 "and.b32 x, %2, 0x2000;\n\t"
                 "setp.ne.u32 hs, x, 0;\n\t"
-                "@!hs or.b32 %3, %3, plo;\n\t"
-                "@!hs or.b32 %4, %4, phi;\n\t"
-                "@hs or.b32 %4, %4, plo;\n\t"
-                "@hs or.b32 %5, %5, phi;\n\t"
-                "add.u32 %2, %2, %9;\n\t"
-                "st.shared.v2.u32 [%6], {%3, %4};\n\t"
+                "selp.b32 %4, %4, phi, hs;\n\t"
+                "@!hs mad.lo.u32 %3, plo, %9, %3;\n\t"
+                "@hs mad.lo.u32 %4, plo, %9, %4;\n\t"
+                "mad.lo.u32 %2, %8, %9, %2;\n\t"
+                "st.shared.v2.u32 [%5], {%3, %4};\n\t"
                 "and.b32 x, %2, 0x4000;\n\t"
                 "setp.ne.u32 dn, x, 0;\n\t"
-                "selp.b32 %3, %5, %3, dn;\n\t"
+                "selp.b32 %3, phi, %3, dn;\n\t"
                 "selp.b32 %4, 0, %4, dn;\n\t"
-                "selp.b32 %5, 0, %5, dn;\n\t"
-                "@dn add.u32 %2, %2, 0xC000;\n\t"  // runs + 1, pending - 64
-                "@dn add.u32 %6, %6, %7;\n\t"
+                "@dn mad.lo.u32 %2, %9, %11, %2;\n\t"  // runs + 1, pending - 64
+                "@dn mad.lo.u32 %5, %9, %6, %5;\n\t"
                 "}"
-                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(p1), "+r"(p2), "+r"(osta)
-                : "n"(kRunBytes), "r"(codes), "r"(meta)
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(p1), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xC000u)
                 : "memory");
         }
     }
@@ -240,7 +265,8 @@ struct WideDecoder {
 // check, until every lane of the warp has reached te; a lane that is ahead
 // keeps decoding up to run cap (the chunk's end).
 template <int STEPS, int BITS, bool SLOW, int LANES, int LPT>
-__device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES> (&ld)[LPT], const uint32_t *slim,
+__device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES> (&ld)[LPT], const Pipes &pk,
+                                               const uint32_t *slim,
                                                const int32_t *soffs, const uint8_t *ssyms, int te, int cap,
                                                int max_len, bool refill_each, int32_t *status) {
     const uint32_t te_c = static_cast<uint32_t>(te) << kRunsShift, cap_c = static_cast<uint32_t>(cap) << kRunsShift;
@@ -253,10 +279,10 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES> (&
             if (ld[0].C < cap_c) {
 #pragma unroll
                 for (int h = 0; h < STEPS / 2; h++) {
-                    ld[0].refill();
-                    ld[0].step(slim, soffs, ssyms, max_len, status);
-                    if (SLOW && refill_each) ld[0].refill();
-                    ld[0].step(slim, soffs, ssyms, max_len, status);
+                    ld[0].refill(pk);
+                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
+                    if (SLOW && refill_each) ld[0].refill(pk);
+                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
                 }
             }
         } else {
@@ -267,14 +293,14 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES> (&
 #pragma unroll
             for (int h = 0; h < STEPS / 2; h++) {
 #pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].refill();
+                for (int k = 0; k < LPT; k++) ld[k].refill(pk);
 #pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], slim, soffs, ssyms, max_len, status);
+                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
                 if (SLOW && refill_each)
 #pragma unroll
-                    for (int k = 0; k < LPT; k++) ld[k].refill();
+                    for (int k = 0; k < LPT; k++) ld[k].refill(pk);
 #pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], slim, soffs, ssyms, max_len, status);
+                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
             }
         }
     }
@@ -282,20 +308,21 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES> (&
 
 // 8 codes of a run slot -> 8 bf16 values (4 words, value of code i in half i)
 template <int BITS>
-__device__ __forceinline__ uint4 slot_values(uint32_t slot, uint32_t vtab, uint32_t vpair) {
+__device__ __forceinline__ uint4 slot_values(uint32_t slot, uint32_t vtab, uint32_t vpair, const Pipes &k) {
     uint4 v;
     if (BITS == 4) {
         const uint32_t c = lds32(slot);
-        v.x = lds32(vpair + ((c & 0xFFu) << 2));
-        v.y = lds32(vpair + (((c >> 8) & 0xFFu) << 2));
-        v.z = lds32(vpair + (((c >> 16) & 0xFFu) << 2));
-        v.w = lds32(vpair + ((c >> 24) << 2));
+        v.x = lds32(imad(byte_of(c, 0), k.four, vpair));
+        v.y = lds32(imad(byte_of(c, 1), k.four, vpair));
+        v.z = lds32(imad(byte_of(c, 2), k.four, vpair));
+        v.w = lds32(imad(imulhi(c, k.two8), k.four, vpair));
     } else {
         const uint2 c = lds64(slot);
-        v.x = __byte_perm(lds32(vtab + ((c.x & 0xFFu) << 2)), lds32(vtab + (((c.x >> 8) & 0xFFu) << 2)), 0x5410);
-        v.y = __byte_perm(lds32(vtab + (((c.x >> 16) & 0xFFu) << 2)), lds32(vtab + ((c.x >> 24) << 2)), 0x5410);
-        v.z = __byte_perm(lds32(vtab + ((c.y & 0xFFu) << 2)), lds32(vtab + (((c.y >> 8) & 0xFFu) << 2)), 0x5410);
-        v.w = __byte_perm(lds32(vtab + (((c.y >> 16) & 0xFFu) << 2)), lds32(vtab + ((c.y >> 24) << 2)), 0x5410);
+        auto val = [&](uint32_t b) { return lds32(imad(b, k.four, vtab)); };
+        v.x = __byte_perm(val(byte_of(c.x, 0)), val(byte_of(c.x, 1)), 0x5410);
+        v.y = __byte_perm(val(byte_of(c.x, 2)), val(imulhi(c.x, k.two8)), 0x5410);
+        v.z = __byte_perm(val(byte_of(c.y, 0)), val(byte_of(c.y, 1)), 0x5410);
+        v.w = __byte_perm(val(byte_of(c.y, 2)), val(imulhi(c.y, k.two8)), 0x5410);
     }
     return v;
 }
@@ -377,6 +404,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
     constexpr int kStepsPerCheck = 6;
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
+    const Pipes pk{a.k_one, a.k_one << 2, a.k_one << 3, a.k_one << 8, a.k_one << 12, a.k_one << 24};
     const RowsLayout L = rows_layout(warps, a.stage_rows * LANES, a.out_words * 4);
     uint64_t *tbar = reinterpret_cast<uint64_t *>(smem_raw + L.tbar);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem_raw + L.bars) + 2 * warp;
@@ -538,7 +566,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                     xrow[nb] = OUT == OUT_GEMV ? g.x + min(8 * nb + gid, a.batch - 1) * sh.K + col0 : nullptr;
                 for (int tb = 0; tb < runs; tb += kRowsBlock) {
                     const int te = min(tb + kRowsBlock, runs);
-                    wide_decode_to<kStepsPerCheck>(ld, slim, soffs, ssyms, te, runs, d.max_len, refill_each,
+                    wide_decode_to<kStepsPerCheck>(ld, pk, slim, soffs, ssyms, te, runs, d.max_len, refill_each,
                                                    a.status);
                     __syncwarp();
                     constexpr uint32_t RB = rows_run_bytes(BITS, LANES), LB = rows_lane_bytes(BITS);
@@ -555,8 +583,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                             const uint32_t sl = runbuf + static_cast<uint32_t>(t) * RB + gid * LB;
 #pragma unroll
                             for (int m = 0; m < kMT; m++) {
-                                const uint4 wlo = slot_values<BITS>(sl + 16 * m * LB, vtab, vpair);
-                                const uint4 whi = slot_values<BITS>(sl + (16 * m + 8) * LB, vtab, vpair);
+                                const uint4 wlo = slot_values<BITS>(sl + 16 * m * LB, vtab, vpair, pk);
+                                const uint4 whi = slot_values<BITS>(sl + (16 * m + 8) * LB, vtab, vpair, pk);
 #pragma unroll
                                 for (int nb = 0; nb < NB; nb++) {
                                     mma_16816_bf16(acc[m][nb], wlo.x, whi.x, wlo.y, whi.y, xv[nb].x, xv[nb].y);
@@ -574,7 +602,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                                 const uint32_t sl = runbuf + static_cast<uint32_t>(t) * RB + l * LB;
                                 const long long pos = (row0 + l) * sh.K + col0 + kRun * t;  // first code's index
                                 if (OUT == OUT_BF16) {
-                                    const uint4 v = slot_values<BITS>(sl, vtab, vpair);
+                                    const uint4 v = slot_values<BITS>(sl, vtab, vpair, pk);
                                     *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(g.out) + pos) = v;
                                 } else if (BITS == 4) {
                                     reinterpret_cast<uint32_t *>(g.out)[pos >> 3] = lds32(sl);
