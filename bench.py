@@ -629,7 +629,7 @@ def run_model(args, dist, rank, world, local_rank):
     achieved = alg / (ms * 1e-3) / 1e9
     partial = " (first %d tensors)" % len(dts) if args.tensors else ""
     line = {"metric": METRIC,
-            "value": round(world / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
+            "value": round(world * args.batch / (ms * 1e-3), 2) if gemv else round(world * n / (ms * 1e-3) / 1e9, 2),
             "unit": (f"tok/s (batch {args.batch})" if gemv else "Gsym/s") + partial, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,

@@ -102,13 +102,16 @@ def test_encoder_identical_on_single_tensor_workloads(name):
     assert got == ref
 
 
-def test_encoder_identical_on_model_shaped_tensor():
-    """One Phi-3-mini-shaped tensor with row-aligned chunks (3072 columns -> 6144-symbol chunks)."""
-    W = workloads.get("phi3_mini_u8")
-    spec = W.tensors[1]          # o projection, 3072 x 3072
-    w = workloads.weights(W, spec).numpy()[:512]
+@pytest.mark.parametrize("name,index,rows", [("phi3_mini_u8", 1, 512), ("mistral_7b_u4", 6, 96)])
+def test_encoder_identical_on_model_shaped_tensor(name, index, rows):
+    """Model-shaped tensors in their workload's row-tile format: a Phi-3-mini-shaped o projection
+    (3072 columns, 32 x 128 tiles) and a Mistral-shaped down projection (14336 columns, 32 x 256
+    tiles, a ragged last row group)."""
+    W = workloads.get(name)
+    spec = W.tensors[index]
+    w = workloads.weights(W, spec).numpy()[:rows]
     C = W.chunk_symbols(spec.cols)
-    assert C == 6144
+    assert W.fmt == oracle.FMT_ROWS
     ref = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, C, lanes=W.lanes)
     got = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
                             chunk_symbols=C, lanes=W.lanes).to_bytes()

@@ -145,12 +145,12 @@ WORKLOADS = {
         "Mistral-7B-shaped (32 layers), Laplace with std 0.02, asymmetric 4-bit, "
         "row tiles of 32 rows x 256 columns, fused GEMV at batch 1", 32),
     "phi3_mini_u8": Workload(
-        "phi3_mini_u8", 4, 8, QUANT_AUTO, 16, FORMAT_LANES, "rows",
+        "phi3_mini_u8", 4, 8, QUANT_AUTO, 16, FORMAT_ROWS, "fixed:4096",
         _phi3_mini(4),
         "Phi-3-mini-shaped (32 layers), t(4) with per-tensor std U(0.01, 0.04), 10% shifted, "
-        "mixed unsigned/asymmetric 8-bit, row-aligned chunks, fused GEMV at batch 1/4/16"),
+        "mixed unsigned/asymmetric 8-bit, row tiles of 32 rows x 128 columns, fused GEMV at batch 1/4/16"),
     "stress_8192_u8": Workload(
-        "stress_8192_u8", 4, 8, QUANT_ASYM, 16, FORMAT_LANES, "rows",
+        "stress_8192_u8", 4, 8, QUANT_ASYM, 16, FORMAT_ROWS, "fixed:4096",
         (TensorSpec("near_uniform", 8192, 8192, "uniform", 1.0, False, 1000),
          TensorSpec("skew", 8192, 8192, "skew", 0.02, False, 1001)),
         "two 8192x8192 stress tensors: near-uniform codes and p(mode)=0.9 skew"),
