@@ -8,21 +8,24 @@
 //     64 lanes; a thread serves one or two lanes).  The chunk's words are
 //     staged into shared memory with cp.async.bulk (one elected lane,
 //     mbarrier completion, double buffered per warp, a copy per CTA).  Each
-//     lane keeps an MSB-first bit window in two 32-bit registers, peeks 12
-//     bits into a shared-memory multi-symbol table (up to six 4-bit or three
-//     8-bit codes per entry), and falls back to canonical length tables for
-//     codes longer than 12 bits.  Lane l emits runs of 8 adjacent weights, so
-//     a warp writes 128/256/512 contiguous bytes per run (uint4 codes / uint8
-//     codes / bf16) with one vector store per lane.
+//     lane decodes with the two-word-table decoder of wide_decoder.cuh (up to
+//     eight 4-bit or four 8-bit codes per 12-bit peek, canonical length tables
+//     for codes longer than 12 bits) into a 16-run ring.  Lane l emits runs of
+//     8 adjacent weights, so a warp writes 128/256/512 contiguous bytes per
+//     run (uint4 codes / uint8 codes / bf16) with one vector store per lane.
+//   * rows kernel (rows.cuh): the row-tile format, lane = row of a tile; codes,
+//     bf16 and the fused GEMV on the tensor cores at every batch size.
 //   * the same kernel dequantizes, w = bf16_rne(float(q - zero) * scale), with
 //     the value of every code computed once per CTA in fp32 and looked up in
 //     a shared-memory table (for 4-bit codes, by byte: two values per entry),
 //     or feeds the bf16 weights straight into an fp32 GEMV with a
 //     warp-shuffle reduction per row (weights never touch memory).
-//   * gemv_mma kernel: the fused GEMV for batches of 3 to 16 activation rows.
-//     The warps of a CTA decode consecutive rows in lockstep and multiply the
-//     decoded weights with warp-level tensor-core MMAs (mma.sync m16n8k16,
-//     bf16 in, fp32 out), reading the A operand from the warps' code rings.
+//   * gemv_mma kernel: the lanes format's fused GEMV for batches of 3 to 16
+//     activation rows.  The warps of a CTA decode consecutive rows in lockstep
+//     (one-word multi-symbol table, up to six 4-bit or three 8-bit codes per
+//     peek) and multiply the decoded weights with warp-level tensor-core MMAs
+//     (mma.sync m16n8k16, bf16 in, fp32 out), reading the A operand from the
+//     warps' code rings.
 //   * segment kernel: the one-bitstream-per-chunk format, one CTA per chunk
 //     of up to 16384 codes.  Its threads decode segments cut at 32-bit
 //     boundaries, re-decode from where the left neighbour stopped until they
@@ -51,6 +54,7 @@
 namespace entro {
 
 constexpr int kLutSize = 1 << kMaxLutBits;   // 4096 entries, 16 KB of shared memory
+constexpr int kWideLutBytes = kLutSize * 8;  // the two-word table: 4096 entries of {codes, meta}
 constexpr long long kWaitCycles = 1LL << 31;  // ~1 s at B200 clocks
 constexpr int kMaxWarps = 16;
 constexpr int kMaxBatch = 16;
@@ -230,10 +234,11 @@ struct SmemOffsets {
 // shared-memory carve-up; identical on host (sizing) and device
 // stage_words: 32-bit words of one staging buffer (rows x lanes); red_bytes:
 // the cross-warp partial sums of the tensor-core GEMV
+// lut_bytes: the decode table (kLutSize * 4, or * 8 for the two-word table)
 __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems, int stage_words, int out_words,
-                                                   size_t red_bytes = 0) {
+                                                   size_t red_bytes = 0, size_t lut_bytes = kLutSize * 4) {
     SmemOffsets o;
-    size_t p = kLutSize * 4 + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
+    size_t p = lut_bytes + 256 * 4 + 256 * 4 + 32 * 4 + 32 * 4 + 256;
     p = align_up(p, 16);
     o.x = p;
     p += (size_t)x_elems * 2;
@@ -254,11 +259,11 @@ __host__ __device__ inline SmemOffsets smem_layout(int warps, long long x_elems,
 }
 
 __device__ __forceinline__ Smem carve(uint8_t *base, int warps, long long x_elems, int stage_words, int out_words,
-                                      size_t red_bytes = 0) {
-    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words, red_bytes);
+                                      size_t red_bytes = 0, size_t lut_bytes = kLutSize * 4) {
+    const SmemOffsets o = smem_layout(warps, x_elems, stage_words, out_words, red_bytes, lut_bytes);
     Smem s;
     s.lut = reinterpret_cast<uint32_t *>(base);
-    s.vtab = s.lut + kLutSize;
+    s.vtab = s.lut + lut_bytes / 4;
     s.vpair = s.vtab + 256;
     s.slim = s.vpair + 256;
     s.soffs = reinterpret_cast<int32_t *>(s.slim + 32);
@@ -283,17 +288,20 @@ __device__ __forceinline__ uint32_t dequant_bf16_bits(int q, int zero, float sca
 // vpair[b] holds the values of both 4-bit codes of byte b.  The decode table,
 // the canonical tables and (GEMV) the activations arrive by bulk copies on the
 // CTA barrier; thread 0 issues them at phase `tphase`.
+// table: 0 = one code per entry (lut), 1 = several (mlut), 2 = the two-word table (wlut)
 template <int OUT, bool SLOW>
-__device__ void issue_tables(const GroupEntry &g, const Smem &s, bool multi, int batch, int x_in_smem,
+__device__ void issue_tables(const GroupEntry &g, const Smem &s, int table, int batch, int x_in_smem,
                              uint32_t tx_extra) {
     if (threadIdx.x != 0) return;
     const DevTensor &d = g.d;
-    uint32_t bytes = kLutSize * 4 + tx_extra;
+    const uint32_t tbytes = table == 2 ? kWideLutBytes : kLutSize * 4;
+    uint32_t bytes = tbytes + tx_extra;
     if (SLOW) bytes += kSlowBytes;
     const uint32_t xbytes = (OUT == OUT_GEMV && x_in_smem) ? static_cast<uint32_t>(d.cols * batch * 2) : 0u;
     bytes += xbytes;
     mbar_arrive_expect_tx(s.tbar, bytes);
-    bulk_copy_g2s(s.lut, multi ? d.mlut : d.lut, kLutSize * 4, s.tbar);
+    const void *src = table == 2 ? static_cast<const void *>(d.wlut) : table == 1 ? d.mlut : d.lut;
+    bulk_copy_g2s(s.lut, src, tbytes, s.tbar);
     if (SLOW) bulk_copy_g2s(s.slim, d.slow_limit, kSlowBytes, s.tbar);
 }
 
@@ -381,6 +389,8 @@ __device__ __forceinline__ uint32_t shr_clamp(uint32_t v, uint32_t n) {
     asm("shr.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(n));
     return r;
 }
+
+#include "wide_decoder.cuh"
 
 template <int BITS, bool SLOW, int LANES>
 struct LaneDecoder {
@@ -760,14 +770,29 @@ __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[L
     }
 }
 
+// The lanes kernel's decoder: the two-word table, run slots in the warp's
+// ring (run t of lane l in slot t mod kRing, word (t mod kRing) * LANES + l
+// for 4-bit codes, double-word for 8-bit).  Lanes that finish a block decode
+// up to kWideLookahead runs of the next; a block, the lookahead and the runs a
+// lane may complete past its last check fit the ring.
+template <int BITS>
+__host__ __device__ constexpr int wide_lookahead() {
+    return kRing - kEmitBlock - wide_runs_per_check(BITS, kLookupsPerCheck) < 3
+               ? kRing - kEmitBlock - wide_runs_per_check(BITS, kLookupsPerCheck)
+               : 3;
+}
+static_assert(wide_lookahead<4>() >= 1 && wide_lookahead<8>() >= 1, "ring too small for the wide decoder");
+template <int BITS, bool SLOW, int LANES>
+using RingDecoder = WideDecoder<BITS, SLOW, LANES, LANES * (BITS == 4 ? 4u : 8u), kRing>;
+
 // Decode chunk c of entry g from its staged words.  Thread `lane` decodes the
 // format lanes lane, lane + 32, ... as independent interleaved streams.  Whole
 // chunks are emitted every kEmitBlock runs, so the stores of one block drain
 // while the lanes decode the next.
 template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
-__device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const uint32_t *buf,
-                                             uint32_t *ost, int stage_rows, long long c, int batch, int x_in_smem,
-                                             int32_t *status) {
+__device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s, const Pipes &pk,
+                                             const uint32_t *buf, uint32_t *ost, int stage_rows, long long c,
+                                             int batch, int x_in_smem, int32_t *status) {
     constexpr int LPT = LANES / kLanes;
     constexpr int kStep = kRun * LANES;  // symbols per lane step
     const DevTensor &d = g.d;
@@ -779,12 +804,13 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
     const long long remain = d.n - first;
     const int nc = static_cast<int>(remain < d.chunk_symbols ? remain : d.chunk_symbols);
     const bool refill_each = SLOW && d.max_len > 16;
-    LaneDecoder<BITS, SLOW, LANES> ld[LPT];
+    RingDecoder<BITS, SLOW, LANES> ld[LPT];
     uint32_t read_limit[LPT];
 #pragma unroll
     for (int k = 0; k < LPT; k++) {
         const int l = lane + kLanes * k;
-        ld[k].init(s, buf + l, ost + (BITS == 4 ? l : 2 * l), stage_rows - 1);
+        ld[k].init(smem_addr(s.lut), smem_addr(buf + l), smem_addr(ost + (BITS == 4 ? l : 2 * l)), stage_rows - 1,
+                   true);
         // a valid lane never moves more than kOverrunRows rows past its words
         read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
     }
@@ -803,8 +829,10 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
                                          : 0;
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
-            // a lane may run up to kLookahead runs into the next block, never past the chunk
-            decode_to<kLookupsPerCheck>(ld, s, te, te < runs ? te + kLookahead : te, d.max_len, refill_each, status);
+            // a lane may run up to wide_lookahead runs into the next block, never past the chunk
+            wide_decode_to<kLookupsPerCheck>(ld, pk, s.slim, s.soffs, s.ssyms, te,
+                                             te < runs ? te + wide_lookahead<BITS>() : te, d.max_len, refill_each,
+                                             status);
             __syncwarp();
             emit_runs<BITS, OUT, BPAD, LANES>(g, s, ost, first, tb, te, batch, x_in_smem, acc, gst, grow);
             __syncwarp();  // the ring slots just read are rewritten by the next block
@@ -824,19 +852,18 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
             for (int k = 0; k < LPT; k++) {
                 const int full_runs = S[k] >> 3, tail = S[k] & 7;
                 const int tf = min(te, full_runs);
-                while (ld[k].t < tf) {
-                    ld[k].refill();
-                    ld[k].step(s, d.max_len, status);
-                    if (SLOW && refill_each) ld[k].refill();
-                    ld[k].step(s, d.max_len, status);
+                while (ld[k].runs() < tf) {
+                    ld[k].refill(pk);
+                    ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
+                    if (SLOW && refill_each) ld[k].refill(pk);
+                    ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
                 }
-                if (tail && ld[k].t == full_runs && full_runs < te) {
-                    while (ld[k].pb < tail * BITS) {
-                        ld[k].refill();
-                        ld[k].lookup(s, d.max_len, status);
+                // a partial last run: its slot holds the codes after every lookup
+                if (tail && full_runs < te)
+                    while (ld[k].runs() == full_runs && ((ld[k].C >> kPbShift) & 0xFFu) < tail * BITS) {
+                        ld[k].refill(pk);
+                        ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
                     }
-                    ld[k].close_run();
-                }
             }
             __syncwarp();
             emit_ragged<BITS, OUT, LANES>(g, s, ost, first, nc, tb, te);
@@ -880,7 +907,8 @@ template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words);
+    const Smem s = carve(smem_raw, warps, a.x_elems, a.stage_rows * LANES, a.out_words, 0, kWideLutBytes);
+    const Pipes pk{a.k_one, a.k_one << 2, a.k_one << 3, a.k_one << 8, a.k_one << 12, a.k_one << 24};
     uint64_t *bar = s.bars + 2 * warp;
     const size_t buf_words = static_cast<size_t>(a.stage_rows) * LANES;
     uint32_t *stage = s.stage + static_cast<size_t>(warp) * 2 * buf_words;
@@ -918,7 +946,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
         long long cb = (s1 - g.sym_begin + C - 1) / C;
         if (cb > g.d.n_chunks) cb = g.d.n_chunks;
         if (ca >= cb) continue;
-        issue_tables<OUT, SLOW>(g, s, true, a.batch, a.x_in_smem, a.tx_extra);
+        issue_tables<OUT, SLOW>(g, s, 2, a.batch, a.x_in_smem, a.tx_extra);
         // warp w takes chunks ca + w, ca + w + warps, ...  double buffered.  The
         // index entries of the first two are read by four lanes at once, and
         // both copies fly while the tables arrive.
@@ -964,8 +992,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
                 if (b) { phase1++; pend1 = false; }
                 else { phase0++; pend0 = false; }
                 if (chunk_words_ok(g.d, c, a.stage_rows, LANES))
-                    decode_chunk<BITS, OUT, SLOW, BPAD, LANES>(g, s, stage + b * buf_words, ost, a.stage_rows, c,
-                                                               a.batch, a.x_in_smem, a.status);
+                    decode_chunk<BITS, OUT, SLOW, BPAD, LANES>(g, s, pk, stage + b * buf_words, ost, a.stage_rows,
+                                                               c, a.batch, a.x_in_smem, a.status);
                 else
                     set_status(a.status, ENTRO_E_CORRUPT);
                 if (c + 2 * warps < cb) {
@@ -1080,7 +1108,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
         long long cb = (s1 - g.sym_begin + C - 1) / C;
         if (cb > d.n_chunks) cb = d.n_chunks;
         if (ca >= cb) continue;
-        issue_tables<OUT_GEMV, SLOW>(g, s, true, batch, 0, a.tx_extra);
+        issue_tables<OUT_GEMV, SLOW>(g, s, 1, batch, 0, a.tx_extra);
         bool pend0 = false, pend1 = false;
         if (!dead) {
             const long long c = ca + warp;
@@ -1332,7 +1360,7 @@ __global__ void __launch_bounds__(256) single_kernel(const __grid_constant__ Lau
     fence_mbar_init();
     grid_launch_dependents();
     __syncthreads();
-    issue_tables<OUT, SLOW>(g, s, false, 1, 0, a.tx_extra);
+    issue_tables<OUT, SLOW>(g, s, 0, 1, 0, a.tx_extra);
     grid_wait_prior();
     if (!finish_tables<OUT, SLOW>(g, s, 0)) {
         set_status(a.status, ENTRO_E_TIMEOUT);
@@ -2098,7 +2126,8 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
         warps = attempt == 0 ? (wave_warps + 1) / 2 : wave_warps;
         for (;;) {
             so = smem_layout(warps, x_elems, stage_rows * lanes, out_words,
-                             mma ? static_cast<size_t>(warps) * mma_batch_tiles(batch) * 32 * 16 : 0);
+                             mma ? static_cast<size_t>(warps) * mma_batch_tiles(batch) * 32 * 16 : 0,
+                             mma ? kLutSize * 4 : kWideLutBytes);
             if ((long long)so.total <= di.smem_optin) break;
             if (warps > 1) warps--;
             else if (x_elems) { x_elems = 0; warps = kMaxWarps; }
@@ -2127,6 +2156,7 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     a.total_syms = total;
     a.status = status;
     a.tx_extra = g_tx_extra.load(std::memory_order_relaxed);
+    a.k_one = 1;
     const cudaError_t e = launch(fn, (unsigned)grid, warps * 32, bytes, st, a, overlap_ok);
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
 }

@@ -1,0 +1,267 @@
+// wide_decoder.cuh -- the lane decoder with two-word table entries, shared by
+// the lanes-format kernels (decode.cu) and the row-tile kernel (rows.cuh).
+// Included by decode.cu inside namespace entro, after the shared helpers.
+//
+// Each lane keeps a 64-bit MSB-first window of its bitstream in two registers
+// and peeks 12 bits into a table of two-word entries {codes, meta}: up to 8
+// 4-bit or 4 8-bit whole codes of the peek (EntroLLM, arXiv 2505.02380v4: the
+// Huffman-coded chunks decode in parallel; several codes per table lookup),
+// and meta = bits they take | (codes * BITS) << 8.  A counter register C holds
+// the window bits consumed (bits 0-7), the pending code bits (bits 8-15) and
+// the runs completed (bits 16-31), so that adding meta to C does both counts
+// at once and meta itself is the window's shift amount.  Codes longer than 12
+// bits take the canonical slow path.  Every 8 codes form a run, stored in a
+// slot of shared memory in output order.
+
+constexpr uint32_t kPbShift = 8;             // pending code bits: bits 8-15 of the counter
+constexpr uint32_t kRunsShift = 16;          // runs completed: bits 16-31 of the counter
+
+__host__ __device__ constexpr int wide_max_codes(int bits) { return bits == 4 ? 8 : 4; }
+
+// Runs a lane may complete past the check that stops it: STEPS lookups of at
+// most wide_max_codes codes on top of at most 7 pending codes.
+__host__ __device__ constexpr int wide_runs_per_check(int bits, int steps) {
+    return (kRun - 1 + steps * wide_max_codes(bits)) / kRun;
+}
+
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+// Integer constants the compiler cannot see (kernel arguments: 1 and powers of
+// two).  A shift or an addition written as a multiply-add with one of them
+// runs on the FMA pipe (IMAD) instead of the ALU pipe, which the lookups would
+// otherwise saturate: the decode and its emission split their integer work
+// over both pipes.
+struct Pipes {
+    uint32_t one, four, eight, two8, two12, two24;
+};
+
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {  // a * b + c
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t imulhi(uint32_t a, uint32_t b) {  // (a * b) >> 32
+    uint32_t d;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t byte_of(uint32_t v, uint32_t sel) {  // byte sel of v, zero-extended
+    return __byte_perm(v, 0u, 0x4440u | sel);
+}
+
+// RB: bytes from a lane's slot of run t to its slot of run t + 1.  RING = 0:
+// every run has its own slot; RING > 0: RING slots used in turn (run t in slot
+// t mod RING).
+template <int BITS, bool SLOW, int LANES, uint32_t RB, int RING>
+struct WideDecoder {
+    static constexpr uint32_t kRowBytes = 4 * LANES;  // one staged word of every lane
+    static constexpr uint32_t kRunBytes = RB;
+    uint32_t tab;         // shared address of the {codes, meta} table
+    uint32_t bufa;        // shared address of the word held in wnext (a refill advances, then loads)
+    uint32_t bufcap;      // shared address of this lane's last readable word
+    uint32_t hi, lo;      // 64-bit window, MSB first
+    uint32_t wnext;       // next word, loaded one refill ahead
+    uint32_t C;           // consumed window bits | pending bits << 8 | runs << 16
+    uint32_t p0, p1;      // pending codes as one bit string, first code at bit 0 of p0 (p1: 8-bit only)
+    uint32_t osta;        // shared address of the current run's slot
+    uint32_t rend;        // RING > 0: address one ring past this lane's slot of run 0
+
+    // b: shared address of this lane's word 0 (word j at b + kRowBytes j);
+    // slot0: its slot of run 0; cap: last readable staging row.
+    __device__ __forceinline__ void init(uint32_t table, uint32_t b, uint32_t slot0, int cap, bool active) {
+        tab = table;
+        bufcap = b + kRowBytes * static_cast<uint32_t>(cap);
+        hi = lds32(b);
+        lo = lds32(b + kRowBytes);
+        bufa = b + 2 * kRowBytes;
+        wnext = lds32(min(bufa, bufcap));
+        C = active ? 0u : 0xFFFF0000u;  // an empty lane counts as done
+        p0 = p1 = 0;
+        osta = slot0;
+        rend = slot0 + static_cast<uint32_t>(RING) * RB;
+    }
+
+    __device__ __forceinline__ int runs() const { return static_cast<int>(C >> kRunsShift); }
+
+    // When 32 or more window bits are consumed (the valid bits then all sit in
+    // hi and lo is zero), the next word lands right below them.
+    __device__ __forceinline__ void refill(const Pipes &k) {
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p;\n\t"
+            ".reg .u32 x, a;\n\t"
+            "and.b32 x, %2, 32;\n\t"
+            "setp.ne.u32 p, x, 0;\n\t"
+            "@p shf.l.wrap.b32 x, %3, 0, %2;\n\t"  // wnext >> (32 - s), s = consumed - 32
+            "@p mad.lo.u32 %0, x, %6, %0;\n\t"     // hi |= x (x lands on hi's zero bits)
+            "@p shf.l.wrap.b32 %1, 0, %3, %2;\n\t"  // wnext << s
+            "@p mad.lo.u32 %2, %6, %7, %2;\n\t"    // consumed - 32
+            "@p mad.lo.u32 %4, %6, %8, %4;\n\t"    // next word
+            "@p min.u32 a, %4, %5;\n\t"
+            "@p ld.shared.u32 %3, [a];\n\t"
+            "}"
+            : "+r"(hi), "+r"(lo), "+r"(C), "+r"(wnext), "+r"(bufa)
+            : "r"(bufcap), "r"(k.one), "r"(0xFFFFFFE0u), "r"(kRowBytes)
+            : "memory");
+    }
+
+    __device__ __forceinline__ uint2 entry(const Pipes &k) const {
+        return lds64(imad(imulhi(hi, k.two12), k.eight, tab));  // table[window >> 52]
+    }
+
+    // One table lookup: the entry of the window's top 12 bits, or, for a code
+    // longer than 12 bits, the canonical slow path's single code.
+    __device__ __forceinline__ void step(const Pipes &k, const uint32_t *slim, const int32_t *soffs,
+                                         const uint8_t *ssyms, int max_len, int32_t *status) {
+        uint2 e = entry(k);
+        if (SLOW && (e.y & 31u) == 0) {
+            const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
+            const uint32_t se = slow_entry(win, max_len, slim, soffs, ssyms, status);
+            e.x = (se >> 8) & 0xFFu;
+            e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
+        }
+        advance(k, e.x, e.y);
+    }
+
+    // The same lookup, made a no-op (no bits consumed, no codes appended) for a
+    // lane that is done: lets the streams of a thread run in one basic block.
+    __device__ __forceinline__ void step_if(bool live, const Pipes &k, const uint32_t *slim, const int32_t *soffs,
+                                            const uint8_t *ssyms, int max_len, int32_t *status) {
+        uint2 e = entry(k);
+        e.x = live ? e.x : 0u;
+        e.y = live ? e.y : 0u;
+        if (SLOW && live && (e.y & 31u) == 0) {
+            const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
+            const uint32_t se = slow_entry(win, max_len, slim, soffs, ssyms, status);
+            e.x = (se >> 8) & 0xFFu;
+            e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
+        }
+        advance(k, e.x, e.y);
+    }
+
+    // Consume meta's bits, append the codes to the pending string, store the
+    // current run's slot, and move to the next slot when a run is whole.
+    // Appends land on zero bits of the string, so they are additions.
+    __device__ __forceinline__ void advance(const Pipes &k, uint32_t codes, uint32_t meta) {
+        advance_linear(k, codes, meta);
+        if (RING > 0) {
+            // the slot after the ring's last is its first
+            asm volatile(
+                "{\n\t"
+                ".reg .pred w;\n\t"
+                "setp.ge.u32 w, %0, %1;\n\t"
+                "@w sub.u32 %0, %0, %2;\n\t"
+                "}"
+                : "+r"(osta)
+                : "r"(rend), "n"(RING * RB));
+        }
+    }
+
+    __device__ __forceinline__ void advance_linear(const Pipes &k, uint32_t codes, uint32_t meta) {
+        if (BITS == 4) {
+            // pending bits < 32 before the append; what passes bit 32 (phi) starts the next run
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 q, plo, phi, x;\n\t"
+                ".reg .pred dn;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %7;\n\t"
+                "shf.l.wrap.b32 %1, 0, %1, %7;\n\t"
+                "mul.hi.u32 q, %2, %9;\n\t"           // pending bits (C >> 8; the shifts use q mod 32)
+                "shf.l.wrap.b32 plo, 0, %6, q;\n\t"
+                "shf.l.wrap.b32 phi, %6, 0, q;\n\t"
+                "mad.lo.u32 %3, plo, %8, %3;\n\t"
+                "mad.lo.u32 %2, %7, %8, %2;\n\t"      // C += meta
+                "st.shared.u32 [%4], %3;\n\t"
+                "and.b32 x, %2, 0x2000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "selp.b32 %3, phi, %3, dn;\n\t"
+                "@dn mad.lo.u32 %2, %8, %10, %2;\n\t"  // runs + 1, pending - 32
+                "@dn mad.lo.u32 %4, %8, %5, %4;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xE000u)
+                : "memory");
+        } else {
+            // pending bits < 64 before the append: below bit 32 of the string the codes
+            // go to p0 and what passes bit 32 to p1 (then zero); above, to p1 and past bit 64
+            // (phi) to the next run
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 q, plo, phi, x;\n\t"
+                ".reg .pred hs, dn;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %8;\n\t"
+                "shf.l.wrap.b32 %1, 0, %1, %8;\n\t"
+                "mul.hi.u32 q, %2, %10;\n\t"
+                "shf.l.wrap.b32 plo, 0, %7, q;\n\t"
+                "shf.l.wrap.b32 phi, %7, 0, q;\n\t"
+                "and.b32 x, %2, 0x2000;\n\t"
+                "setp.ne.u32 hs, x, 0;\n\t"
+                "selp.b32 %4, %4, phi, hs;\n\t"
+                "@!hs mad.lo.u32 %3, plo, %9, %3;\n\t"
+                "@hs mad.lo.u32 %4, plo, %9, %4;\n\t"
+                "mad.lo.u32 %2, %8, %9, %2;\n\t"
+                "st.shared.v2.u32 [%5], {%3, %4};\n\t"
+                "and.b32 x, %2, 0x4000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "selp.b32 %3, phi, %3, dn;\n\t"
+                "selp.b32 %4, 0, %4, dn;\n\t"
+                "@dn mad.lo.u32 %2, %9, %11, %2;\n\t"  // runs + 1, pending - 64
+                "@dn mad.lo.u32 %5, %9, %6, %5;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(p1), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xC000u)
+                : "memory");
+        }
+    }
+};
+
+// Advance every lane the thread serves to at least run te, STEPS lookups per
+// check, until every lane of the warp has reached te; a lane that is ahead
+// keeps decoding up to run cap (the chunk's end).
+template <int STEPS, int BITS, bool SLOW, int LANES, uint32_t RB, int RING, int LPT>
+__device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB, RING> (&ld)[LPT], const Pipes &pk,
+                                               const uint32_t *slim,
+                                               const int32_t *soffs, const uint8_t *ssyms, int te, int cap,
+                                               int max_len, bool refill_each, int32_t *status) {
+    const uint32_t te_c = static_cast<uint32_t>(te) << kRunsShift, cap_c = static_cast<uint32_t>(cap) << kRunsShift;
+    for (;;) {
+        bool behind = false;
+#pragma unroll
+        for (int k = 0; k < LPT; k++) behind = behind || ld[k].C < te_c;
+        if (!__any_sync(0xffffffffu, behind)) break;
+        if (LPT == 1) {
+            if (ld[0].C < cap_c) {
+#pragma unroll
+                for (int h = 0; h < STEPS / 2; h++) {
+                    ld[0].refill(pk);
+                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
+                    if (SLOW && refill_each) ld[0].refill(pk);
+                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
+                }
+            }
+        } else {
+            // several streams per thread: their lookups interleave (independent chains)
+            bool live[LPT];
+#pragma unroll
+            for (int k = 0; k < LPT; k++) live[k] = ld[k].C < cap_c;
+#pragma unroll
+            for (int h = 0; h < STEPS / 2; h++) {
+#pragma unroll
+                for (int k = 0; k < LPT; k++) ld[k].refill(pk);
+#pragma unroll
+                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
+                if (SLOW && refill_each)
+#pragma unroll
+                    for (int k = 0; k < LPT; k++) ld[k].refill(pk);
+#pragma unroll
+                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
+            }
+        }
+    }
+}
+
