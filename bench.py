@@ -1,7 +1,7 @@
 """Benchmark of the Huffman weight-decoding hot path on B200.
 
-The line's headline is BASELINE's fused-GEMV metric on its Mistral-7B-shaped
-configuration: one simulated token-generation step = the fused decode ->
+The line's headline is the fused-GEMV rate on a Mistral-7B-shaped model: one
+simulated token-generation step = the fused decode ->
 dequantize -> GEMV of all 224 projection tensors (32 layers of q, k, v, o,
 gate, up, down; Laplace weights, tensor-level asymmetric 4-bit codes, one
 Huffman code per tensor, 6.98 G weights, ~1.42 GB of coded bytes) against bf16
@@ -23,6 +23,10 @@ With N > 1 (torchrun) every rank runs the step on its own GPU (tensors are
 independent problems; no data-path collective) and the line reports the
 whole-job rate from the slowest rank ("weak" scaling).  --impl reference times
 the CPU oracle doing the same step on a bounded sample and extrapolates.
+
+--profile runs only W warm-up and K timed launches of the chosen workload (no
+burn-in, end-to-end leg, extras or CPU leg), so that a profiler attached to it
+sees few launches; its line carries the launch time but no clocks.
 """
 from __future__ import annotations
 
@@ -233,7 +237,7 @@ def _time_launches(fn, steps, stream, sleep_s=0.0):
 
 
 def _step_bytes(infos, step):
-    """Algorithmic bytes of one GEMV step (SURVEY section 8(d)): coded bits of every
+    """Algorithmic bytes of one GEMV step: coded bits of every
     tensor (lane padding excluded) / 8 + chunk index + one copy of each tensor's decode
     tables + activations + outputs.  The bf16 weights are never written."""
     table = 32768 + 512
@@ -451,7 +455,7 @@ def _smollm_bf16(entro, device, stream, steps, peak):
     return out
 
 
-def _tensor_kernels(entro, device, stream, steps, peak, clk_mhz, sms):
+def _tensor_kernels(entro, device, stream, steps, peak, clk_mhz, sms, min_steps=20):
     """The 4096x4096 4-bit tensor (32 interleaved lanes per 8192-symbol chunk): decode to
     codes, to bf16 and the batch-1 GEMV, each K launches back to back over 40 rotating
     replicas (160 MB of coded words, inputs larger than L2)."""
@@ -486,7 +490,7 @@ def _tensor_kernels(entro, device, stream, steps, peak, clk_mhz, sms):
            "gemv": coded + index + 2.0 * spec.cols + 4.0 * spec.rows}
     out = {}
     for name, fn in kernels:
-        ms = _time_launches(fn, max(steps, 20), stream, 1e-4)
+        ms = _time_launches(fn, max(steps, min_steps), stream, 1e-4 if min_steps else 0.0)
         gbs = alg[name] / (ms * 1e-3) / 1e9
         out[name] = {"us": round(1e3 * ms, 3), "gsym_s": round(n / (ms * 1e-3) / 1e9, 2), "alg_bytes": int(alg[name]),
                      "achieved_gbs": round(gbs, 1), "hbm_frac": round(gbs / peak, 4),
@@ -517,6 +521,8 @@ def run_step(args, dist, rank, world, local_rank):
     for _ in range(max(3, args.warmup)):
         step.launch(status)
     torch.cuda.synchronize(device)
+    if args.profile:
+        return _profile_line(W, infos, lambda: step.launch(status), args, stream, status, dist, rank)
     clocks = ClockSampler(device)
     clocks.start()
     t_end = time.perf_counter() + 1.0  # burn-in, so that clock samples cover a loaded GPU
@@ -581,6 +587,19 @@ def run_step(args, dist, rank, world, local_rank):
     return 0
 
 
+def _profile_line(W, infos, launch, args, stream, status, dist, rank):
+    """--profile: K launches after the warm-up, one short line, nothing else launched."""
+    device = status.device
+    ms = _time_launches(launch, args.steps, stream)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    ms = _max_over_ranks(dist, ms, device)
+    if rank == 0:
+        print(json.dumps({"profile": W.name, "tensors": len(infos), "symbols": sum(i["n"] for i in infos),
+                          "warmup": args.warmup, "steps": args.steps, "ms_per_launch": round(ms, 5),
+                          "note": "profiling run: no burn-in or clock samples; not a bench value"}), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ other workloads (not the default line)
 
 def run_model(args, dist, rank, world, local_rank):
@@ -611,6 +630,8 @@ def run_model(args, dist, rank, world, local_rank):
     for _ in range(args.warmup):
         launch()
     torch.cuda.synchronize(device)
+    if args.profile:
+        return _profile_line(W, infos, launch, args, stream, status, dist, rank)
     clocks = ClockSampler(device)
     clocks.start()
     t_end = time.perf_counter() + 1.0
@@ -659,7 +680,7 @@ def run_tensor(args, dist, rank, world, local_rank):
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     clocks = ClockSampler(device)
     clocks.start()
-    out = _tensor_kernels(entro, device, stream, args.steps, peak, None, sms)
+    out = _tensor_kernels(entro, device, stream, args.steps, peak, None, sms, 0 if args.profile else 20)
     clk = clocks.stop()
     if rank == 0:
         print(json.dumps({"workload": TENSOR_WORKLOAD, "kernels": out, "clocks": clk}), flush=True)
@@ -741,6 +762,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="default line without its extra workloads")
+    ap.add_argument("--profile", action="store_true",
+                    help="warm-up and timed launches only (no burn-in, e2e, extras or CPU leg): for ncu")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch without overlap (programmatic dependent launch, on by default)")
     ap.add_argument("--workload", default=WORKLOAD,

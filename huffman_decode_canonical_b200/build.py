@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libentro.so")
 SOURCES = [os.path.join(CSRC, "decode.cu"), os.path.join(CSRC, "encoder.cpp")]
-HEADERS = [os.path.join(CSRC, f) for f in ("blob_format.h", "entro_internal.h")] + [
+HEADERS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))) + [
     os.path.join(ROOT, "include", "entro.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

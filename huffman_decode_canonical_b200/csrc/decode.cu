@@ -282,10 +282,20 @@ __device__ __forceinline__ uint32_t dequant_bf16_bits(int q, int zero, float sca
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
+// The 4-bit value-pair table (the bf16 values of both codes of a byte) is stored
+// at a swizzled index: bits 5..7 of the byte (the high code's upper three bits)
+// are XORed into bits 2..4.  A warp's 32 lookups take bytes of 32 different
+// runs; with the plain index a byte's bank is its low code and the high code's
+// lowest bit, so the frequent high codes 6, 8, 10 (or 7, 9) of a centred
+// 4-bit distribution share banks.  The swizzle is a bijection and keeps the
+// table at 256 words; one shift and one LOP3 swizzle all four bytes of a slot.
+__host__ __device__ constexpr uint32_t vpair_index(uint32_t b) { return b ^ ((b >> 3) & 0x1Cu); }
+__device__ __forceinline__ uint32_t vpair_swizzle4(uint32_t c) { return c ^ ((c >> 3) & 0x1C1C1C1Cu); }
+
 // Per-tensor tables into shared memory.  vtab[q] is the dequantized weight
 // bf16_rne(float(q - zero) * scale) (EntroLLM: weights are kept as quantized
 // codes and dequantized for inference), computed here in fp32 once per CTA;
-// vpair[b] holds the values of both 4-bit codes of byte b.  The decode table,
+// vpair[vpair_index(b)] holds the values of both 4-bit codes of byte b.  The decode table,
 // the canonical tables and (GEMV) the activations arrive by bulk copies on the
 // CTA barrier; thread 0 issues them at phase `tphase`.
 // table: 0 = one code per entry (lut), 1 = several (mlut), 2 = the two-word table (wlut)
@@ -322,7 +332,7 @@ __device__ bool finish_tables(const GroupEntry &g, const Smem &s, uint32_t tphas
             const uint32_t v = q < (1 << d.bits) ? dequant_bf16_bits(q, d.zero, d.scale) : 0u;
             s.vtab[q] = v;
             if (d.bits == 4)
-                s.vpair[q] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
+                s.vpair[vpair_index(q)] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
                              (dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
         }
     }
@@ -569,7 +579,7 @@ template <int BITS>
 __device__ __forceinline__ uint4 values8(const Smem &s, const uint32_t *ost, int w) {
     uint4 v;
     if (BITS == 4) {
-        const uint32_t c = ost[w];
+        const uint32_t c = vpair_swizzle4(ost[w]);
         v.x = s.vpair[c & 0xFFu];
         v.y = s.vpair[(c >> 8) & 0xFFu];
         v.z = s.vpair[(c >> 16) & 0xFFu];

@@ -75,7 +75,7 @@ template <int BITS>
 __device__ __forceinline__ uint4 slot_values(uint32_t slot, uint32_t vtab, uint32_t vpair, const Pipes &k) {
     uint4 v;
     if (BITS == 4) {
-        const uint32_t c = lds32(slot);
+        const uint32_t c = vpair_swizzle4(lds32(slot));
         v.x = lds32(imad(byte_of(c, 0), k.four, vpair));
         v.y = lds32(imad(byte_of(c, 1), k.four, vpair));
         v.z = lds32(imad(byte_of(c, 2), k.four, vpair));
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
             for (int q = threadIdx.x; q < 256; q += blockDim.x) {
                 svtab[q] = q < (1 << d.bits) ? dequant_bf16_bits(q, d.zero, d.scale) : 0u;
                 if (BITS == 4)
-                    svpair[q] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
+                    svpair[vpair_index(q)] = dequant_bf16_bits(q & 15, d.zero, d.scale) |
                                 (dequant_bf16_bits(q >> 4, d.zero, d.scale) << 16);
             }
         }
