@@ -30,7 +30,7 @@ _lock = threading.Lock()
 OK, EINVAL, ELIMIT, EFORMAT, ECORRUPT, ENOMEM = 0, -1, -2, -3, -4, -5
 MODE_AUTO, MODE_UNSIGNED, MODE_ASYM = 0, 1, 2
 SCHEME_UNSIGNED, SCHEME_ASYM = 0, 1
-FMT_SINGLE, FMT_LANES, FMT_ROWS = 1, 2, 3
+FMT_SINGLE, FMT_LANES, FMT_ROWS, FMT_ROWS_CO = 1, 2, 3, 4
 
 
 class OracleError(RuntimeError):
@@ -177,7 +177,7 @@ def _chunk_first(p: Dict, c: int) -> int:
     """Symbols in the chunks before chunk c, from the blob's geometry (chunk order)."""
     if c >= p["n_chunks"]:
         return p["n"]
-    if p["format"] != FMT_ROWS:
+    if p["format"] not in (FMT_ROWS, FMT_ROWS_CO):
         return min(p["n"], c * p["chunk_symbols"])
     rows, cols, lanes = p["rows"], p["cols"], p["lanes"]
     kc = p["chunk_symbols"] // lanes

@@ -44,6 +44,9 @@
  *    column tile) codes in column order; a tile with fewer than L rows leaves
  *    the remaining lanes empty.  Lanes are padded and word-interleaved as
  *    above.  Columns and Kc must be multiples of 8.
+ *  - consumption-order row tiles: the same tiles and lane streams, each lane
+ *    keeping only its own words, stored in the order a lock-step reference
+ *    decoder takes them (section 5b).
  *
  * Numeric formulas checked elsewhere against independent pins (see tests).
  */
@@ -69,6 +72,7 @@
 #define OR_FMT_SINGLE 1
 #define OR_FMT_LANES 2
 #define OR_FMT_ROWS 3
+#define OR_FMT_ROWS_CO 4
 
 #define OR_RUN 8
 #define OR_HEADER_BYTES 128
@@ -419,10 +423,134 @@ static tile tile_of(int64_t rows, int64_t cols, int lanes, int64_t chunk_symbols
     return t;
 }
 
+/* ------------------------------------------------------------------ */
+/* 5b. Row tiles in consumption order (format 4).
+ *
+ * A tile's lanes code the same bits as in the row-tile layout; what differs
+ * is where their words sit.  Word-by-word interleaving pads every lane to the
+ * tile's longest lane; here a lane keeps only its own words, and after its
+ * first three they are stored in the order a reference decoder running all
+ * lanes in lock step takes them.  A chunk is
+ *   [the number of words of each lane: L counts of 1 byte, or of 2 bytes
+ *    when ceil(Kc * max_len / 32) > 255, little-endian, zero-padded to whole
+ *    words]
+ *   [words 0, 1, 2 of every lane, word j of lane l at row j, column l (zero
+ *    where the lane has fewer words)]
+ *   [every later word, in the order the reference decoder takes them]
+ *   [zero words up to a multiple of 4 words]
+ * The reference decoder, per lane:
+ *   - a lookup takes, from the lane's next codes, the longest run of whole
+ *     codes whose lengths add up to at most 12 bits, at most 8 codes (4-bit)
+ *     or 4 (8-bit); when the next code is longer than 12 bits it takes that
+ *     code alone;
+ *   - lookups are numbered 0, 1, 2, ...; a refill point comes before each
+ *     even-numbered lookup (before every lookup when the tensor's longest
+ *     code is longer than 16 bits);
+ *   - the lane adds the bits of each lookup to a count c (0 at the start); at
+ *     a refill point with c >= 32 it subtracts 32 and, if some of its words
+ *     are not yet placed, takes the next one;
+ *   - the words taken at one refill point are placed in lane order.
+ */
+#define OR_PEEK_BITS 12
+
+static int co_count_bytes(int64_t kc, int max_len) { return ((int64_t)kc * max_len + 31) / 32 <= 255 ? 1 : 2; }
+
+static uint64_t co_header_words(int lanes, int count_bytes) { return ((uint64_t)lanes * (uint64_t)count_bytes + 3) / 4; }
+
+typedef struct {
+    int64_t width;      /* codes of the lane */
+    int64_t done;       /* codes its lookups have taken */
+    int64_t lookups;    /* lookups made */
+    int c;              /* bits taken since the start, less 32 per refill */
+    uint64_t nw, taken; /* words of the lane; words placed so far */
+} co_lane;
+
+/* length of code i of a lane (decoding it first if needed), < 0 on error */
+typedef int (*co_len_fn)(void *ctx, int lane, int64_t i);
+/* word `word` of a lane is the next one placed */
+typedef int (*co_place_fn)(void *ctx, int lane, uint64_t word);
+
+/* Replay the reference decoder over the lanes of one tile, calling place()
+ * for each word after a lane's first three, in placement order. */
+static int co_schedule(co_lane *ln, int lanes, int every, int bits, co_len_fn len_of, co_place_fn place,
+                       void *ctx) {
+    const int m = bits == 4 ? 8 : 4;
+    for (uint64_t p = 0;; p++) {
+        int open = 0;
+        for (int l = 0; l < lanes; l++) {
+            co_lane *s = &ln[l];
+            if (s->taken >= s->nw) continue;
+            open = 1;
+            const int64_t before = every ? (int64_t)p : 2 * (int64_t)p; /* lookups before this refill point */
+            while (s->lookups < before) {
+                if (s->done >= s->width) return OR_ECORRUPT; /* words left but no codes */
+                int first = len_of(ctx, l, s->done);
+                if (first < 0) return first;
+                int used = 0;
+                int64_t k = 0;
+                if (first > OR_PEEK_BITS) {
+                    used = first;
+                    k = 1;
+                } else {
+                    while (k < m && s->done + k < s->width) {
+                        int lk = len_of(ctx, l, s->done + k);
+                        if (lk < 0) return lk;
+                        if (used + lk > OR_PEEK_BITS) break;
+                        used += lk;
+                        k++;
+                    }
+                }
+                s->done += k;
+                s->c += used;
+                s->lookups++;
+            }
+            if (s->c >= 32) {
+                s->c -= 32;
+                int r = place(ctx, l, s->taken);
+                if (r != OR_OK) return r;
+                s->taken++;
+            }
+        }
+        if (!open) return OR_OK;
+    }
+}
+
+static int longest_code(const uint8_t *len) {
+    int mx = 0;
+    for (int s = 0; s < 256; s++)
+        if (len[s] > mx) mx = len[s];
+    return mx;
+}
+
+/* encoder side: the lanes' code lengths are known */
+typedef struct {
+    const uint8_t *const *lens; /* per lane, code lengths in column order */
+    uint32_t *const *words;     /* per lane, its words */
+    uint32_t *out;              /* the chunk's words */
+    uint64_t pos;               /* next placement */
+} co_enc;
+
+static int co_enc_len(void *ctx, int lane, int64_t i) { return ((co_enc *)ctx)->lens[lane][i]; }
+
+static int co_enc_place(void *ctx, int lane, uint64_t word) {
+    co_enc *e = (co_enc *)ctx;
+    e->out[e->pos++] = e->words[lane][word];
+    return OR_OK;
+}
+
+/* words of one consumption-order tile (header, three rows, the rest, padding) */
+static uint64_t co_tile_words(const uint64_t *nw, int lanes, int count_bytes) {
+    uint64_t w = co_header_words(lanes, count_bytes) + 3 * (uint64_t)lanes;
+    for (int l = 0; l < lanes; l++) w += nw[l] > 3 ? nw[l] - 3 : 0;
+    return (w + 3) & ~(uint64_t)3;
+}
+
 int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, int max_len,
               int format, int64_t chunk_symbols, int lanes, uint8_t *out, uint64_t cap, uint64_t *out_size) {
     if (rows < 0 || cols < 0 || (bits != 4 && bits != 8)) return OR_EINVAL;
-    if (format != OR_FMT_SINGLE && format != OR_FMT_LANES && format != OR_FMT_ROWS) return OR_EINVAL;
+    if (format != OR_FMT_SINGLE && format != OR_FMT_LANES && format != OR_FMT_ROWS && format != OR_FMT_ROWS_CO)
+        return OR_EINVAL;
+    const int tiles = format == OR_FMT_ROWS || format == OR_FMT_ROWS_CO;
     if (max_len == 0) max_len = (bits == 8) ? 16 : 12;
     if (max_len < 1 || max_len > 24) return OR_EINVAL;
     if (chunk_symbols == 0) chunk_symbols = (format == OR_FMT_SINGLE) ? 4096 : 8192;
@@ -433,7 +561,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     if (format != OR_FMT_SINGLE &&
         (chunk_symbols < step || chunk_symbols > 16384 || chunk_symbols % step != 0))
         return OR_EINVAL;
-    if (format == OR_FMT_ROWS && cols % OR_RUN != 0) return OR_EINVAL;
+    if (tiles && cols % OR_RUN != 0) return OR_EINVAL;
     int64_t n = rows * cols;
     int nsym = 1 << bits;
 
@@ -454,7 +582,9 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     or_canonical_codes(len, 256, code);
 
     uint64_t n_chunks = n > 0 ? (uint64_t)((n + chunk_symbols - 1) / chunk_symbols) : 0;
-    if (format == OR_FMT_ROWS) n_chunks = rows_tiles(rows, cols, lanes, chunk_symbols);
+    if (tiles) n_chunks = rows_tiles(rows, cols, lanes, chunk_symbols);
+    const int count_bytes = co_count_bytes(chunk_symbols / lanes, max_len);
+    const int every = longest_code(len) > 16;
 
     /* pass 1: sizes.  Single stream: total bits.  Lanes: per-chunk word count. */
     uint64_t *start = (uint64_t *)calloc(n_chunks + 1, sizeof(uint64_t));
@@ -470,6 +600,21 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
         }
         start[n_chunks] = bitpos;
         payload_words = (bitpos + 31) / 32;
+    } else if (format == OR_FMT_ROWS_CO) {
+        uint64_t wpos = 0, nw[64];
+        for (uint64_t c = 0; c < n_chunks; c++) {
+            start[c] = wpos;
+            tile t = tile_of(rows, cols, lanes, chunk_symbols, c);
+            for (int l = 0; l < lanes; l++) {
+                uint64_t lane_bits = 0;
+                if (l < t.nrows)
+                    for (int64_t k = 0; k < t.width; k++) lane_bits += len[q[(t.row0 + l) * cols + t.col0 + k]];
+                nw[l] = (lane_bits + 31) / 32;
+            }
+            wpos += co_tile_words(nw, lanes, count_bytes);
+        }
+        start[n_chunks] = wpos;
+        payload_words = wpos;
     } else if (format == OR_FMT_ROWS) {
         uint64_t wpos = 0;
         for (uint64_t c = 0; c < n_chunks; c++) {
@@ -534,7 +679,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     uint8_t *idx = out + OR_HEADER_BYTES + OR_LENGTHS_BYTES;
     for (uint64_t c = 0; c <= n_chunks; c++) {
         uint64_t first = c * (uint64_t)chunk_symbols;
-        if (format == OR_FMT_ROWS) first = c < n_chunks ? tile_of(rows, cols, lanes, chunk_symbols, c).first : (uint64_t)n;
+        if (tiles) first = c < n_chunks ? tile_of(rows, cols, lanes, chunk_symbols, c).first : (uint64_t)n;
         if (first > (uint64_t)n) first = (uint64_t)n;
         put_u64(idx + 16 * c, start[c]);
         put_u64(idx + 16 * c + 8, first);
@@ -546,6 +691,55 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     if (format == OR_FMT_SINGLE) {
         bitw bw = {payload, 0};
         for (int64_t i = 0; i < n; i++) put_code(&bw, code[q[i]], len[q[i]]);
+    } else if (format == OR_FMT_ROWS_CO) {
+        const int64_t kc = chunk_symbols / lanes;
+        const uint64_t max_words = ((uint64_t)kc * (uint64_t)max_len + 31) / 32;
+        uint32_t *lw[64];
+        uint8_t *ll[64];
+        uint64_t nw[64];
+        int rc = OR_OK;
+        for (int l = 0; l < lanes; l++) {
+            lw[l] = (uint32_t *)calloc(max_words + 1, sizeof(uint32_t));
+            ll[l] = (uint8_t *)malloc((size_t)kc);
+            if (!lw[l] || !ll[l]) rc = OR_ENOMEM;
+        }
+        for (uint64_t c = 0; rc == OR_OK && c < n_chunks; c++) {
+            tile t = tile_of(rows, cols, lanes, chunk_symbols, c);
+            co_lane st[64];
+            for (int l = 0; l < lanes; l++) {
+                memset(lw[l], 0, sizeof(uint32_t) * (max_words + 1));
+                bitw bw = {lw[l], 0};
+                int64_t width = l < t.nrows ? t.width : 0;
+                for (int64_t k = 0; k < width; k++) {
+                    uint8_t v = q[(t.row0 + l) * cols + t.col0 + k];
+                    put_code(&bw, code[v], len[v]);
+                    ll[l][k] = len[v];
+                }
+                nw[l] = (bw.nbits + 31) / 32;
+                st[l].width = width;
+                st[l].done = st[l].lookups = 0;
+                st[l].c = 0;
+                st[l].nw = nw[l];
+                st[l].taken = nw[l] < 3 ? nw[l] : 3;
+            }
+            uint32_t *chunk = payload + start[c];
+            /* counts, little-endian, count_bytes each */
+            uint8_t *hdr = (uint8_t *)chunk;
+            for (int l = 0; l < lanes; l++) {
+                hdr[count_bytes * l] = (uint8_t)(nw[l] & 0xFF);
+                if (count_bytes == 2) hdr[2 * l + 1] = (uint8_t)(nw[l] >> 8);
+            }
+            /* the header bytes were written into host-order words: make them little-endian words */
+            const uint64_t hw = co_header_words(lanes, count_bytes);
+            for (uint64_t j = 0; j < hw; j++) chunk[j] = get_u32(hdr + 4 * j);
+            for (int j = 0; j < 3; j++)
+                for (int l = 0; l < lanes; l++) chunk[hw + (uint64_t)lanes * j + l] = (uint64_t)j < nw[l] ? lw[l][j] : 0;
+            co_enc e = {(const uint8_t *const *)ll, (uint32_t *const *)lw, chunk, hw + 3 * (uint64_t)lanes};
+            rc = co_schedule(st, lanes, every, bits, co_enc_len, co_enc_place, &e);
+            if (rc == OR_OK && start[c] + e.pos > start[c + 1]) rc = OR_EINVAL;
+        }
+        for (int l = 0; l < lanes; l++) { free(lw[l]); free(ll[l]); }
+        if (rc != OR_OK) { free(q); free(start); free(payload); return rc; }
     } else if (format == OR_FMT_ROWS) {
         for (uint64_t c = 0; c < n_chunks; c++) {
             tile t = tile_of(rows, cols, lanes, chunk_symbols, c);
@@ -626,12 +820,14 @@ static int parse(const uint8_t *blob, uint64_t size, or_blob *b) {
     b->zero = (int32_t)get_u32(blob + 76);
     b->payload_words = get_u64(blob + 80);
     if (b->bits != 4 && b->bits != 8) return OR_EFORMAT;
-    if (b->format != OR_FMT_SINGLE && b->format != OR_FMT_LANES && b->format != OR_FMT_ROWS) return OR_EFORMAT;
+    if (b->format != OR_FMT_SINGLE && b->format != OR_FMT_LANES && b->format != OR_FMT_ROWS &&
+        b->format != OR_FMT_ROWS_CO)
+        return OR_EFORMAT;
     if (b->format != OR_FMT_SINGLE && b->lanes != 32 && b->lanes != 64) return OR_EFORMAT;
     if (b->format == OR_FMT_SINGLE && b->lanes != 1) return OR_EFORMAT;
     if (b->max_len < 1 || b->max_len > 24) return OR_EFORMAT;
     if (b->chunk_symbols == 0 || b->n != b->rows * b->cols) return OR_EFORMAT;
-    if (b->format == OR_FMT_ROWS) {
+    if (b->format == OR_FMT_ROWS || b->format == OR_FMT_ROWS_CO) {
         if (b->chunk_symbols % (OR_RUN * (uint64_t)b->lanes) || b->cols % OR_RUN) return OR_EFORMAT;
         if (b->n_chunks != rows_tiles((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols))
             return OR_EFORMAT;
@@ -702,6 +898,112 @@ static int decode_symbol(const or_blob *b, bit_fn fn, const void *ctx, uint64_t 
     return OR_ECORRUPT;
 }
 
+/* Consumption-order tile c: replay the reference decoder to find each lane's
+ * words, decoding each lane's codes bit by bit as the replay needs their
+ * lengths, then decode the rest of every lane. */
+typedef struct {
+    const or_blob *b;
+    const uint8_t *chunk; /* the chunk's bytes */
+    uint64_t chunk_words, pos;
+    int lanes;
+    uint32_t *words[64];  /* per lane: its words in order */
+    uint64_t nw[64];
+    uint64_t bitpos[64];  /* bits of the lane its decoded codes took */
+    int64_t decoded[64];  /* codes decoded */
+    uint8_t *sym[64];     /* decoded symbols */
+    uint8_t *len[64];     /* their lengths */
+    uint64_t have[64];    /* words of the lane known so far */
+} co_dec;
+
+typedef struct {
+    const co_dec *d;
+    int lane;
+} co_bits;
+
+static int bit_co(const or_blob *b, const void *ctx, uint64_t pos) {
+    (void)b;
+    const co_bits *cb = (const co_bits *)ctx;
+    uint64_t j = pos >> 5;
+    if (j >= cb->d->have[cb->lane]) return -1;
+    return (int)((cb->d->words[cb->lane][j] >> (31 - (pos & 31))) & 1u);
+}
+
+static int co_dec_len(void *ctx, int lane, int64_t i) {
+    co_dec *d = (co_dec *)ctx;
+    while (d->decoded[lane] <= i) {
+        co_bits cb = {d, lane};
+        uint64_t before = d->bitpos[lane];
+        int s = decode_symbol(d->b, bit_co, &cb, &d->bitpos[lane]);
+        if (s < 0) return s;
+        d->sym[lane][d->decoded[lane]] = (uint8_t)s;
+        d->len[lane][d->decoded[lane]] = (uint8_t)(d->bitpos[lane] - before);
+        d->decoded[lane]++;
+    }
+    return d->len[lane][i];
+}
+
+static int co_dec_place(void *ctx, int lane, uint64_t word) {
+    co_dec *d = (co_dec *)ctx;
+    if (d->pos >= d->chunk_words || word != d->have[lane]) return OR_ECORRUPT;
+    d->words[lane][d->have[lane]++] = get_u32(d->chunk + 4 * d->pos);
+    d->pos++;
+    return OR_OK;
+}
+
+static int decode_tile_co(const or_blob *b, uint64_t c, uint64_t start, uint64_t next, const tile *t, uint8_t *out) {
+    const int L = b->lanes;
+    const int cbytes = co_count_bytes((int64_t)(b->chunk_symbols / (uint64_t)L), b->max_len);
+    const uint64_t hw = co_header_words(L, cbytes);
+    (void)c;
+    if (next < start || next > b->payload_words || (next - start) % 4 || next - start < hw + 3 * (uint64_t)L)
+        return OR_ECORRUPT;
+    co_dec d;
+    memset(&d, 0, sizeof(d));
+    d.b = b;
+    d.chunk = b->payload + 4 * start;
+    d.chunk_words = next - start;
+    d.lanes = L;
+    d.pos = hw + 3 * (uint64_t)L;
+    const uint64_t max_words = ((b->chunk_symbols / (uint64_t)L) * (uint64_t)b->max_len + 31) / 32;
+    int r = OR_OK;
+    co_lane st[64];
+    for (int l = 0; l < L; l++) {
+        uint64_t n = d.chunk[cbytes * l];
+        if (cbytes == 2) n |= (uint64_t)d.chunk[2 * l + 1] << 8;
+        int64_t width = l < t->nrows ? t->width : 0;
+        if (n > max_words || (width == 0 && n != 0) || (width > 0 && n == 0)) r = OR_ECORRUPT;
+        d.nw[l] = n;
+        d.words[l] = (uint32_t *)calloc(max_words + 1, sizeof(uint32_t));
+        d.sym[l] = (uint8_t *)malloc((size_t)(t->width > 0 ? t->width : 1));
+        d.len[l] = (uint8_t *)malloc((size_t)(t->width > 0 ? t->width : 1));
+        if (!d.words[l] || !d.sym[l] || !d.len[l]) r = OR_ENOMEM;
+        if (r != OR_OK) continue;
+        for (uint64_t j = 0; j < 3 && j < n; j++) d.words[l][j] = get_u32(d.chunk + 4 * (hw + (uint64_t)L * j + (uint64_t)l));
+        d.have[l] = n < 3 ? n : 3;
+        st[l].width = width;
+        st[l].done = st[l].lookups = 0;
+        st[l].c = 0;
+        st[l].nw = n;
+        st[l].taken = d.have[l];
+    }
+    if (r == OR_OK) {
+        int longest = 0;
+        for (int s = 0; s < 256; s++)
+            if (b->len[s] > longest) longest = b->len[s];
+        r = co_schedule(st, L, longest > 16, b->bits, co_dec_len, co_dec_place, &d);
+    }
+    if (r == OR_OK && ((d.pos + 3) & ~(uint64_t)3) != d.chunk_words) r = OR_ECORRUPT;
+    for (int l = 0; r == OR_OK && l < t->nrows; l++) {
+        for (int64_t k = 0; r == OR_OK && k < t->width; k++) {
+            int lk = co_dec_len(&d, l, k);
+            if (lk < 0) r = lk;
+        }
+        for (int64_t k = 0; r == OR_OK && k < t->width; k++) out[(uint64_t)l * (uint64_t)t->width + (uint64_t)k] = d.sym[l][k];
+    }
+    for (int l = 0; l < L; l++) { free(d.words[l]); free(d.sym[l]); free(d.len[l]); }
+    return r;
+}
+
 /* Chunk c of the row-tile layout into out (the tile's rows one after the
  * other, each in column order). */
 static int decode_tile(const or_blob *b, uint64_t c, uint8_t *out) {
@@ -709,6 +1011,7 @@ static int decode_tile(const or_blob *b, uint64_t c, uint8_t *out) {
     uint64_t first = get_u64(b->index + 16 * c + 8), last = get_u64(b->index + 16 * (c + 1) + 8);
     tile t = tile_of((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols, c);
     if (first != t.first || last != first + (uint64_t)t.nrows * (uint64_t)t.width) return OR_ECORRUPT;
+    if (b->format == OR_FMT_ROWS_CO) return decode_tile_co(b, c, start, next, &t, out);
     const uint64_t L = (uint64_t)b->lanes;
     if (next < start || next > b->payload_words || (next - start) % L) return OR_ECORRUPT;
     lane_ctx lc = {start, 0, b->lanes, (next - start) / L};
@@ -725,7 +1028,7 @@ static int decode_tile(const or_blob *b, uint64_t c, uint8_t *out) {
 }
 
 static int decode_chunk(const or_blob *b, uint64_t c, uint8_t *out /* chunk-local */) {
-    if (b->format == OR_FMT_ROWS) return decode_tile(b, c, out);
+    if (b->format == OR_FMT_ROWS || b->format == OR_FMT_ROWS_CO) return decode_tile(b, c, out);
     uint64_t start = get_u64(b->index + 16 * c), next = get_u64(b->index + 16 * (c + 1));
     uint64_t first = get_u64(b->index + 16 * c + 8), last = get_u64(b->index + 16 * (c + 1) + 8);
     if (first != c * b->chunk_symbols || last < first || last > b->n) return OR_ECORRUPT;
@@ -777,7 +1080,7 @@ int or_blob_params(const uint8_t *blob, uint64_t size, int64_t *out /* 14 entrie
 
 /* symbols in the chunks before chunk c (chunk order) */
 static uint64_t chunk_first(const or_blob *b, uint64_t c) {
-    if (b->format == OR_FMT_ROWS)
+    if (b->format == OR_FMT_ROWS || b->format == OR_FMT_ROWS_CO)
         return c < b->n_chunks ? tile_of((int64_t)b->rows, (int64_t)b->cols, b->lanes, (int64_t)b->chunk_symbols, c).first
                                : b->n;
     uint64_t f = c * b->chunk_symbols;
@@ -805,7 +1108,7 @@ int or_decode(const uint8_t *blob, uint64_t size, uint8_t *out) {
     or_blob *b = (or_blob *)malloc(sizeof(or_blob));
     if (!b) return OR_ENOMEM;
     int r = parse(blob, size, b);
-    if (r != OR_OK || b->format != OR_FMT_ROWS) {
+    if (r != OR_OK || (b->format != OR_FMT_ROWS && b->format != OR_FMT_ROWS_CO)) {
         uint64_t nch = b->n_chunks;
         free(b);
         if (r != OR_OK) return r;

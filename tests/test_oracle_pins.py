@@ -459,3 +459,223 @@ def test_corrupted_blobs_are_rejected_or_detected():
         assert not (got == q).all()
     except oracle.OracleError:
         pass
+
+
+# ---------------------------------------------------------------- consumption-order row tiles
+
+def _co_expected_payload(q, rows, cols, bits, lanes, chunk, lengths, lmax):
+    """The consumption-order layout restated in Python from its definition: each lane's
+    words from its codes (canonical, MSB first); a count header; words 0-2 of every lane
+    in three rows; the later words in the order a lock-step reference decoder takes them
+    (lookups of at most 8 / 4 whole codes within 12 bits, or one longer code; a refill
+    point before every even lookup, before every lookup when a code is longer than 16
+    bits; a lane whose taken bits reach 32 there gives back 32 and takes a word)."""
+    codes = oracle.canonical_codes(lengths)
+    Q = q.reshape(rows, cols)
+    kc = chunk // lanes
+    every = int(lengths.max()) > 16
+    m = 8 if bits == 4 else 4
+    out = []
+    for g in range(-(-rows // lanes)):
+        for j in range(-(-cols // kc)):
+            r0, c0 = g * lanes, j * kc
+            nr, wd = min(lanes, rows - r0), min(kc, cols - c0)
+            lane_words, lane_lens = [], []
+            for lane in range(lanes):
+                bitstr = ""
+                ln = []
+                if lane < nr:
+                    for v in Q[r0 + lane, c0:c0 + wd]:
+                        bitstr += format(int(codes[v]), "0%db" % int(lengths[v]))
+                        ln.append(int(lengths[v]))
+                nwl = -(-len(bitstr) // 32)
+                bitstr += "0" * (32 * nwl - len(bitstr))
+                lane_words.append([int(bitstr[32 * i:32 * i + 32], 2) for i in range(nwl)])
+                lane_lens.append(ln)
+            # schedule
+            state = [dict(done=0, lookups=0, c=0, taken=min(3, len(lane_words[l]))) for l in range(lanes)]
+            order = []
+            p = 0
+            while any(state[l]["taken"] < len(lane_words[l]) for l in range(lanes)):
+                for l in range(lanes):
+                    s = state[l]
+                    if s["taken"] >= len(lane_words[l]):
+                        continue
+                    while s["lookups"] < (p if every else 2 * p):
+                        ln = lane_lens[l]
+                        if ln[s["done"]] > 12:
+                            used, k = ln[s["done"]], 1
+                        else:
+                            used = k = 0
+                            while k < m and s["done"] + k < len(ln) and used + ln[s["done"] + k] <= 12:
+                                used += ln[s["done"] + k]
+                                k += 1
+                        s["done"] += k
+                        s["c"] += used
+                        s["lookups"] += 1
+                    if s["c"] >= 32:
+                        s["c"] -= 32
+                        order.append(lane_words[l][s["taken"]])
+                        s["taken"] += 1
+                p += 1
+            nws = [len(w) for w in lane_words]
+            cb = 1 if -(-kc * lmax // 32) <= 255 else 2
+            hdr = b"".join(int(n).to_bytes(cb, "little") for n in nws)
+            hdr += b"\0" * (-len(hdr) % 4)
+            words = list(np.frombuffer(hdr, np.uint32))
+            for r in range(3):
+                words += [lane_words[l][r] if r < nws[l] else 0 for l in range(lanes)]
+            words += order
+            words += [0] * (-len(words) % 4)
+            out.extend(words)
+    return np.array(out, dtype=np.uint32)
+
+
+@pytest.mark.parametrize("kind,bits,lmax,chunk,rows,cols,lanes", [
+    ("laplace", 4, 12, 8192, 40, 1000, 32),
+    ("t4", 8, 16, 4096, 36, 264, 32),
+    ("laplace", 4, 12, 16384, 70, 512, 64),
+])
+def test_consumption_order_layout_restated(kind, bits, lmax, chunk, rows, cols, lanes):
+    """The oracle's consumption-order payload equals the layout rebuilt from its
+    definition by an independent Python statement, word for word."""
+    w = workloads.small_tensor(kind, rows, cols, seed=7 + rows)
+    blob = oracle.encode(w, bits, oracle.MODE_ASYM, lmax, oracle.FMT_ROWS_CO, chunk, lanes=lanes)
+    prm = oracle.params(blob)
+    q, _, _, _ = oracle.quantize(w, bits, oracle.MODE_ASYM)
+    want = _co_expected_payload(q, rows, cols, bits, lanes, chunk, prm["lengths"], lmax)
+    n_chunks = prm["n_chunks"]
+    got = np.frombuffer(blob, np.uint32, prm["payload_words"], 384 + 16 * (n_chunks + 1))
+    assert got.size == want.size and (got == want).all()
+    assert (oracle.decode(blob) == q).all()
+
+
+@pytest.mark.parametrize("lanes", [32, 64])
+def test_consumption_order_closed_form(lanes):
+    """One-bit codes: every lookup takes 8 codes (8 bits), so a lane's count reaches 32 at
+    every second refill point: word 3 + k of every lane is taken at refill point 2k + 2,
+    all lanes of the tile in lane order.  Tiles of 160 and 104 columns (5 and 4 words per
+    lane), a second row group of 6 rows."""
+    kc = 160
+    rows, cols = lanes + 6, kc + 104
+    b = (((np.arange(rows)[:, None] * 3 + np.arange(cols)[None, :] * 5) % 11) < 4).astype(np.uint8)
+    blob = oracle.encode(_two_code_tensor(b), 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS_CO, lanes * kc,
+                         lanes=lanes)
+    prm = oracle.params(blob)
+    assert prm["format"] == oracle.FMT_ROWS_CO and prm["n_chunks"] == 4
+    assert prm["lengths"][0] == 1 and prm["lengths"][15] == 1 and prm["lengths"].sum() == 2
+    idx = np.frombuffer(blob, np.uint64, 10, 384).reshape(-1, 2)
+    words = np.frombuffer(blob, np.uint32, prm["payload_words"], 384 + 80)
+    hw = lanes // 4                                       # one count byte per lane
+    start = 0
+    for c, (g, j) in enumerate([(0, 0), (0, 1), (1, 0), (1, 1)]):
+        r0, c0 = g * lanes, j * kc
+        nr, wd = min(lanes, rows - r0), min(kc, cols - c0)
+        nw = -(-wd // 32)
+
+        def lane_word(lane, i):
+            e = 0
+            for k in range(32):
+                if 32 * i + k < wd:
+                    e |= int(b[r0 + lane, c0 + 32 * i + k]) << (31 - k)
+            return e
+
+        assert int(idx[c, 0]) == start
+        counts = np.frombuffer(words[start:start + hw].tobytes(), np.uint8)
+        assert counts.tolist() == [nw] * nr + [0] * (lanes - nr)
+        for r in range(3):
+            for lane in range(lanes):
+                assert int(words[start + hw + lanes * r + lane]) == (lane_word(lane, r) if lane < nr else 0)
+        pos = start + hw + 3 * lanes
+        for k in range(nw - 3):
+            for lane in range(nr):
+                assert int(words[pos]) == lane_word(lane, 3 + k), (c, k, lane)
+                pos += 1
+        size = hw + 3 * lanes + nr * (nw - 3)
+        size += -size % 4
+        assert all(int(x) == 0 for x in words[pos:start + size])
+        start += size
+    assert int(idx[-1, 0]) == start == prm["payload_words"]
+
+
+def _long_code_tensor(rows, cols, seed):
+    """8-bit codes with geometric frequencies (symbol k about 2^-k of the weights), so
+    that the Huffman lengths reach past 16 bits under a 20-bit limit."""
+    n = rows * cols
+    counts = [max(1, n >> (k + 1)) for k in range(24)]
+    vals = np.concatenate([np.full(c, k, np.float32) for k, c in enumerate(counts)])
+    vals = np.concatenate([vals, np.full(max(0, n - vals.size), 0, np.float32)])[:n]
+    vals[-1] = 255.0                                     # scale 1, zero 0: q = w
+    rng = np.random.default_rng(seed)
+    rng.shuffle(vals)
+    return vals.reshape(rows, cols)
+
+
+CO_CASES = [
+    ("laplace", 4, oracle.MODE_ASYM, 12, 8192, 100, 1000, 32),
+    ("t4", 8, oracle.MODE_AUTO, 16, 4096, 70, 3072, 32),
+    ("skew", 8, oracle.MODE_ASYM, 16, 512, 33, 24, 32),
+    ("laplace", 4, oracle.MODE_ASYM, 12, 1024, 130, 520, 64),
+    ("uniform", 8, oracle.MODE_ASYM, 16, 16384, 40, 1024, 32),
+    ("two_values", 4, oracle.MODE_ASYM, 12, 256, 1, 8, 32),
+]
+
+
+@pytest.mark.parametrize("case", CO_CASES, ids=[f"{c[0]}-b{c[1]}-c{c[4]}-{c[5]}x{c[6]}-L{c[7]}" for c in CO_CASES])
+def test_consumption_order_identity(case):
+    kind, bits, mode, lmax, chunk, rows, cols, lanes = case
+    w = workloads.small_tensor(kind, rows, cols, seed=rows + cols)
+    blob = oracle.encode(w, bits, mode, lmax, oracle.FMT_ROWS_CO, chunk, lanes=lanes)
+    q, _, _, _ = oracle.quantize(w, bits, mode)
+    assert (oracle.decode(blob) == q).all()
+    static = oracle.encode(w, bits, mode, lmax, oracle.FMT_ROWS, chunk, lanes=lanes)
+    assert oracle.params(blob)["lengths"].tolist() == oracle.params(static)["lengths"].tolist()
+    prm = oracle.params(blob)
+    if prm["n_chunks"] > 1:
+        Q = q.reshape(rows, cols)
+        part = oracle.decode_chunks(blob, 1, prm["n_chunks"])
+        tiles = [oracle.tile(prm, c) for c in range(1, prm["n_chunks"])]
+        want = np.concatenate([Q[r0:r0 + nr, k0:k0 + wd].reshape(-1) for r0, k0, nr, wd in tiles])
+        assert (part == want).all()
+
+
+def test_consumption_order_long_codes():
+    """Codes longer than 16 bits: refill points before every lookup."""
+    w = _long_code_tensor(256, 1024, 5)
+    blob = oracle.encode(w, 8, oracle.MODE_ASYM, 20, oracle.FMT_ROWS_CO, 8192, lanes=32)
+    prm = oracle.params(blob)
+    assert int(prm["lengths"].max()) > 16
+    q, _, _, _ = oracle.quantize(w, 8, oracle.MODE_ASYM)
+    assert (oracle.decode(blob) == q).all()
+    want = _co_expected_payload(q, 256, 1024, 8, 32, 8192, prm["lengths"], 20)
+    got = np.frombuffer(blob, np.uint32, prm["payload_words"], 384 + 16 * (prm["n_chunks"] + 1))
+    assert (got == want).all()
+
+
+def test_consumption_order_smaller_than_padded_lanes():
+    """On a Mistral-shaped 4-bit tile set the consumption order stores fewer words than
+    lanes padded to the tile's longest (the point of the layout)."""
+    W = workloads.get("mistral_7b_u4")
+    w = workloads.weights(W, W.tensors[1]).numpy()[:128]
+    co = oracle.params(oracle.encode(w, 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS_CO, 8192))["payload_words"]
+    st = oracle.params(oracle.encode(w, 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS, 8192))["payload_words"]
+    assert co < 0.97 * st, (co, st)
+
+
+def test_consumption_order_corrupt_counts():
+    w = workloads.small_tensor("laplace", 64, 512, seed=3)
+    blob = bytearray(oracle.encode(w, 4, oracle.MODE_ASYM, 12, oracle.FMT_ROWS_CO, 8192))
+    prm = oracle.params(bytes(blob))
+    base = 384 + 16 * (prm["n_chunks"] + 1)
+    q, _, _, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
+    for extra, must_raise in ((40, True), (200, True), (1, False)):
+        bad = bytearray(blob)
+        bad[base + 5] = (bad[base + 5] + extra) & 0xFF    # lane 5 claims more words than it has
+        if must_raise:                                    # it runs out of codes, or past the limit
+            with pytest.raises(oracle.OracleError):
+                oracle.decode(bytes(bad))
+        else:                                             # every later word shifts: never the same codes
+            try:
+                assert not (oracle.decode(bytes(bad)) == q).all()
+            except oracle.OracleError:
+                pass
