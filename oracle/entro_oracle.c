@@ -444,8 +444,8 @@ static tile tile_of(int64_t rows, int64_t cols, int lanes, int64_t chunk_symbols
  *     or 4 (8-bit); when the next code is longer than 12 bits it takes that
  *     code alone;
  *   - lookups are numbered 0, 1, 2, ...; a refill point comes before each
- *     even-numbered lookup (before every lookup when the tensor's longest
- *     code is longer than 16 bits);
+ *     even-numbered lookup (before every lookup when the code length limit
+ *     max_len is above 16);
  *   - the lane adds the bits of each lookup to a count c (0 at the start); at
  *     a refill point with c >= 32 it subtracts 32 and, if some of its words
  *     are not yet placed, takes the next one;
@@ -515,13 +515,6 @@ static int co_schedule(co_lane *ln, int lanes, int every, int bits, co_len_fn le
     }
 }
 
-static int longest_code(const uint8_t *len) {
-    int mx = 0;
-    for (int s = 0; s < 256; s++)
-        if (len[s] > mx) mx = len[s];
-    return mx;
-}
-
 /* encoder side: the lanes' code lengths are known */
 typedef struct {
     const uint8_t *const *lens; /* per lane, code lengths in column order */
@@ -584,7 +577,7 @@ int or_encode(const float *w, int64_t rows, int64_t cols, int bits, int mode, in
     uint64_t n_chunks = n > 0 ? (uint64_t)((n + chunk_symbols - 1) / chunk_symbols) : 0;
     if (tiles) n_chunks = rows_tiles(rows, cols, lanes, chunk_symbols);
     const int count_bytes = co_count_bytes(chunk_symbols / lanes, max_len);
-    const int every = longest_code(len) > 16;
+    const int every = max_len > 16;
 
     /* pass 1: sizes.  Single stream: total bits.  Lanes: per-chunk word count. */
     uint64_t *start = (uint64_t *)calloc(n_chunks + 1, sizeof(uint64_t));
@@ -986,12 +979,7 @@ static int decode_tile_co(const or_blob *b, uint64_t c, uint64_t start, uint64_t
         st[l].nw = n;
         st[l].taken = d.have[l];
     }
-    if (r == OR_OK) {
-        int longest = 0;
-        for (int s = 0; s < 256; s++)
-            if (b->len[s] > longest) longest = b->len[s];
-        r = co_schedule(st, L, longest > 16, b->bits, co_dec_len, co_dec_place, &d);
-    }
+    if (r == OR_OK) r = co_schedule(st, L, b->max_len > 16, b->bits, co_dec_len, co_dec_place, &d);
     if (r == OR_OK && ((d.pos + 3) & ~(uint64_t)3) != d.chunk_words) r = OR_ECORRUPT;
     for (int l = 0; r == OR_OK && l < t->nrows; l++) {
         for (int64_t k = 0; r == OR_OK && k < t->width; k++) {

@@ -468,12 +468,12 @@ def _co_expected_payload(q, rows, cols, bits, lanes, chunk, lengths, lmax):
     words from its codes (canonical, MSB first); a count header; words 0-2 of every lane
     in three rows; the later words in the order a lock-step reference decoder takes them
     (lookups of at most 8 / 4 whole codes within 12 bits, or one longer code; a refill
-    point before every even lookup, before every lookup when a code is longer than 16
-    bits; a lane whose taken bits reach 32 there gives back 32 and takes a word)."""
+    point before every even lookup, before every lookup when the length limit is above
+    16; a lane whose taken bits reach 32 there gives back 32 and takes a word)."""
     codes = oracle.canonical_codes(lengths)
     Q = q.reshape(rows, cols)
     kc = chunk // lanes
-    every = int(lengths.max()) > 16
+    every = lmax > 16
     m = 8 if bits == 4 else 4
     out = []
     for g in range(-(-rows // lanes)):
@@ -640,7 +640,7 @@ def test_consumption_order_identity(case):
 
 
 def test_consumption_order_long_codes():
-    """Codes longer than 16 bits: refill points before every lookup."""
+    """Length limit 20 (codes longer than 16 bits): refill points before every lookup."""
     w = _long_code_tensor(256, 1024, 5)
     blob = oracle.encode(w, 8, oracle.MODE_ASYM, 20, oracle.FMT_ROWS_CO, 8192, lanes=32)
     prm = oracle.params(blob)
