@@ -54,6 +54,7 @@ TENSOR_WORKLOAD = "laplace_4096x4096_u4"
 REPLICAS = 40
 NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e, HGX figure (context beside the measured copy peak)
 KERNEL_SOURCES = ("huffman_decode_canonical_b200/csrc/decode.cu", "huffman_decode_canonical_b200/csrc/rows.cuh",
+                  "huffman_decode_canonical_b200/csrc/wide_decoder.cuh",
                   "huffman_decode_canonical_b200/csrc/blob_format.h")
 
 
@@ -188,11 +189,18 @@ def encode_model(entro, W: workloads.Workload, device, limit=None, keep=0):
 
 
 def _override(W, args):
-    if not getattr(args, "fmt", ""):
+    if not (getattr(args, "fmt", "") or getattr(args, "lanes", 0) or getattr(args, "chunk", 0)):
         return W
-    fmt = {"lanes": workloads.FORMAT_LANES, "rows": workloads.FORMAT_ROWS}[args.fmt]
+    fmt = {"lanes": workloads.FORMAT_LANES, "rows": workloads.FORMAT_ROWS, "rows_co": workloads.FORMAT_ROWS_CO,
+           "": W.fmt}[args.fmt]
     lanes = args.lanes or W.lanes
-    rule = W.chunk_rule if fmt == workloads.FORMAT_LANES else "fixed:%d" % (args.chunk or 256 * lanes)
+    tiles = (workloads.FORMAT_ROWS, workloads.FORMAT_ROWS_CO)
+    if fmt == workloads.FORMAT_LANES:
+        rule = W.chunk_rule
+    elif args.chunk:
+        rule = "fixed:%d" % args.chunk
+    else:  # row tiles: the workload's own tile size when it has one, else 256 columns
+        rule = W.chunk_rule if W.fmt in tiles and lanes == W.lanes else "fixed:%d" % (256 * lanes)
     return dataclasses.replace(W, fmt=fmt, lanes=lanes, chunk_rule=rule)
 
 
@@ -279,7 +287,7 @@ def _oracle_pass(sample, threads: int, seed: int):
         blob, p, x, c = job
         q = oracle.decode_chunks(blob, c, c + 1)
         wb = oracle.dequant_bf16(q, p["scale"], p["zero"])
-        if p["format"] == oracle.FMT_ROWS:
+        if p["format"] in (oracle.FMT_ROWS, oracle.FMT_ROWS_CO):
             r0, k0, nr, wd = oracle.tile(p, c)
             oracle.gemv(wb.reshape(nr, wd), np.ascontiguousarray(x[:, k0:k0 + wd]))
         else:
@@ -343,7 +351,8 @@ def run_reference(args, rank, world):
 
 def _step_config(W, batch):
     return {"workload": W.name, "tensors": len(W.tensors), "symbols": W.n, "bits": W.bits, "batch": batch,
-            "format": {workloads.FORMAT_LANES: "lanes", workloads.FORMAT_ROWS: "row tiles"}.get(W.fmt, "single"),
+            "format": {workloads.FORMAT_LANES: "lanes", workloads.FORMAT_ROWS: "row tiles",
+                       workloads.FORMAT_ROWS_CO: "row tiles, consumption order"}.get(W.fmt, "single"),
             "lanes": W.lanes, "chunk_symbols": W.chunk_symbols(4096),
             "l2": "inputs larger than L2: the step streams 1.4 GB of coded weights (L2 126 MB); no flush"}
 
@@ -773,7 +782,8 @@ def main(argv=None):
                          "step")
     ap.add_argument("--batch", type=int, default=1, help="GEMV batch for the model-scale GEMV workloads")
     ap.add_argument("--tensors", type=int, default=0, help="model-scale workloads: only the first N tensors")
-    ap.add_argument("--fmt", choices=["lanes", "rows"], default="", help="model-scale workloads: chunk format")
+    ap.add_argument("--fmt", choices=["lanes", "rows", "rows_co"], default="",
+                    help="model-scale workloads: chunk format (rows_co: row tiles in consumption order)")
     ap.add_argument("--lanes", type=int, default=0, help="model-scale workloads: lanes (rows per tile) per chunk")
     ap.add_argument("--chunk", type=int, default=0, help="model-scale workloads, row tiles: symbols per chunk")
     args = ap.parse_args(argv)

@@ -30,7 +30,7 @@ OK = 0
 E_INVAL, E_LIMIT, E_FORMAT, E_CORRUPT, E_OVERRUN, E_NOMEM, E_CUDA, E_TIMEOUT = -1, -2, -3, -4, -5, -6, -7, -8
 QUANT_AUTO, QUANT_UNSIGNED, QUANT_ASYM = 0, 1, 2
 SCHEME_UNSIGNED, SCHEME_ASYM = 0, 1
-FORMAT_SINGLE, FORMAT_LANES, FORMAT_ROWS = 1, 2, 3
+FORMAT_SINGLE, FORMAT_LANES, FORMAT_ROWS, FORMAT_ROWS_CO = 1, 2, 3, 4
 GROUP_GEMV, GROUP_BF16 = 1, 2
 
 
@@ -345,6 +345,6 @@ def set_overlap(enable: bool) -> bool:
 
 __all__ = ["Blob", "DeviceTensor", "Group", "EntroError", "encode", "upload", "lib", "version", "set_overlap", "EXPORTS",
            "decode_gemv_group_static", "STATIC_GROUP_MAX",
-           "test_stall_tables", "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES",
+           "test_stall_tables", "QUANT_AUTO", "QUANT_UNSIGNED", "QUANT_ASYM", "FORMAT_SINGLE", "FORMAT_LANES", "FORMAT_ROWS_CO",
            "FORMAT_ROWS", "GROUP_GEMV",
            "GROUP_BF16", "SCHEME_UNSIGNED", "SCHEME_ASYM"]

@@ -24,8 +24,30 @@
 // row of a ragged row group are empty.  Padding and word interleave as in the
 // lanes format.  cols and Kc are multiples of 8.  The index's first_symbol is
 // the number of symbols in earlier tiles.
+//
+// Row tiles in consumption order (format 4): the tiles and lane bitstreams of
+// the row-tile format, each lane keeping only its own n_l = ceil(bits / 32)
+// words.  A chunk is [n_l of every lane: one byte each, two (little-endian)
+// when ceil(Kc * max_len / 32) > 255, zero-padded to whole words] [words 0-2
+// of every lane as three rows of L words (zero past n_l)] [the later words in
+// the order a lock-step reference decoder takes them] [zero words up to a
+// multiple of 4].  The reference decoder: a lookup takes the longest run of
+// whole codes within kCoPeekBits bits, at most kCoCodes4 (4-bit) or kCoCodes8
+// (8-bit) codes, or one longer code alone; a refill point precedes every
+// even-numbered lookup of a lane (every lookup when the length limit max_len
+// is above kCoRefillEachAbove); the bits a lane's lookups take add up in a count
+// that, at a refill point, gives back 32 when it has reached 32, and the lane
+// then takes its next word if it has one left; the words taken at one refill
+// point are stored in lane order.  The decoder of a warp finds its words with
+// a ballot and a population count, so no lane is padded.
 #pragma once
 #include <stdint.h>
+
+#ifdef __CUDACC__
+#define ENTRO_HD __host__ __device__
+#else
+#define ENTRO_HD
+#endif
 
 namespace entro {
 
@@ -42,6 +64,13 @@ constexpr int kMaxLenLimit = 24;
 constexpr int64_t kMaxLanesChunk = 16384;
 constexpr int64_t kMaxSingleChunk = int64_t(1) << 20;
 constexpr double kMaxZero = 16777216.0;  // |zero| <= 2^24
+constexpr int kCoPeekBits = 12;          // consumption order: the reference lookup's peek
+constexpr int kCoCodes4 = 8, kCoCodes8 = 4;
+constexpr int kCoRefillEachAbove = 16;
+
+// consumption order: bytes of a lane's word count in the chunk header
+ENTRO_HD inline int co_count_bytes(uint64_t kc, uint32_t max_len) { return (kc * max_len + 31) / 32 <= 255 ? 1 : 2; }
+ENTRO_HD inline uint64_t co_header_words(uint64_t lanes, int count_bytes) { return (lanes * count_bytes + 3) / 4; }
 
 #pragma pack(push, 1)
 struct BlobHeader {

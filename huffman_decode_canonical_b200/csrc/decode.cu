@@ -899,18 +899,23 @@ __device__ __forceinline__ bool chunk_words_ok(const DevTensor &d, long long c, 
 
 // Issue the staging copy of a chunk whose words are [st, nx) (one lane).  An
 // inconsistent index arrives with no bytes; the consumer re-checks and skips.
+// A chunk's words [st, nx) into a staging buffer of stage_rows rows of `lanes`
+// words; unit: the chunk sizes the format allows are multiples of it (lanes
+// for word-interleaved lanes, 4 for consumption order).  A chunk that does not
+// fit is not copied (the barrier completes with no bytes; the decode checks
+// the same bounds and reports it).
 __device__ __forceinline__ void issue_words(const DevTensor &d, uint64_t st, uint64_t nx, uint32_t *buf,
-                                            uint64_t *bar, int stage_rows, int lanes) {
-    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % lanes == 0 &&
-                    (nx - st) / lanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
+                                            uint64_t *bar, int stage_rows, int lanes, int unit) {
+    const bool ok = nx >= st && nx <= static_cast<uint64_t>(d.payload_words) && (nx - st) % unit == 0 &&
+                    (nx - st + lanes - 1) / lanes + kSlackRows <= static_cast<uint64_t>(stage_rows);
     const uint32_t bytes = ok ? static_cast<uint32_t>((nx - st) * 4) : 0u;
     mbar_arrive_expect_tx(bar, bytes);
     if (bytes) bulk_copy_g2s(buf, d.payload + st, bytes, bar);
 }
 
 __device__ __forceinline__ void issue_chunk(const DevTensor &d, long long c, uint32_t *buf, uint64_t *bar,
-                                            int stage_rows, int lanes) {
-    issue_words(d, d.index[2 * c], d.index[2 * c + 2], buf, bar, stage_rows, lanes);
+                                            int stage_rows, int lanes, int unit) {
+    issue_words(d, d.index[2 * c], d.index[2 * c + 2], buf, bar, stage_rows, lanes, unit);
 }
 
 template <int BITS, int OUT, bool SLOW, int BPAD, int LANES>
@@ -969,8 +974,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
             const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
             const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
             if (lane == 0) {
-                if (c < cb) issue_words(g.d, st0, nx0, stage, bar, a.stage_rows, LANES);
-                if (c + warps < cb) issue_words(g.d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES);
+                if (c < cb) issue_words(g.d, st0, nx0, stage, bar, a.stage_rows, LANES, LANES);
+                if (c + warps < cb)
+                    issue_words(g.d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES, LANES);
             }
             pend0 = c < cb;
             pend1 = c + warps < cb;
@@ -1009,7 +1015,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) lanes_kernel(const __grid_c
                 if (c + 2 * warps < cb) {
                     if (lane == 0) {
                         fence_proxy_async();
-                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES);
+                        issue_chunk(g.d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES, LANES);
                     }
                     if (b) pend1 = true;
                     else pend0 = true;
@@ -1128,8 +1134,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
             const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
             const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
             if (lane == 0) {
-                if (c < cb) issue_words(d, st0, nx0, stage, bar, a.stage_rows, LANES);
-                if (c + warps < cb) issue_words(d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES);
+                if (c < cb) issue_words(d, st0, nx0, stage, bar, a.stage_rows, LANES, LANES);
+                if (c + warps < cb) issue_words(d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES, LANES);
             }
             pend0 = c < cb;
             pend1 = c + warps < cb;
@@ -1279,7 +1285,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_mma_kernel(const __gri
             if (c < cb && !dead && c + 2 * warps < cb) {
                 if (lane == 0) {
                     fence_proxy_async();
-                    issue_chunk(d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES);
+                    issue_chunk(d, c + 2 * warps, stage + b * buf_words, bar + b, a.stage_rows, LANES, LANES);
                 }
                 if (b) pend1 = true;
                 else pend0 = true;
@@ -2171,35 +2177,42 @@ static int launch_lanes(const TensorHandle *const *ts, int count, int out_kind, 
     return e == cudaSuccess ? ENTRO_OK : cuda_fail(e, "lanes kernel launch");
 }
 
-template <int BITS, int OUT, int LANES>
+template <int BITS, int OUT, int LANES, bool CO>
 static LanesFn pick_rows3(bool slow, int nb) {
-    if (OUT != OUT_GEMV) return slow ? rows_kernel<BITS, OUT, true, LANES, 1> : rows_kernel<BITS, OUT, false, LANES, 1>;
-    if (nb == 2) return slow ? rows_kernel<BITS, OUT, true, LANES, 2> : rows_kernel<BITS, OUT, false, LANES, 2>;
-    return slow ? rows_kernel<BITS, OUT, true, LANES, 1> : rows_kernel<BITS, OUT, false, LANES, 1>;
+    if constexpr (OUT == OUT_GEMV) {
+        if (nb == 2)
+            return slow ? rows_kernel<BITS, OUT, true, LANES, 2, CO> : rows_kernel<BITS, OUT, false, LANES, 2, CO>;
+    }
+    return slow ? rows_kernel<BITS, OUT, true, LANES, 1, CO> : rows_kernel<BITS, OUT, false, LANES, 1, CO>;
 }
 
-template <int BITS, int LANES>
+template <int BITS, int LANES, bool CO>
 static LanesFn pick_rows2(int out, bool slow, int nb) {
-    if (out == OUT_CODES) return pick_rows3<BITS, OUT_CODES, LANES>(slow, nb);
-    if (out == OUT_BF16) return pick_rows3<BITS, OUT_BF16, LANES>(slow, nb);
-    return pick_rows3<BITS, OUT_GEMV, LANES>(slow, nb);
+    if (out == OUT_CODES) return pick_rows3<BITS, OUT_CODES, LANES, CO>(slow, nb);
+    if (out == OUT_BF16) return pick_rows3<BITS, OUT_BF16, LANES, CO>(slow, nb);
+    return pick_rows3<BITS, OUT_GEMV, LANES, CO>(slow, nb);
 }
 
-static LanesFn pick_rows(int bits, int out, bool slow, int nb, int lanes) {
-    if (bits == 4) return lanes == 64 ? pick_rows2<4, 64>(out, slow, nb) : pick_rows2<4, 32>(out, slow, nb);
-    return lanes == 64 ? pick_rows2<8, 64>(out, slow, nb) : pick_rows2<8, 32>(out, slow, nb);
+// consumption order: 32-lane tiles only (one lane per thread)
+static LanesFn pick_rows(int bits, int out, bool slow, int nb, int lanes, bool co) {
+    if (co) return bits == 4 ? pick_rows2<4, 32, true>(out, slow, nb) : pick_rows2<8, 32, true>(out, slow, nb);
+    if (bits == 4)
+        return lanes == 64 ? pick_rows2<4, 64, false>(out, slow, nb) : pick_rows2<4, 32, false>(out, slow, nb);
+    return lanes == 64 ? pick_rows2<8, 64, false>(out, slow, nb) : pick_rows2<8, 32, false>(out, slow, nb);
 }
 
 // Launch the row-tile kernel over `count` entries (table on device, or `one`).
 static int launch_rows(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
                        const GroupEntry &one, int32_t *status, cudaStream_t st) {
     bool slow = false;
-    const int bits = ts[0]->d.bits, lanes = ts[0]->d.lanes;
+    const int bits = ts[0]->d.bits, lanes = ts[0]->d.lanes, format = ts[0]->d.format;
+    const bool co = format == ENTRO_FORMAT_ROWS_CO;
+    if (co && lanes != 32) return ENTRO_E_INVAL;
     int max_words = 0;
     long long max_runs = 0, total = 0, units = 0;
     for (int i = 0; i < count; i++) {
         const DevTensor &d = ts[i]->d;
-        if (d.format != ENTRO_FORMAT_ROWS || d.bits != bits || d.lanes != lanes) return ENTRO_E_INVAL;
+        if (d.format != format || d.bits != bits || d.lanes != lanes) return ENTRO_E_INVAL;
         slow = slow || ts[i]->slow;
         max_words = std::max(max_words, d.max_chunk_words);
         max_runs = std::max(max_runs, d.chunk_symbols / lanes / kRun);
@@ -2210,10 +2223,10 @@ static int launch_rows(const TensorHandle *const *ts, int count, int out_kind, i
     DeviceInfo di;
     if (device_info(ts[0]->device, &di) != ENTRO_OK) return ENTRO_E_CUDA;
     const int nb = out_kind == OUT_GEMV && batch > 8 ? 2 : 1;
-    LanesFn fn = pick_rows(bits, out_kind, slow, nb, lanes);
+    LanesFn fn = pick_rows(bits, out_kind, slow, nb, lanes, co);
     const int stage_rows = max_words + kSlackRows;
     // a run slot for every run of a chunk, plus the runs a lane may complete past its last check
-    int run_buf_bytes = static_cast<int>(max_runs + wide_runs_per_check(bits, 6)) * rows_run_bytes(bits, lanes);
+    int run_buf_bytes = static_cast<int>(max_runs + wide_runs_per_check(bits, 8)) * rows_run_bytes(bits, lanes);
     // the GEMV parks two sets of partial sums (fp32 D fragments) in a warp's run buffer
     if (out_kind == OUT_GEMV) run_buf_bytes = std::max(run_buf_bytes, 2 * (lanes / 16) * nb * 4 * 32 * 4);
     int warps = (int)std::min<long long>(kMaxWarps, std::max<long long>(1, (units + di.sms - 1) / di.sms));
@@ -2248,7 +2261,7 @@ static int launch_rows(const TensorHandle *const *ts, int count, int out_kind, i
 // A grouped launch of tensors of one format.
 static int launch_group(const TensorHandle *const *ts, int count, int out_kind, int batch, const GroupEntry *d_table,
                         const GroupEntry &one, int32_t *status, cudaStream_t st) {
-    if (ts[0]->d.format == ENTRO_FORMAT_ROWS)
+    if (ts[0]->d.format == ENTRO_FORMAT_ROWS || ts[0]->d.format == ENTRO_FORMAT_ROWS_CO)
         return launch_rows(ts, count, out_kind, batch, d_table, one, status, st);
     return launch_lanes(ts, count, out_kind, batch, d_table, one, status, st);
 }
@@ -2328,7 +2341,8 @@ static int gemv_check(const TensorHandle *t, const void *x, int batch, const flo
     if (!t || !x || !y || batch < 1 || batch > kMaxBatch) return ENTRO_E_INVAL;
     if (reinterpret_cast<uintptr_t>(x) & 15) return ENTRO_E_INVAL;
     const DevTensor &d = t->d;
-    if (d.format == ENTRO_FORMAT_ROWS) return ENTRO_OK;  // any shape of the format (cols a multiple of 8)
+    if (d.format == ENTRO_FORMAT_ROWS || d.format == ENTRO_FORMAT_ROWS_CO)
+        return ENTRO_OK;  // any shape of the formats (cols a multiple of 8)
     if (d.format != ENTRO_FORMAT_LANES) return ENTRO_E_INVAL;
     if (d.cols <= 0 || d.cols % (kRun * d.lanes) || d.chunk_symbols % d.cols) return ENTRO_E_INVAL;
     return ENTRO_OK;

@@ -314,19 +314,93 @@ struct BitSink {
 
 // ------------------------------------------------------------ encoder
 
+// One tile in consumption order (the layout is described in blob_format.h).
+// Each lane's words are coded on their own; a pass over each lane's code
+// lengths finds the refill points where it takes its later words; sorting the
+// takes by (refill point, lane) gives their places.
+static int write_consumption_tile(const TileGeom &t, const uint8_t *q, int64_t cols, int L, int bits, int max_len,
+                                  int count_bytes, const uint32_t *code, const uint8_t *len, uint32_t *dst,
+                                  uint64_t dst_words) {
+    const int per_lookup = bits == 4 ? kCoCodes4 : kCoCodes8;
+    const bool each = max_len > kCoRefillEachAbove;
+    std::vector<std::vector<uint32_t>> words((size_t)L);
+    struct Take {
+        uint64_t point;
+        int lane;
+        uint32_t word;
+    };
+    std::vector<Take> takes;
+    std::vector<uint8_t> lens((size_t)t.width);
+    for (int l = 0; l < t.nrows; l++) {
+        const uint8_t *row = q + (t.row0 + l) * cols + t.col0;
+        uint64_t bits_l = 0;
+        for (int64_t k = 0; k < t.width; k++) {
+            lens[(size_t)k] = len[row[k]];
+            bits_l += len[row[k]];
+        }
+        std::vector<uint32_t> &w = words[(size_t)l];
+        w.assign((size_t)((bits_l + 31) / 32) + 1, 0u);
+        BitSink s{w.data(), 1};
+        for (int64_t k = 0; k < t.width; k++) s.put(code[row[k]], len[row[k]]);
+        s.flush();
+        w.resize((size_t)((bits_l + 31) / 32));
+        // the lane's refill points: count the bits each lookup takes
+        size_t next_word = std::min<size_t>(3, w.size());
+        int64_t i = 0;
+        uint32_t used_since = 0;
+        for (uint64_t j = 0; next_word < w.size(); j++) {
+            if ((each || (j & 1) == 0) && used_since >= 32) {
+                used_since -= 32;
+                takes.push_back({each ? j : j / 2, l, w[next_word++]});
+                if (next_word == w.size()) break;
+            }
+            if (i >= t.width) return ENTRO_E_INVAL;  // cannot happen: words left means codes left
+            if (lens[(size_t)i] > kCoPeekBits) {
+                used_since += lens[(size_t)i++];
+                continue;
+            }
+            uint32_t peek = 0;
+            for (int k = 0; k < per_lookup && i < t.width && peek + lens[(size_t)i] <= (uint32_t)kCoPeekBits; k++)
+                peek += lens[(size_t)i++];
+            used_since += peek;
+        }
+    }
+    std::stable_sort(takes.begin(), takes.end(), [](const Take &a, const Take &b) {
+        return a.point != b.point ? a.point < b.point : a.lane < b.lane;
+    });
+    const uint64_t hw = co_header_words((uint64_t)L, count_bytes);
+    const uint64_t need = hw + 3 * (uint64_t)L + takes.size();
+    if (((need + 3) & ~3ull) != dst_words) return ENTRO_E_INVAL;
+    std::memset(dst, 0, dst_words * 4);
+    uint8_t *hdr = reinterpret_cast<uint8_t *>(dst);  // little-endian host
+    for (int l = 0; l < L; l++) {
+        const uint32_t nw = (uint32_t)words[(size_t)l].size();
+        hdr[count_bytes * l] = (uint8_t)nw;
+        if (count_bytes == 2) hdr[2 * l + 1] = (uint8_t)(nw >> 8);
+    }
+    for (int r = 0; r < 3; r++)
+        for (int l = 0; l < L; l++)
+            if ((size_t)r < words[(size_t)l].size()) dst[hw + (uint64_t)L * r + l] = words[(size_t)l][(size_t)r];
+    uint64_t p = hw + 3 * (uint64_t)L;
+    for (const Take &tk : takes) dst[p++] = tk.word;
+    return ENTRO_OK;
+}
+
 static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_encode_opts *o, Blob **out) {
     if (!out || !o || rows < 0 || cols < 0) return ENTRO_E_INVAL;
     if ((rows * cols > 0) && !w) return ENTRO_E_INVAL;
     if (o->bits != 4 && o->bits != 8) return ENTRO_E_INVAL;
     if (o->quant_mode < 0 || o->quant_mode > 2) return ENTRO_E_INVAL;
-    if (o->format != ENTRO_FORMAT_SINGLE && o->format != ENTRO_FORMAT_LANES && o->format != ENTRO_FORMAT_ROWS)
+    if (o->format != ENTRO_FORMAT_SINGLE && o->format != ENTRO_FORMAT_LANES && o->format != ENTRO_FORMAT_ROWS &&
+        o->format != ENTRO_FORMAT_ROWS_CO)
         return ENTRO_E_INVAL;
     if (o->threads < 0) return ENTRO_E_INVAL;
     const int bits = o->bits, nsym = 1 << bits;
     const int max_len = o->max_len ? o->max_len : (bits == 8 ? 16 : 12);
     if (max_len < 1 || max_len > kMaxLenLimit) return ENTRO_E_INVAL;
-    const bool tiles = o->format == ENTRO_FORMAT_ROWS;
-    const bool lanes = o->format == ENTRO_FORMAT_LANES || tiles;  // word-interleaved lanes
+    const bool consume = o->format == ENTRO_FORMAT_ROWS_CO;
+    const bool tiles = o->format == ENTRO_FORMAT_ROWS || consume;
+    const bool lanes = o->format == ENTRO_FORMAT_LANES || tiles;  // lane bitstreams
     const int L = lanes ? (o->lanes ? o->lanes : kLanes) : 1;
     if (lanes && L != 32 && L != 64) return ENTRO_E_INVAL;
     const int64_t step = (int64_t)kRun * L;
@@ -367,6 +441,7 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     const uint64_t n_chunks = tiles ? tile_count((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C)
                                     : n > 0 ? (uint64_t)((n + C - 1) / C) : 0;
     std::vector<uint64_t> start(n_chunks + 1, 0);
+    const int count_bytes = co_count_bytes((uint64_t)(C / L), (uint32_t)max_len);
 
     // pass 1: per-chunk size (bits for single stream, words for lanes)
     std::vector<uint64_t> csize(n_chunks, 0);
@@ -375,14 +450,16 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
             const int64_t a = c * C, b = std::min<int64_t>(n, a + C);
             if (tiles) {
                 const TileGeom t = tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, (uint64_t)c);
-                uint64_t wmax = 0;
+                uint64_t wmax = 0, later = 0;
                 for (int l = 0; l < t.nrows; l++) {
                     const uint8_t *row = q.data() + (t.row0 + l) * cols + t.col0;
                     uint64_t s = 0;
                     for (int64_t k = 0; k < t.width; k++) s += len[row[k]];
                     wmax = std::max<uint64_t>(wmax, (s + 31) / 32);
+                    later += (s + 31) / 32 > 3 ? (s + 31) / 32 - 3 : 0;
                 }
-                csize[c] = wmax * (uint64_t)L;
+                csize[c] = consume ? (co_header_words((uint64_t)L, count_bytes) + 3 * (uint64_t)L + later + 3) & ~3ull
+                                   : wmax * (uint64_t)L;
             } else if (!lanes) {
                 uint64_t s = 0;
                 for (int64_t i = a; i < b; i++) s += len[q[i]];
@@ -440,11 +517,17 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
     uint32_t *payload = reinterpret_cast<uint32_t *>(base + payload_offset(n_chunks));
 
     // pass 2: bits
+    std::atomic<int> failed{ENTRO_OK};
     parallel_for(threads, (int64_t)n_chunks, [&](int64_t c0, int64_t c1, int) {
         std::vector<uint32_t> tmp;
         for (int64_t c = c0; c < c1; c++) {
             const int64_t a = c * C, b = std::min<int64_t>(n, a + C);
-            if (tiles) {
+            if (consume) {
+                const TileGeom t = tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, (uint64_t)c);
+                const int r2 = write_consumption_tile(t, q.data(), cols, L, bits, max_len, count_bytes, code, len,
+                                                      payload + start[c], start[c + 1] - start[c]);
+                if (r2 != ENTRO_OK) failed.store(r2, std::memory_order_relaxed);
+            } else if (tiles) {
                 const TileGeom t = tile_geom((uint64_t)rows, (uint64_t)cols, (uint64_t)L, (uint64_t)C, (uint64_t)c);
                 uint32_t *cbase = payload + start[c];
                 for (int l = 0; l < t.nrows; l++) {
@@ -485,7 +568,8 @@ static int encode_impl(const float *w, int64_t rows, int64_t cols, const entro_e
             }
         }
     });
-    r = blob->finalize_info();
+    r = failed.load();
+    if (r == ENTRO_OK) r = blob->finalize_info();
     if (r != ENTRO_OK) {
         delete blob;
         return r;
@@ -509,7 +593,8 @@ int Blob::finalize_info() {
     if (h.bits != 4 && h.bits != 8) return ENTRO_E_FORMAT;
     if (h.scheme > 1) return ENTRO_E_FORMAT;
     if (h.max_len < 1 || h.max_len > (uint32_t)kMaxLenLimit) return ENTRO_E_FORMAT;
-    const bool tiles = h.format == ENTRO_FORMAT_ROWS;
+    const bool consume = h.format == ENTRO_FORMAT_ROWS_CO;
+    const bool tiles = h.format == ENTRO_FORMAT_ROWS || consume;
     const bool lanes = h.format == ENTRO_FORMAT_LANES || tiles;
     if (!lanes && h.format != ENTRO_FORMAT_SINGLE) return ENTRO_E_FORMAT;
     if (lanes ? (h.lanes != 32 && h.lanes != 64) : h.lanes != 1) return ENTRO_E_FORMAT;
@@ -554,8 +639,15 @@ int Blob::finalize_info() {
         if (c == 0 ? st != 0 : st < prev) return ENTRO_E_FORMAT;
         if (c > 0 && lanes) {
             const uint64_t wc = st - prev;
-            if (wc % h.lanes) return ENTRO_E_FORMAT;
-            maxw = std::max<uint64_t>(maxw, wc / h.lanes);
+            if (consume) {  // header + three rows at least, whole 16-byte groups
+                if (wc % 4 || wc < co_header_words(h.lanes, co_count_bytes(h.chunk_symbols / h.lanes, h.max_len)) +
+                                       3ull * h.lanes)
+                    return ENTRO_E_FORMAT;
+                maxw = std::max<uint64_t>(maxw, (wc + h.lanes - 1) / h.lanes);
+            } else {
+                if (wc % h.lanes) return ENTRO_E_FORMAT;
+                maxw = std::max<uint64_t>(maxw, wc / h.lanes);
+            }
         }
         if (c > 0 && !lanes) maxw = std::max<uint64_t>(maxw, (st + 31) / 32 - prev / 32);
         prev = st;

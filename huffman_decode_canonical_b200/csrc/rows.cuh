@@ -26,6 +26,11 @@
 
 constexpr int kRowsBlock = 8;  // runs per emission block
 
+// The consumption-order format is defined by a reference decoder; this one must
+// take the same codes per lookup and refill at the same points.
+static_assert(kCoPeekBits == kMaxLutBits && kCoCodes4 == wide_max_codes(4) && kCoCodes8 == wide_max_codes(8),
+              "consumption order: lookups as the format defines them");
+
 // Run-buffer geometry: a run of every lane, then the next run.  4-bit: one
 // word per lane, runs LANES + 8 words apart; 8-bit: two words per lane, runs
 // 2 * (LANES + 4) words apart.  The pads put the slots that one fragment load
@@ -160,12 +165,13 @@ __device__ __forceinline__ void rows_store_y(const GroupEntry &g, const DevTenso
 // barrier: the warp that began it adds the other warps' partial sums in warp
 // order (a fixed order: results do not depend on timing).  OUT_CODES /
 // OUT_BF16: warps take tiles in turn.
-template <int BITS, int OUT, bool SLOW, int LANES, int NB>
+template <int BITS, int OUT, bool SLOW, int LANES, int NB, bool CO>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_constant__ LaunchArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     constexpr int LPT = LANES / kLanes;  // lanes (rows) per thread
     constexpr int kMT = LANES / 16;      // 16-row MMA tiles per row group
-    constexpr int kStepsPerCheck = 6;
+    constexpr int kStepsPerCheck = 8;
+    constexpr int kUnit = CO ? 4 : LANES;  // chunk sizes are multiples of it
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
     const Pipes pk{a.k_one, a.k_one << 2, a.k_one << 3, a.k_one << 8, a.k_one << 12, a.k_one << 24};
@@ -239,8 +245,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
             const uint64_t st0 = __shfl_sync(0xffffffffu, iv, 0), nx0 = __shfl_sync(0xffffffffu, iv, 1);
             const uint64_t st1 = __shfl_sync(0xffffffffu, iv, 2), nx1 = __shfl_sync(0xffffffffu, iv, 3);
             if (lane == 0) {
-                if (c0 >= 0) issue_words(d, st0, nx0, stage, bar, a.stage_rows, LANES);
-                if (c1 >= 0) issue_words(d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES);
+                if (c0 >= 0) issue_words(d, st0, nx0, stage, bar, a.stage_rows, LANES, kUnit);
+                if (c1 >= 0) issue_words(d, st1, nx1, stage + buf_words, bar + 1, a.stage_rows, LANES, kUnit);
             }
             pend0 = c0 >= 0;
             pend1 = c1 >= 0;
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
             __syncthreads();
             return;
         }
-        const bool refill_each = SLOW && d.max_len > 16;
+        const bool refill_each = SLOW && d.max_len > kCoRefillEachAbove;
         float acc[kMT][NB][4];
         float hacc[kMT][NB][4];           // partial sums of a row group begun by an earlier warp
         long long head_g = -1, tail_g = -1;  // row groups of this warp's partial sums (hacc, acc)
@@ -310,18 +316,32 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                         for (int i = 0; i < 4; i++) acc[m][nb][i] = 0.f;
             }
             const uint64_t wst = d.index[2 * c], wnx = d.index[2 * c + 2];
-            if (wnx >= wst && wnx <= static_cast<uint64_t>(d.payload_words) && (wnx - wst) % LANES == 0 &&
-                (wnx - wst) / LANES + kSlackRows <= static_cast<uint64_t>(a.stage_rows)) {
+            // consumption order: a count header, then three rows of every lane's first words
+            const int cbytes = CO ? co_count_bytes(static_cast<uint64_t>(sh.Kc), static_cast<uint32_t>(d.max_len)) : 0;
+            const uint32_t hwords = CO ? static_cast<uint32_t>(co_header_words(LANES, cbytes)) : 0u;
+            if (wnx >= wst && wnx <= static_cast<uint64_t>(d.payload_words) && (wnx - wst) % kUnit == 0 &&
+                (!CO || wnx - wst >= hwords + 3u * LANES) &&
+                (wnx - wst + LANES - 1) / LANES + kSlackRows <= static_cast<uint64_t>(a.stage_rows)) {
                 const uint32_t *buf = stage + b * buf_words;
                 const int words = static_cast<int>((wnx - wst) / LANES);
-                WideDecoder<BITS, SLOW, LANES, rows_run_bytes(BITS, LANES), 0> ld[LPT];
+                WideDecoder<BITS, SLOW, LANES, rows_run_bytes(BITS, LANES), 0, CO> ld[LPT];
                 uint32_t read_limit[LPT];
 #pragma unroll
                 for (int q = 0; q < LPT; q++) {
                     const int l = lane + kLanes * q;
-                    ld[q].init(wlut, smem_addr(buf + l), runbuf + l * rows_lane_bytes(BITS), a.stage_rows - 1,
-                               l < nrows);
-                    read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
+                    if (CO) {
+                        const uint32_t base = smem_addr(buf), cw = static_cast<uint32_t>(wnx - wst);
+                        const uint8_t *hdr = reinterpret_cast<const uint8_t *>(buf);
+                        const uint32_t nw = cbytes == 1 ? hdr[l] : hdr[2 * l] | (static_cast<uint32_t>(hdr[2 * l + 1]) << 8);
+                        ld[q].init_co(wlut, base + 4u * (hwords + l), runbuf + l * rows_lane_bytes(BITS),
+                                      base + 4u * (hwords + 3u * LANES), nw > 3u ? nw - 3u : 0u, base + 4u * (cw - 1u),
+                                      l < nrows);
+                        read_limit[q] = base + 4u * cw;  // the cursor may end here, not past it
+                    } else {
+                        ld[q].init(wlut, smem_addr(buf + l), runbuf + l * rows_lane_bytes(BITS), a.stage_rows - 1,
+                                   l < nrows);
+                        read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
+                    }
                 }
                 // GEMV: this thread's row of x (batch row 8 nb + gid) at the tile's first column
                 const __nv_bfloat16 *xrow[NB];
@@ -379,8 +399,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                 }
                 bool ok = true;
 #pragma unroll
-                for (int q = 0; q < LPT; q++)
-                    if (lane + kLanes * q < nrows) ok = ok && ld[q].bufa <= read_limit[q];
+                for (int q = 0; q < LPT; q++) {
+                    if (CO) {
+                        // every lane took all its words, and no more words than the chunk holds
+                        if (ld[q].left != 0) set_status(a.status, ENTRO_E_CORRUPT);
+                        ok = ok && ld[q].cur <= read_limit[q];
+                    } else if (lane + kLanes * q < nrows) {
+                        ok = ok && ld[q].bufa <= read_limit[q];
+                    }
+                }
                 if (!ok) set_status(a.status, ENTRO_E_OVERRUN);
             } else {
                 set_status(a.status, ENTRO_E_CORRUPT);
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
             if (cn >= 0) {
                 if (lane == 0) {
                     fence_proxy_async();
-                    issue_chunk(d, cn, stage + b * buf_words, bar + b, a.stage_rows, LANES);
+                    issue_chunk(d, cn, stage + b * buf_words, bar + b, a.stage_rows, LANES, kUnit);
                 }
                 if (b) pend1 = true;
                 else pend0 = true;

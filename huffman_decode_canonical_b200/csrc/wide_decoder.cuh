@@ -56,8 +56,12 @@ __device__ __forceinline__ uint32_t byte_of(uint32_t v, uint32_t sel) {  // byte
 
 // RB: bytes from a lane's slot of run t to its slot of run t + 1.  RING = 0:
 // every run has its own slot; RING > 0: RING slots used in turn (run t in slot
-// t mod RING).
-template <int BITS, bool SLOW, int LANES, uint32_t RB, int RING>
+// t mod RING).  CO: the chunk's words are in consumption order (row tiles,
+// format 4): after its first three words a lane takes its next word from a
+// cursor shared by the warp, in lane order among the lanes that refill at the
+// same point (a ballot and a population count), and only while it has words
+// left; the loop that drives it must keep the warp converged.
+template <int BITS, bool SLOW, int LANES, uint32_t RB, int RING, bool CO = false>
 struct WideDecoder {
     static constexpr uint32_t kRowBytes = 4 * LANES;  // one staged word of every lane
     static constexpr uint32_t kRunBytes = RB;
@@ -70,6 +74,9 @@ struct WideDecoder {
     uint32_t p0, p1;      // pending codes as one bit string, first code at bit 0 of p0 (p1: 8-bit only)
     uint32_t osta;        // shared address of the current run's slot
     uint32_t rend;        // RING > 0: address one ring past this lane's slot of run 0
+    uint32_t cur;         // CO: shared address of the chunk's next unplaced word (same in every lane)
+    uint32_t left;        // CO: words this lane has still to take
+    uint32_t lt;          // CO: the lanes below this one
 
     // b: shared address of this lane's word 0 (word j at b + kRowBytes j);
     // slot0: its slot of run 0; cap: last readable staging row.
@@ -86,11 +93,60 @@ struct WideDecoder {
         rend = slot0 + static_cast<uint32_t>(RING) * RB;
     }
 
+    // Consumption order: b = this lane's word 0 (rows of kRowBytes as above),
+    // next = the chunk's first word after the three rows, words = the words this
+    // lane has after those three, last = the chunk's last word.
+    __device__ __forceinline__ void init_co(uint32_t table, uint32_t b, uint32_t slot0, uint32_t next, uint32_t words,
+                                           uint32_t last, bool active) {
+        tab = table;
+        bufa = b;
+        bufcap = last;
+        hi = lds32(b);
+        lo = lds32(b + kRowBytes);
+        wnext = lds32(b + 2 * kRowBytes);
+        C = active ? 0u : 0xFFFF0000u;
+        p0 = p1 = 0;
+        osta = slot0;
+        rend = slot0 + static_cast<uint32_t>(RING) * RB;
+        cur = next;
+        left = words;
+        asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
+    }
+
     __device__ __forceinline__ int runs() const { return static_cast<int>(C >> kRunsShift); }
 
     // When 32 or more window bits are consumed (the valid bits then all sit in
     // hi and lo is zero), the next word lands right below them.
     __device__ __forceinline__ void refill(const Pipes &k) {
+        if (CO) {
+            // every lane of the warp runs this (the ballot); a lane that refills and has words
+            // left takes the word at cur + 4 * (refilling lanes below it)
+            asm volatile(
+                "{\n\t"
+                ".reg .pred p, t;\n\t"
+                ".reg .u32 x, m, r, a;\n\t"
+                "and.b32 x, %2, 32;\n\t"
+                "setp.ne.u32 p, x, 0;\n\t"
+                "setp.ne.and.u32 t, %5, 0, p;\n\t"
+                "vote.sync.ballot.b32 m, t, 0xffffffff;\n\t"
+                "and.b32 r, m, %7;\n\t"
+                "popc.b32 r, r;\n\t"
+                "@p shf.l.wrap.b32 x, %3, 0, %2;\n\t"  // wnext >> (32 - s), s = consumed - 32
+                "@p mad.lo.u32 %0, x, %8, %0;\n\t"     // hi |= x
+                "@p shf.l.wrap.b32 %1, 0, %3, %2;\n\t"  // wnext << s
+                "@p mad.lo.u32 %2, %8, %9, %2;\n\t"    // consumed - 32
+                "@t mad.lo.u32 a, r, %10, %4;\n\t"
+                "@t min.u32 a, a, %6;\n\t"
+                "@t ld.shared.u32 %3, [a];\n\t"
+                "@t sub.u32 %5, %5, 1;\n\t"
+                "popc.b32 m, m;\n\t"
+                "mad.lo.u32 %4, m, %10, %4;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(wnext), "+r"(cur), "+r"(left)
+                : "r"(bufcap), "r"(lt), "r"(k.one), "r"(0xFFFFFFE0u), "r"(k.four)
+                : "memory");
+            return;
+        }
         asm volatile(
             "{\n\t"
             ".reg .pred p;\n\t"
@@ -163,7 +219,31 @@ struct WideDecoder {
     }
 
     __device__ __forceinline__ void advance_linear(const Pipes &k, uint32_t codes, uint32_t meta) {
-        if (BITS == 4) {
+        if (BITS == 4 && RING == 0) {
+            // every run of a slot-per-run buffer completes (row tiles: Kc is a multiple of 8),
+            // so a lane stores its run word once, when the run is whole
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 q, plo, phi, x;\n\t"
+                ".reg .pred dn;\n\t"
+                "shf.l.wrap.b32 %0, %1, %0, %7;\n\t"
+                "shf.l.wrap.b32 %1, 0, %1, %7;\n\t"
+                "mul.hi.u32 q, %2, %9;\n\t"
+                "shf.l.wrap.b32 plo, 0, %6, q;\n\t"
+                "shf.l.wrap.b32 phi, %6, 0, q;\n\t"
+                "mad.lo.u32 %3, plo, %8, %3;\n\t"
+                "mad.lo.u32 %2, %7, %8, %2;\n\t"
+                "and.b32 x, %2, 0x2000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "@dn st.shared.u32 [%4], %3;\n\t"
+                "selp.b32 %3, phi, %3, dn;\n\t"
+                "@dn mad.lo.u32 %2, %8, %10, %2;\n\t"
+                "@dn mad.lo.u32 %4, %8, %5, %4;\n\t"
+                "}"
+                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xE000u)
+                : "memory");
+        } else if (BITS == 4) {
             // pending bits < 32 before the append; what passes bit 32 (phi) starts the next run
             asm volatile(
                 "{\n\t"
@@ -223,9 +303,9 @@ struct WideDecoder {
 // Advance every lane the thread serves to at least run te, STEPS lookups per
 // check, until every lane of the warp has reached te; a lane that is ahead
 // keeps decoding up to run cap (the chunk's end).
-template <int STEPS, int BITS, bool SLOW, int LANES, uint32_t RB, int RING, int LPT>
-__device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB, RING> (&ld)[LPT], const Pipes &pk,
-                                               const uint32_t *slim,
+template <int STEPS, int BITS, bool SLOW, int LANES, uint32_t RB, int RING, bool CO, int LPT>
+__device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB, RING, CO> (&ld)[LPT],
+                                               const Pipes &pk, const uint32_t *slim,
                                                const int32_t *soffs, const uint8_t *ssyms, int te, int cap,
                                                int max_len, bool refill_each, int32_t *status) {
     const uint32_t te_c = static_cast<uint32_t>(te) << kRunsShift, cap_c = static_cast<uint32_t>(cap) << kRunsShift;
@@ -234,7 +314,19 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB
 #pragma unroll
         for (int k = 0; k < LPT; k++) behind = behind || ld[k].C < te_c;
         if (!__any_sync(0xffffffffu, behind)) break;
-        if (LPT == 1) {
+        if (CO) {
+            // the refills' ballot needs the whole warp: a lane at its chunk's end runs
+            // no-op lookups (and, having no words left, takes none)
+            static_assert(!CO || LPT == 1, "consumption order: one lane per thread");
+            const bool live = ld[0].C < cap_c;
+#pragma unroll
+            for (int h = 0; h < STEPS / 2; h++) {
+                ld[0].refill(pk);
+                ld[0].step_if(live, pk, slim, soffs, ssyms, max_len, status);
+                if (SLOW && refill_each) ld[0].refill(pk);
+                ld[0].step_if(live, pk, slim, soffs, ssyms, max_len, status);
+            }
+        } else if (LPT == 1) {
             if (ld[0].C < cap_c) {
 #pragma unroll
                 for (int h = 0; h < STEPS / 2; h++) {

@@ -69,6 +69,11 @@ extern "C" {
 #define ENTRO_FORMAT_ROWS 3   /* row tiles: a chunk is L = 32 (or 64) rows by chunk_symbols / L columns,
                                  lane l holding row l of the tile; word-interleaved like LANES.  Made for
                                  the fused GEMV; cols must be a multiple of 8 */
+#define ENTRO_FORMAT_ROWS_CO 4 /* row tiles in consumption order: the tiles and lane bitstreams of ROWS,
+                                  each lane keeping only its own words (a per-lane word count leads the
+                                  chunk), stored in the order a lock-step decoder takes them instead of
+                                  padded to the tile's longest lane.  Decodes through every call ROWS
+                                  does (32-lane tiles) */
 
 typedef struct entro_encode_opts {
     int32_t bits;          /* 4 or 8 */

@@ -6,7 +6,9 @@ Expected values come from the oracle only (quantize -> codes, dequantize -> bf16
 bit patterns, fp64 GEMV).  Shapes cover ragged row groups (rows not a multiple of
 the tile height), ragged column tiles, tiles narrower than a 4-run MMA group, both
 tile heights, 4- and 8-bit codes, codes longer than the 12-bit table (limits 16 and
-20) and a binding limit below it (9), and a one-symbol alphabet.
+20) and a binding limit below it (9), and a one-symbol alphabet.  The 32-lane cases
+run again in consumption order (format 4), whose layout is checked against the
+oracle's bytes before the decode.
 """
 import numpy as np
 import pytest
@@ -63,19 +65,28 @@ def _ids(c):
     return f"{c[0]}-b{c[1]}-m{c[2]}-L{c[3]}-c{c[4]}-l{c[5]}-{c[6]}x{c[7]}"
 
 
-def _encode(entro, case):
+def _encode(entro, case, consumption=False):
     kind, bits, mode, lmax, chunk, lanes, rows, cols = case
     w = workloads.small_tensor(kind, rows, cols, seed=rows * 7 + cols)
     q, s, z, _ = oracle.quantize(w, bits, _mode(mode))
-    blob = entro.Blob.encode(w, bits=bits, quant_mode=mode, max_len=lmax, fmt=entro.FORMAT_ROWS,
-                             chunk_symbols=chunk, lanes=lanes)
+    fmt = entro.FORMAT_ROWS_CO if consumption else entro.FORMAT_ROWS
+    blob = entro.Blob.encode(w, bits=bits, quant_mode=mode, max_len=lmax, fmt=fmt, chunk_symbols=chunk, lanes=lanes)
+    if consumption:   # the stored layout is the oracle's, byte for byte
+        assert blob.to_bytes() == oracle.encode(w, bits, _mode(mode), lmax, oracle.FMT_ROWS_CO, chunk, lanes=lanes)
     return entro.upload(blob), q, s, z
 
 
+# consumption order (format 4): the 32-lane cases
+CO_CASES = [c for c in CASES if c[5] == 32]
+
+
+@pytest.mark.parametrize("consumption", [False, True], ids=["padded", "consumption"])
 @pytest.mark.parametrize("case", CASES, ids=[_ids(c) for c in CASES])
-def test_rows_decode_codes_and_bf16(entro, case):
+def test_rows_decode_codes_and_bf16(entro, case, consumption):
     bits = case[1]
-    dt, q, s, z = _encode(entro, case)
+    if consumption and case[5] != 32:
+        pytest.skip("consumption order: 32-lane tiles")
+    dt, q, s, z = _encode(entro, case, consumption)
     st = _status()
     codes = dt.decode_codes(status=st)
     bf = dt.decode_dequant_bf16(status=st)
@@ -110,14 +121,65 @@ def test_rows_gemv(entro, case, batch):
     assert torch.equal(y, y2)
 
 
-def test_rows_group_gemv_and_bf16(entro):
+@pytest.mark.parametrize("batch", [1, 5, 16])
+@pytest.mark.parametrize("case", CO_CASES, ids=[_ids(c) for c in CO_CASES])
+def test_rows_consumption_order_gemv(entro, case, batch):
+    """The same products from the consumption-order layout: within the tolerance of the
+    oracle, and bit for bit the padded layout's (the same codes, the same summation)."""
+    dt, q, s, z = _encode(entro, case, consumption=True)
+    err, y = _gemv_err(dt, q, s, z, batch, seed=batch)
+    assert err <= GEMV_TOL, err
+    dt2, _, _, _ = _encode(entro, case)
+    _, y2 = _gemv_err(dt2, q, s, z, batch, seed=batch)
+    assert torch.equal(y, y2)
+
+
+def test_rows_consumption_order_needs_32_lanes(entro):
+    w = workloads.small_tensor("laplace", 130, 520, seed=1)
+    dt = entro.upload(entro.Blob.encode(w, bits=4, fmt=entro.FORMAT_ROWS_CO, chunk_symbols=16384, lanes=64))
+    with pytest.raises(entro.EntroError) as e:
+        dt.decode_codes(status=_status())
+    assert e.value.code == entro.E_INVAL
+
+
+def test_rows_consumption_order_corrupt(entro):
+    """A lane's word count raised far past its words (it runs out of codes with words
+    still to take) is reported; a count one too high (its extra word shifts the later
+    lanes' words) and random payload bits end with a status, never a hang."""
+    w = workloads.small_tensor("laplace", 64, 1024, seed=3)
+    blob = entro.Blob.encode(w, bits=4, fmt=entro.FORMAT_ROWS_CO, chunk_symbols=8192)
+    for extra, allowed in ((40, (entro.E_CORRUPT, entro.E_OVERRUN)), (1, (0, entro.E_CORRUPT, entro.E_OVERRUN))):
+        dt = entro.upload(blob)
+        off = _payload_offset(dt)
+        dt.mem[off + 5] += extra                      # chunk 0, lane 5's count
+        torch.cuda.synchronize()
+        st = _status()
+        dt.decode_codes(status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) in allowed
+    dt = entro.upload(blob)
+    off = _payload_offset(dt)
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    dt.mem[off: off + dt.info["payload_bytes"]] = torch.randint(
+        0, 256, (dt.info["payload_bytes"],), dtype=torch.uint8, device="cuda", generator=gen)
+    torch.cuda.synchronize()
+    st = _status()
+    dt.decode_dequant_bf16(status=st)
+    dt.decode_gemv(workloads.activations(0, 1, 1024).cuda(), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) in (0, entro.E_OVERRUN, entro.E_CORRUPT)
+
+
+@pytest.mark.parametrize("consumption", [False, True], ids=["padded", "consumption"])
+def test_rows_group_gemv_and_bf16(entro, consumption):
     """One grouped launch over tensors of different shapes (row groups split across CTAs)."""
     shapes = [(96, 512), (1000, 256), (33, 3072), (512, 1024)]
+    fmt = entro.FORMAT_ROWS_CO if consumption else entro.FORMAT_ROWS
     dts, qs = [], []
     for i, (r, c) in enumerate(shapes):
         w = workloads.small_tensor("laplace", r, c, seed=100 + i)
         q, s, z, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
-        blob = entro.Blob.encode(w, bits=4, quant_mode=entro.QUANT_ASYM, fmt=entro.FORMAT_ROWS, chunk_symbols=8192)
+        blob = entro.Blob.encode(w, bits=4, quant_mode=entro.QUANT_ASYM, fmt=fmt, chunk_symbols=8192)
         dts.append(entro.upload(blob))
         qs.append((q, s, z))
     for batch in (1, 4, 16):

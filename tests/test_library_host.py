@@ -62,6 +62,13 @@ CASES = [
     ("skew", 8, oracle.MODE_ASYM, 16, 3, 512, 33, 24),
     ("laplace", 4, oracle.MODE_ASYM, 12, 3, -1024, 130, 520),    # 64-row tiles
     ("t4", 8, oracle.MODE_ASYM, 16, 3, 256, 0, 16),
+    ("laplace", 4, oracle.MODE_ASYM, 12, 4, 8192, 100, 1000),     # row tiles in consumption order
+    ("t4", 8, oracle.MODE_AUTO, 16, 4, 4096, 70, 3072),
+    ("skew", 8, oracle.MODE_ASYM, 16, 4, 512, 33, 24),
+    ("skew", 8, oracle.MODE_ASYM, 20, 4, 2048, 64, 200),          # refill before every lookup
+    ("laplace", 4, oracle.MODE_ASYM, 12, 4, -1024, 130, 520),
+    ("constant", 8, oracle.MODE_AUTO, 16, 4, 256, 5, 80),
+    ("t4", 8, oracle.MODE_ASYM, 16, 4, 256, 0, 16),
 ]
 
 
@@ -102,18 +109,20 @@ def test_encoder_identical_on_single_tensor_workloads(name):
     assert got == ref
 
 
+@pytest.mark.parametrize("consumption", [False, True], ids=["padded", "consumption"])
 @pytest.mark.parametrize("name,index,rows", [("phi3_mini_u8", 1, 512), ("mistral_7b_u4", 6, 96)])
-def test_encoder_identical_on_model_shaped_tensor(name, index, rows):
-    """Model-shaped tensors in their workload's row-tile format: a Phi-3-mini-shaped o projection
-    (3072 columns, 32 x 128 tiles) and a Mistral-shaped down projection (14336 columns, 32 x 256
-    tiles, a ragged last row group)."""
+def test_encoder_identical_on_model_shaped_tensor(name, index, rows, consumption):
+    """Model-shaped tensors in their workload's row-tile format (and in consumption order): a
+    Phi-3-mini-shaped o projection (3072 columns, 32 x 128 tiles) and a Mistral-shaped down
+    projection (14336 columns, 32 x 256 tiles, a ragged last row group)."""
     W = workloads.get(name)
     spec = W.tensors[index]
     w = workloads.weights(W, spec).numpy()[:rows]
     C = W.chunk_symbols(spec.cols)
     assert W.fmt == oracle.FMT_ROWS
-    ref = oracle.encode(w, W.bits, W.quant_mode, W.max_len, W.fmt, C, lanes=W.lanes)
-    got = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=W.fmt,
+    fmt = oracle.FMT_ROWS_CO if consumption else W.fmt
+    ref = oracle.encode(w, W.bits, W.quant_mode, W.max_len, fmt, C, lanes=W.lanes)
+    got = entro.Blob.encode(w, bits=W.bits, quant_mode=W.quant_mode, max_len=W.max_len, fmt=fmt,
                             chunk_symbols=C, lanes=W.lanes).to_bytes()
     assert got == ref
 
@@ -134,7 +143,7 @@ def test_encoder_errors_match_oracle():
     assert e.value.code == entro.E_LIMIT
     with pytest.raises(oracle.OracleError):
         oracle.encode(many, 8, oracle.MODE_ASYM, 7, 2, 256)
-    for kw in ({"bits": 5}, {"fmt": 4}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25},
+    for kw in ({"bits": 5}, {"fmt": 5}, {"chunk_symbols": 300}, {"chunk_symbols": 32768}, {"max_len": 25},
                {"lanes": 48}, {"lanes": 64, "chunk_symbols": 768}, {"fmt": 3, "chunk_symbols": 300}):
         with pytest.raises(entro.EntroError):
             entro.Blob.encode(many, **kw)

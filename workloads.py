@@ -41,6 +41,7 @@ QUANT_ASYM = 2
 FORMAT_SINGLE = 1      # one bitstream per chunk
 FORMAT_LANES = 2       # 32 word-interleaved lane bitstreams per chunk
 FORMAT_ROWS = 3        # row tiles: lane l of a chunk is row l of a 32- or 64-row tile
+FORMAT_ROWS_CO = 4     # row tiles, each lane's words in consumption order (no lane padding)
 
 
 @dataclasses.dataclass(frozen=True)
