@@ -209,8 +209,7 @@ ENTRO_API const char *entro_strerror(int code);
  * on `stream` and launches; nothing is allocated or freed, on the host heap
  * or on the device.  The tensors' device must be the current device.  The
  * first call on a device looks up the table's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * All calls share the one table, so calls whose launches may overlap on the
+ * (cudaGetSymbolAddress).  All calls share the one table, so calls whose launches may overlap on the
  * GPU (other streams, other host threads) race: serialise them.  Errors:
  * ENTRO_E_LIMIT when count > ENTRO_STATIC_GROUP_MAX, otherwise as
  * entro_decode_gemv. */

@@ -82,5 +82,5 @@ def test_source_hash_ignores_comments_but_not_code(root):
 def test_committed_record_names_its_command():
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         t = json.load(f)
-    assert t["command"].startswith("ncu ") and "--clock-control none" in t["command"]
+    assert t["commands"] and all(c.startswith("ncu ") and "--clock-control none" in c for c in t["commands"])
     assert t["kernels"] and set(t["kernels"]) == set(t["warp_inst"])
