@@ -383,6 +383,10 @@ __host__ __device__ constexpr int runs_per_check(int lookups) {
     return (kRun - 1 + lookups * kMaxCodesPerLookup) / kRun;
 }
 constexpr int kLookupsPerCheck = 6;    // lanes kernel: table lookups between two checks of a lane's run count
+// the lanes kernel's two-word decoder: 6 lookups per check for 4-bit codes (up to 8 per
+// lookup, so the ring holds the overshoot), 8 for 8-bit codes (up to 4 per lookup)
+template <int BITS>
+__host__ __device__ constexpr int wide_lookups_per_check() { return BITS == 8 ? 8 : kLookupsPerCheck; }
 constexpr int kRunsPerCheck = runs_per_check(kLookupsPerCheck);
 constexpr int kLookahead = 3;          // lanes kernel: runs a lane may decode ahead into the next block
 static_assert(kRing >= kEmitBlock + kLookahead + kRunsPerCheck, "ring too small for the decode overshoot");
@@ -787,8 +791,8 @@ __device__ __forceinline__ void decode_to(LaneDecoder<BITS, SLOW, LANES> (&ld)[L
 // lane may complete past its last check fit the ring.
 template <int BITS>
 __host__ __device__ constexpr int wide_lookahead() {
-    return kRing - kEmitBlock - wide_runs_per_check(BITS, kLookupsPerCheck) < 3
-               ? kRing - kEmitBlock - wide_runs_per_check(BITS, kLookupsPerCheck)
+    return kRing - kEmitBlock - wide_runs_per_check(BITS, wide_lookups_per_check<BITS>()) < 3
+               ? kRing - kEmitBlock - wide_runs_per_check(BITS, wide_lookups_per_check<BITS>())
                : 3;
 }
 static_assert(wide_lookahead<4>() >= 1 && wide_lookahead<8>() >= 1, "ring too small for the wide decoder");
@@ -819,8 +823,8 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
 #pragma unroll
     for (int k = 0; k < LPT; k++) {
         const int l = lane + kLanes * k;
-        ld[k].init(smem_addr(s.lut), smem_addr(buf + l), smem_addr(ost + (BITS == 4 ? l : 2 * l)), stage_rows - 1,
-                   true);
+        ld[k].init(pk, smem_addr(s.lut), smem_addr(buf + l), smem_addr(ost + (BITS == 4 ? l : 2 * l)),
+                   stage_rows - 1, true);
         // a valid lane never moves more than kOverrunRows rows past its words
         read_limit[k] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
     }
@@ -840,7 +844,7 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
         for (int tb = 0; tb < runs; tb += kEmitBlock) {
             const int te = min(tb + kEmitBlock, runs);
             // a lane may run up to wide_lookahead runs into the next block, never past the chunk
-            wide_decode_to<kLookupsPerCheck>(ld, pk, s.slim, s.soffs, s.ssyms, te,
+            wide_decode_to<wide_lookups_per_check<BITS>()>(ld, pk, s.slim, s.soffs, s.ssyms, te,
                                              te < runs ? te + wide_lookahead<BITS>() : te, d.max_len, refill_each,
                                              status);
             __syncwarp();
@@ -863,17 +867,13 @@ __device__ __forceinline__ void decode_chunk(const GroupEntry &g, const Smem &s,
                 const int full_runs = S[k] >> 3, tail = S[k] & 7;
                 const int tf = min(te, full_runs);
                 while (ld[k].runs() < tf) {
-                    ld[k].refill(pk);
-                    ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
-                    if (SLOW && refill_each) ld[k].refill(pk);
-                    ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
+                    ld[k].step(pk, SLOW && refill_each, s.slim, s.soffs, s.ssyms, d.max_len, status);
+                    ld[k].step(pk, true, s.slim, s.soffs, s.ssyms, d.max_len, status);
                 }
                 // a partial last run: its slot holds the codes after every lookup
                 if (tail && full_runs < te)
-                    while (ld[k].runs() == full_runs && ((ld[k].C >> kPbShift) & 0xFFu) < tail * BITS) {
-                        ld[k].refill(pk);
-                        ld[k].step(pk, s.slim, s.soffs, s.ssyms, d.max_len, status);
-                    }
+                    while (ld[k].runs() == full_runs && ((ld[k].C >> kPbShift) & 0xFFu) < tail * BITS)
+                        ld[k].step(pk, true, s.slim, s.soffs, s.ssyms, d.max_len, status);
             }
             __syncwarp();
             emit_ragged<BITS, OUT, LANES>(g, s, ost, first, nc, tb, te);

@@ -333,12 +333,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                         const uint32_t base = smem_addr(buf), cw = static_cast<uint32_t>(wnx - wst);
                         const uint8_t *hdr = reinterpret_cast<const uint8_t *>(buf);
                         const uint32_t nw = cbytes == 1 ? hdr[l] : hdr[2 * l] | (static_cast<uint32_t>(hdr[2 * l + 1]) << 8);
-                        ld[q].init_co(wlut, base + 4u * (hwords + l), runbuf + l * rows_lane_bytes(BITS),
+                        ld[q].init_co(pk, wlut, base + 4u * (hwords + l), runbuf + l * rows_lane_bytes(BITS),
                                       base + 4u * (hwords + 3u * LANES), nw > 3u ? nw - 3u : 0u, base + 4u * (cw - 1u),
                                       l < nrows);
                         read_limit[q] = base + 4u * cw;  // the cursor may end here, not past it
                     } else {
-                        ld[q].init(wlut, smem_addr(buf + l), runbuf + l * rows_lane_bytes(BITS), a.stage_rows - 1,
+                        ld[q].init(pk, wlut, smem_addr(buf + l), runbuf + l * rows_lane_bytes(BITS), a.stage_rows - 1,
                                    l < nrows);
                         read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
                     }

@@ -65,6 +65,10 @@ template <int BITS, bool SLOW, int LANES, uint32_t RB, int RING, bool CO = false
 struct WideDecoder {
     static constexpr uint32_t kRowBytes = 4 * LANES;  // one staged word of every lane
     static constexpr uint32_t kRunBytes = RB;
+    // Load the next lookup's entry before the append (8-bit codes: ~3 codes per
+    // lookup, the append's work hides the load) or at the lookup (4-bit codes:
+    // measured faster that way).
+    static constexpr bool kAhead = BITS == 8;
     uint32_t tab;         // shared address of the {codes, meta} table
     uint32_t bufa;        // shared address of the word held in wnext (a refill advances, then loads)
     uint32_t bufcap;      // shared address of this lane's last readable word
@@ -77,10 +81,12 @@ struct WideDecoder {
     uint32_t cur;         // CO: shared address of the chunk's next unplaced word (same in every lane)
     uint32_t left;        // CO: words this lane has still to take
     uint32_t lt;          // CO: the lanes below this one
+    uint2 e;              // table entry of the window's top 12 bits, loaded one lookup ahead
 
     // b: shared address of this lane's word 0 (word j at b + kRowBytes j);
     // slot0: its slot of run 0; cap: last readable staging row.
-    __device__ __forceinline__ void init(uint32_t table, uint32_t b, uint32_t slot0, int cap, bool active) {
+    __device__ __forceinline__ void init(const Pipes &k, uint32_t table, uint32_t b, uint32_t slot0, int cap,
+                                         bool active) {
         tab = table;
         bufcap = b + kRowBytes * static_cast<uint32_t>(cap);
         hi = lds32(b);
@@ -91,13 +97,14 @@ struct WideDecoder {
         p0 = p1 = 0;
         osta = slot0;
         rend = slot0 + static_cast<uint32_t>(RING) * RB;
+        e = entry(k);
     }
 
     // Consumption order: b = this lane's word 0 (rows of kRowBytes as above),
     // next = the chunk's first word after the three rows, words = the words this
     // lane has after those three, last = the chunk's last word.
-    __device__ __forceinline__ void init_co(uint32_t table, uint32_t b, uint32_t slot0, uint32_t next, uint32_t words,
-                                           uint32_t last, bool active) {
+    __device__ __forceinline__ void init_co(const Pipes &k, uint32_t table, uint32_t b, uint32_t slot0, uint32_t next,
+                                           uint32_t words, uint32_t last, bool active) {
         tab = table;
         bufa = b;
         bufcap = last;
@@ -111,6 +118,7 @@ struct WideDecoder {
         cur = next;
         left = words;
         asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
+        e = entry(k);
     }
 
     __device__ __forceinline__ int runs() const { return static_cast<int>(C >> kRunsShift); }
@@ -170,41 +178,147 @@ struct WideDecoder {
         return lds64(imad(imulhi(hi, k.two12), k.eight, tab));  // table[window >> 52]
     }
 
-    // One table lookup: the entry of the window's top 12 bits, or, for a code
-    // longer than 12 bits, the canonical slow path's single code.
-    __device__ __forceinline__ void step(const Pipes &k, const uint32_t *slim, const int32_t *soffs,
-                                         const uint8_t *ssyms, int max_len, int32_t *status) {
-        uint2 e = entry(k);
-        if (SLOW && (e.y & 31u) == 0) {
+    // One lookup.  e, the entry of the window's top 12 bits, is loaded here or
+    // (kAhead) was loaded by the lookup before (or by init); for a code longer
+    // than 12 bits the canonical slow path gives the single code instead.  The
+    // window moves past the codes, a refill follows when r (a refill point
+    // comes next) and the codes are appended to the current run; with kAhead
+    // the next entry's load is issued before the append, whose integer work
+    // then runs while the load is in flight.  live = false (a lane at its
+    // chunk's end, kept in step with its warp) makes the lookup a no-op.
+    __device__ __forceinline__ void step(const Pipes &k, bool r, const uint32_t *slim, const int32_t *soffs,
+                                         const uint8_t *ssyms, int max_len, int32_t *status, bool live = true) {
+        if (!kAhead) e = entry(k);
+        uint32_t codes = live ? e.x : 0u, meta = live ? e.y : 0u;
+        if (SLOW && live && (meta & 31u) == 0) {
             const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
             const uint32_t se = slow_entry(win, max_len, slim, soffs, ssyms, status);
-            e.x = (se >> 8) & 0xFFu;
-            e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
+            codes = (se >> 8) & 0xFFu;
+            meta = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
         }
-        advance(k, e.x, e.y);
+        const uint32_t q = shift(k, meta);
+        if (kAhead) {
+            if (r) refill(k);
+            e = entry(k);
+            append(k, codes, q);
+        } else {
+            append(k, codes, q);
+            if (r) refill(k);
+        }
     }
 
-    // The same lookup, made a no-op (no bits consumed, no codes appended) for a
-    // lane that is done: lets the streams of a thread run in one basic block.
-    __device__ __forceinline__ void step_if(bool live, const Pipes &k, const uint32_t *slim, const int32_t *soffs,
-                                            const uint8_t *ssyms, int max_len, int32_t *status) {
-        uint2 e = entry(k);
-        e.x = live ? e.x : 0u;
-        e.y = live ? e.y : 0u;
-        if (SLOW && live && (e.y & 31u) == 0) {
-            const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
-            const uint32_t se = slow_entry(win, max_len, slim, soffs, ssyms, status);
-            e.x = (se >> 8) & 0xFFu;
-            e.y = (se & 31u) | (static_cast<uint32_t>(BITS) << kPbShift);
-        }
-        advance(k, e.x, e.y);
+    // Move the window past meta's bits and add meta to C; returns the pending
+    // bits before this lookup's codes (C >> 8; the shifts use it mod 32).
+    __device__ __forceinline__ uint32_t shift(const Pipes &k, uint32_t meta) {
+        uint32_t q;
+        asm volatile(
+            "mul.hi.u32 %0, %3, %5;\n\t"
+            "shf.l.wrap.b32 %1, %2, %1, %4;\n\t"
+            "shf.l.wrap.b32 %2, 0, %2, %4;\n\t"
+            "mad.lo.u32 %3, %4, %6, %3;\n\t"  // C += meta
+            : "=r"(q), "+r"(hi), "+r"(lo), "+r"(C)
+            : "r"(meta), "r"(k.two24), "r"(k.one));
+        return q;
     }
 
-    // Consume meta's bits, append the codes to the pending string, store the
-    // current run's slot, and move to the next slot when a run is whole.
-    // Appends land on zero bits of the string, so they are additions.
-    __device__ __forceinline__ void advance(const Pipes &k, uint32_t codes, uint32_t meta) {
-        advance_linear(k, codes, meta);
+    // Append the codes to the pending string at bit q, store the run's slot,
+    // and move to the next slot when a run is whole.  Appends land on zero bits
+    // of the string, so they are additions.
+    __device__ __forceinline__ void append(const Pipes &k, uint32_t codes, uint32_t q) {
+        if (BITS == 4 && RING == 0) {
+            // every run of a slot-per-run buffer completes (row tiles: Kc is a multiple of 8),
+            // so a lane stores its run word once, when the run is whole; what passes bit 32
+            // (phi) starts the next run (pending bits < 32 before the append)
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 plo, phi, x;\n\t"
+                ".reg .pred dn;\n\t"
+                "shf.l.wrap.b32 plo, 0, %4, %5;\n\t"
+                "shf.l.wrap.b32 phi, %4, 0, %5;\n\t"
+                "mad.lo.u32 %0, plo, %6, %0;\n\t"
+                "and.b32 x, %1, 0x2000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "@dn st.shared.u32 [%2], %0;\n\t"
+                "selp.b32 %0, phi, %0, dn;\n\t"
+                "@dn mad.lo.u32 %1, %6, %7, %1;\n\t"  // runs + 1, pending - 32
+                "@dn mad.lo.u32 %2, %6, %3, %2;\n\t"
+                "}"
+                : "+r"(p0), "+r"(C), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(q), "r"(k.one), "r"(0xE000u)
+                : "memory");
+        } else if (BITS == 4) {
+            // a ring: the slot holds the run so far after every lookup (a chunk's last run may
+            // stay partial)
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 plo, phi, x;\n\t"
+                ".reg .pred dn;\n\t"
+                "shf.l.wrap.b32 plo, 0, %4, %5;\n\t"
+                "shf.l.wrap.b32 phi, %4, 0, %5;\n\t"
+                "mad.lo.u32 %0, plo, %6, %0;\n\t"
+                "st.shared.u32 [%2], %0;\n\t"
+                "and.b32 x, %1, 0x2000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "selp.b32 %0, phi, %0, dn;\n\t"
+                "@dn mad.lo.u32 %1, %6, %7, %1;\n\t"
+                "@dn mad.lo.u32 %2, %6, %3, %2;\n\t"
+                "}"
+                : "+r"(p0), "+r"(C), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(q), "r"(k.one), "r"(0xE000u)
+                : "memory");
+        } else if (RING == 0) {
+            // pending bits < 64 before the append: below bit 32 of the string the codes
+            // go to p0 and what passes bit 32 to p1 (then zero); above, to p1 and past bit 64
+            // (phi) to the next run; the run's two words are stored once, when it is whole
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 plo, phi, x;\n\t"
+                ".reg .pred hs, dn;\n\t"
+                "shf.l.wrap.b32 plo, 0, %5, %6;\n\t"
+                "shf.l.wrap.b32 phi, %5, 0, %6;\n\t"
+                "and.b32 x, %6, 32;\n\t"
+                "setp.ne.u32 hs, x, 0;\n\t"
+                "selp.b32 %1, %1, phi, hs;\n\t"
+                "@!hs mad.lo.u32 %0, plo, %7, %0;\n\t"
+                "@hs mad.lo.u32 %1, plo, %7, %1;\n\t"
+                "and.b32 x, %2, 0x4000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "@dn st.shared.v2.u32 [%3], {%0, %1};\n\t"
+                "selp.b32 %0, phi, %0, dn;\n\t"
+                "selp.b32 %1, 0, %1, dn;\n\t"
+                "@dn mad.lo.u32 %2, %7, %8, %2;\n\t"  // runs + 1, pending - 64
+                "@dn mad.lo.u32 %3, %7, %4, %3;\n\t"
+                "}"
+                : "+r"(p0), "+r"(p1), "+r"(C), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(q), "r"(k.one), "r"(0xC000u)
+                : "memory");
+        } else {
+            // pending bits < 64 before the append: below bit 32 of the string the codes
+            // go to p0 and what passes bit 32 to p1 (then zero); above, to p1 and past bit 64
+            // (phi) to the next run; a ring's slot holds the run so far after every lookup
+            asm volatile(
+                "{\n\t"
+                ".reg .u32 plo, phi, x;\n\t"
+                ".reg .pred hs, dn;\n\t"
+                "shf.l.wrap.b32 plo, 0, %5, %6;\n\t"
+                "shf.l.wrap.b32 phi, %5, 0, %6;\n\t"
+                "and.b32 x, %6, 32;\n\t"
+                "setp.ne.u32 hs, x, 0;\n\t"
+                "selp.b32 %1, %1, phi, hs;\n\t"
+                "@!hs mad.lo.u32 %0, plo, %7, %0;\n\t"
+                "@hs mad.lo.u32 %1, plo, %7, %1;\n\t"
+                "st.shared.v2.u32 [%3], {%0, %1};\n\t"
+                "and.b32 x, %2, 0x4000;\n\t"
+                "setp.ne.u32 dn, x, 0;\n\t"
+                "selp.b32 %0, phi, %0, dn;\n\t"
+                "selp.b32 %1, 0, %1, dn;\n\t"
+                "@dn mad.lo.u32 %2, %7, %8, %2;\n\t"  // runs + 1, pending - 64
+                "@dn mad.lo.u32 %3, %7, %4, %3;\n\t"
+                "}"
+                : "+r"(p0), "+r"(p1), "+r"(C), "+r"(osta)
+                : "r"(kRunBytes), "r"(codes), "r"(q), "r"(k.one), "r"(0xC000u)
+                : "memory");
+        }
         if (RING > 0) {
             // the slot after the ring's last is its first
             asm volatile(
@@ -215,87 +329,6 @@ struct WideDecoder {
                 "}"
                 : "+r"(osta)
                 : "r"(rend), "n"(RING * RB));
-        }
-    }
-
-    __device__ __forceinline__ void advance_linear(const Pipes &k, uint32_t codes, uint32_t meta) {
-        if (BITS == 4 && RING == 0) {
-            // every run of a slot-per-run buffer completes (row tiles: Kc is a multiple of 8),
-            // so a lane stores its run word once, when the run is whole
-            asm volatile(
-                "{\n\t"
-                ".reg .u32 q, plo, phi, x;\n\t"
-                ".reg .pred dn;\n\t"
-                "shf.l.wrap.b32 %0, %1, %0, %7;\n\t"
-                "shf.l.wrap.b32 %1, 0, %1, %7;\n\t"
-                "mul.hi.u32 q, %2, %9;\n\t"
-                "shf.l.wrap.b32 plo, 0, %6, q;\n\t"
-                "shf.l.wrap.b32 phi, %6, 0, q;\n\t"
-                "mad.lo.u32 %3, plo, %8, %3;\n\t"
-                "mad.lo.u32 %2, %7, %8, %2;\n\t"
-                "and.b32 x, %2, 0x2000;\n\t"
-                "setp.ne.u32 dn, x, 0;\n\t"
-                "@dn st.shared.u32 [%4], %3;\n\t"
-                "selp.b32 %3, phi, %3, dn;\n\t"
-                "@dn mad.lo.u32 %2, %8, %10, %2;\n\t"
-                "@dn mad.lo.u32 %4, %8, %5, %4;\n\t"
-                "}"
-                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(osta)
-                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xE000u)
-                : "memory");
-        } else if (BITS == 4) {
-            // pending bits < 32 before the append; what passes bit 32 (phi) starts the next run
-            asm volatile(
-                "{\n\t"
-                ".reg .u32 q, plo, phi, x;\n\t"
-                ".reg .pred dn;\n\t"
-                "shf.l.wrap.b32 %0, %1, %0, %7;\n\t"
-                "shf.l.wrap.b32 %1, 0, %1, %7;\n\t"
-                "mul.hi.u32 q, %2, %9;\n\t"           // pending bits (C >> 8; the shifts use q mod 32)
-                "shf.l.wrap.b32 plo, 0, %6, q;\n\t"
-                "shf.l.wrap.b32 phi, %6, 0, q;\n\t"
-                "mad.lo.u32 %3, plo, %8, %3;\n\t"
-                "mad.lo.u32 %2, %7, %8, %2;\n\t"      // C += meta
-                "st.shared.u32 [%4], %3;\n\t"
-                "and.b32 x, %2, 0x2000;\n\t"
-                "setp.ne.u32 dn, x, 0;\n\t"
-                "selp.b32 %3, phi, %3, dn;\n\t"
-                "@dn mad.lo.u32 %2, %8, %10, %2;\n\t"  // runs + 1, pending - 32
-                "@dn mad.lo.u32 %4, %8, %5, %4;\n\t"
-                "}"
-                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(osta)
-                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xE000u)
-                : "memory");
-        } else {
-            // pending bits < 64 before the append: below bit 32 of the string the codes
-            // go to p0 and what passes bit 32 to p1 (then zero); above, to p1 and past bit 64
-            // (phi) to the next run
-            asm volatile(
-                "{\n\t"
-                ".reg .u32 q, plo, phi, x;\n\t"
-                ".reg .pred hs, dn;\n\t"
-                "shf.l.wrap.b32 %0, %1, %0, %8;\n\t"
-                "shf.l.wrap.b32 %1, 0, %1, %8;\n\t"
-                "mul.hi.u32 q, %2, %10;\n\t"
-                "shf.l.wrap.b32 plo, 0, %7, q;\n\t"
-                "shf.l.wrap.b32 phi, %7, 0, q;\n\t"
-                "and.b32 x, %2, 0x2000;\n\t"
-                "setp.ne.u32 hs, x, 0;\n\t"
-                "selp.b32 %4, %4, phi, hs;\n\t"
-                "@!hs mad.lo.u32 %3, plo, %9, %3;\n\t"
-                "@hs mad.lo.u32 %4, plo, %9, %4;\n\t"
-                "mad.lo.u32 %2, %8, %9, %2;\n\t"
-                "st.shared.v2.u32 [%5], {%3, %4};\n\t"
-                "and.b32 x, %2, 0x4000;\n\t"
-                "setp.ne.u32 dn, x, 0;\n\t"
-                "selp.b32 %3, phi, %3, dn;\n\t"
-                "selp.b32 %4, 0, %4, dn;\n\t"
-                "@dn mad.lo.u32 %2, %9, %11, %2;\n\t"  // runs + 1, pending - 64
-                "@dn mad.lo.u32 %5, %9, %6, %5;\n\t"
-                "}"
-                : "+r"(hi), "+r"(lo), "+r"(C), "+r"(p0), "+r"(p1), "+r"(osta)
-                : "r"(kRunBytes), "r"(codes), "r"(meta), "r"(k.one), "r"(k.two24), "r"(0xC000u)
-                : "memory");
         }
     }
 };
@@ -314,6 +347,8 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB
 #pragma unroll
         for (int k = 0; k < LPT; k++) behind = behind || ld[k].C < te_c;
         if (!__any_sync(0xffffffffu, behind)) break;
+        // refill points: after every second lookup, or after every lookup when refill_each
+        const bool r0 = SLOW && refill_each;
         if (CO) {
             // the refills' ballot needs the whole warp: a lane at its chunk's end runs
             // no-op lookups (and, having no words left, takes none)
@@ -321,19 +356,15 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB
             const bool live = ld[0].C < cap_c;
 #pragma unroll
             for (int h = 0; h < STEPS / 2; h++) {
-                ld[0].refill(pk);
-                ld[0].step_if(live, pk, slim, soffs, ssyms, max_len, status);
-                if (SLOW && refill_each) ld[0].refill(pk);
-                ld[0].step_if(live, pk, slim, soffs, ssyms, max_len, status);
+                ld[0].step(pk, r0, slim, soffs, ssyms, max_len, status, live);
+                ld[0].step(pk, true, slim, soffs, ssyms, max_len, status, live);
             }
         } else if (LPT == 1) {
             if (ld[0].C < cap_c) {
 #pragma unroll
                 for (int h = 0; h < STEPS / 2; h++) {
-                    ld[0].refill(pk);
-                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
-                    if (SLOW && refill_each) ld[0].refill(pk);
-                    ld[0].step(pk, slim, soffs, ssyms, max_len, status);
+                    ld[0].step(pk, r0, slim, soffs, ssyms, max_len, status);
+                    ld[0].step(pk, true, slim, soffs, ssyms, max_len, status);
                 }
             }
         } else {
@@ -344,14 +375,9 @@ __device__ __forceinline__ void wide_decode_to(WideDecoder<BITS, SLOW, LANES, RB
 #pragma unroll
             for (int h = 0; h < STEPS / 2; h++) {
 #pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].refill(pk);
+                for (int k = 0; k < LPT; k++) ld[k].step(pk, r0, slim, soffs, ssyms, max_len, status, live[k]);
 #pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
-                if (SLOW && refill_each)
-#pragma unroll
-                    for (int k = 0; k < LPT; k++) ld[k].refill(pk);
-#pragma unroll
-                for (int k = 0; k < LPT; k++) ld[k].step_if(live[k], pk, slim, soffs, ssyms, max_len, status);
+                for (int k = 0; k < LPT; k++) ld[k].step(pk, true, slim, soffs, ssyms, max_len, status, live[k]);
             }
         }
     }

@@ -136,7 +136,7 @@ WORKLOADS = {
         "single 4096x4096 tensor, Laplace(0, 0.015), asymmetric 4-bit, max code length 12, "
         "32 word-interleaved lanes per 8192-symbol chunk"),
     "smollm_1p7b_u8": Workload(
-        "smollm_1p7b_u8", 2, 8, QUANT_AUTO, 16, FORMAT_LANES, "fixed:8192",
+        "smollm_1p7b_u8", 2, 8, QUANT_AUTO, 16, FORMAT_ROWS, "fixed:4096",
         _smollm_1p7b(2),
         "SmolLM-1.7B-shaped (24 layers + 49152x2048 embedding), t(4) with per-tensor std "
         "U(0.01, 0.04), 10% shifted non-negative, mixed unsigned/asymmetric 8-bit"),
