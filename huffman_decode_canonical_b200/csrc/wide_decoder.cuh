@@ -65,10 +65,10 @@ template <int BITS, bool SLOW, int LANES, uint32_t RB, int RING, bool CO = false
 struct WideDecoder {
     static constexpr uint32_t kRowBytes = 4 * LANES;  // one staged word of every lane
     static constexpr uint32_t kRunBytes = RB;
-    // Load the next lookup's entry before the append (8-bit codes: ~3 codes per
-    // lookup, the append's work hides the load) or at the lookup (4-bit codes:
-    // measured faster that way).
-    static constexpr bool kAhead = BITS == 8;
+    // Load the next lookup's entry before the append, so that the append's work
+    // hides the load (8-bit codes, and the ring of the lanes kernel), or at the
+    // lookup (4-bit row tiles: measured faster that way).
+    static constexpr bool kAhead = BITS == 8 || RING > 0;
     uint32_t tab;         // shared address of the {codes, meta} table
     uint32_t bufa;        // shared address of the word held in wnext (a refill advances, then loads)
     uint32_t bufcap;      // shared address of this lane's last readable word
