@@ -54,7 +54,7 @@ def test_static_group_gemv_matches_group_launch():
     assert e.value.code == entro.E_LIMIT
 
 
-@pytest.mark.parametrize("fmt", ["lanes", "rows"])
+@pytest.mark.parametrize("fmt", ["lanes", "rows", "rows_co"])
 def test_static_group_gemv_many_tensors_against_oracle(fmt):
     """70 small tensors: the fixed table is filled in three host-to-device copies of up to
     32 entries, so the later copies' offsets and running chunk and symbol counts are used.
@@ -64,7 +64,7 @@ def test_static_group_gemv_many_tensors_against_oracle(fmt):
     import oracle
     import huffman_decode_canonical_b200 as entro
 
-    f = entro.FORMAT_ROWS if fmt == "rows" else entro.FORMAT_LANES
+    f = {"rows": entro.FORMAT_ROWS, "rows_co": entro.FORMAT_ROWS_CO, "lanes": entro.FORMAT_LANES}[fmt]
     batch = 2
     dts, xs, refs = [], [], []
     for i in range(70):
@@ -72,7 +72,7 @@ def test_static_group_gemv_many_tensors_against_oracle(fmt):
         w = workloads.small_tensor("laplace", r, c, seed=200 + i)
         q, s, z, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
         dt = entro.upload(entro.Blob.encode(w, bits=4, quant_mode=entro.QUANT_ASYM, fmt=f,
-                                            chunk_symbols=8192 if fmt == "rows" else max(1, 8192 // c) * c))
+                                            chunk_symbols=8192 if fmt != "lanes" else max(1, 8192 // c) * c))
         x = workloads.activations(300 + i, batch, c)
         refs.append(oracle.gemv(oracle.dequant_bf16(q, s, z).reshape(r, c), workloads.bf16_bits(x)))
         dts.append(dt)
