@@ -40,6 +40,12 @@ __host__ __device__ constexpr int rows_lane_bytes(int bits) { return bits == 4 ?
 __host__ __device__ constexpr int rows_run_bytes(int bits, int lanes) {
     return bits == 4 ? 4 * (lanes + 8) : 8 * (lanes + 4);
 }
+// Slot of row l within a run.  quad (the 4-bit 32-row GEMV at batch 9-16):
+// rows l, l + 8, l + 16, l + 24 are adjacent, so thread (gid, tig) fetches the
+// four slots it feeds to the tensor cores (rows gid + 8 j at one run) with one
+// 16-byte load, and a run's 32 slots stay in 32 different banks.  (At batch
+// 1-8 the plain order measured faster.)
+__host__ __device__ constexpr int rows_slot(bool quad, int l) { return quad ? 4 * (l & 7) + (l >> 3) : l; }
 
 struct RowsLayout {
     size_t wlut, vtab, vpair, slow, tbar, tags, bars, stage, runs, total;
@@ -75,16 +81,29 @@ __host__ __device__ inline RowsLayout rows_layout(int warps, int stage_words, in
     return o;
 }
 
+// the 8 4-bit codes of a run word -> 8 bf16 values (4 words, value of code i in half i)
+__device__ __forceinline__ uint4 run_values4(uint32_t word, uint32_t vpair, const Pipes &k) {
+    const uint32_t c = vpair_swizzle4(word);
+    uint4 v;
+    v.x = lds32(imad(byte_of(c, 0), k.four, vpair));
+    v.y = lds32(imad(byte_of(c, 1), k.four, vpair));
+    v.z = lds32(imad(byte_of(c, 2), k.four, vpair));
+    v.w = lds32(imad(imulhi(c, k.two8), k.four, vpair));
+    return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
 // 8 codes of a run slot -> 8 bf16 values (4 words, value of code i in half i)
 template <int BITS>
 __device__ __forceinline__ uint4 slot_values(uint32_t slot, uint32_t vtab, uint32_t vpair, const Pipes &k) {
     uint4 v;
     if (BITS == 4) {
-        const uint32_t c = vpair_swizzle4(lds32(slot));
-        v.x = lds32(imad(byte_of(c, 0), k.four, vpair));
-        v.y = lds32(imad(byte_of(c, 1), k.four, vpair));
-        v.z = lds32(imad(byte_of(c, 2), k.four, vpair));
-        v.w = lds32(imad(imulhi(c, k.two8), k.four, vpair));
+        v = run_values4(lds32(slot), vpair, k);
     } else {
         const uint2 c = lds64(slot);
         auto val = [&](uint32_t b) { return lds32(imad(b, k.four, vtab)); };
@@ -172,6 +191,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
     constexpr int kMT = LANES / 16;      // 16-row MMA tiles per row group
     constexpr int kStepsPerCheck = 8;
     constexpr int kUnit = CO ? 4 : LANES;  // chunk sizes are multiples of it
+    constexpr bool kQuad = BITS == 4 && LANES == 32 && OUT == OUT_GEMV && NB == 2;  // slot order, see rows_slot
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
     const Pipes pk{a.k_one, a.k_one << 2, a.k_one << 3, a.k_one << 8, a.k_one << 12, a.k_one << 24};
@@ -333,13 +353,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                         const uint32_t base = smem_addr(buf), cw = static_cast<uint32_t>(wnx - wst);
                         const uint8_t *hdr = reinterpret_cast<const uint8_t *>(buf);
                         const uint32_t nw = cbytes == 1 ? hdr[l] : hdr[2 * l] | (static_cast<uint32_t>(hdr[2 * l + 1]) << 8);
-                        ld[q].init_co(pk, wlut, base + 4u * (hwords + l), runbuf + l * rows_lane_bytes(BITS),
+                        ld[q].init_co(pk, wlut, base + 4u * (hwords + l), runbuf + rows_slot(kQuad, l) * rows_lane_bytes(BITS),
                                       base + 4u * (hwords + 3u * LANES), nw > 3u ? nw - 3u : 0u, base + 4u * (cw - 1u),
                                       l < nrows);
                         read_limit[q] = base + 4u * cw;  // the cursor may end here, not past it
                     } else {
-                        ld[q].init(pk, wlut, smem_addr(buf + l), runbuf + l * rows_lane_bytes(BITS), a.stage_rows - 1,
-                                   l < nrows);
+                        ld[q].init(pk, wlut, smem_addr(buf + l), runbuf + rows_slot(kQuad, l) * rows_lane_bytes(BITS),
+                                   a.stage_rows - 1, l < nrows);
                         read_limit[q] = smem_addr(buf + l) + 4u * LANES * static_cast<uint32_t>(words + kOverrunRows);
                     }
                 }
@@ -364,15 +384,31 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                             for (int nb = 0; nb < NB; nb++)
                                 xv[nb] = (t < te && 8 * nb + gid < a.batch) ? ldg_nc_v4(xrow[nb] + kRun * t)
                                                                             : make_uint4(0u, 0u, 0u, 0u);
-                            const uint32_t sl = runbuf + static_cast<uint32_t>(t) * RB + gid * LB;
+                            if (kQuad) {
+                                // the slots of rows gid, gid + 8, gid + 16, gid + 24 at run t
+                                const uint4 w4 = lds128(runbuf + static_cast<uint32_t>(t) * RB + 16u * gid);
+                                const uint32_t wr[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                            for (int m = 0; m < kMT; m++) {
-                                const uint4 wlo = slot_values<BITS>(sl + 16 * m * LB, vtab, vpair, pk);
-                                const uint4 whi = slot_values<BITS>(sl + (16 * m + 8) * LB, vtab, vpair, pk);
+                                for (int m = 0; m < kMT; m++) {
+                                    const uint4 wlo = run_values4(wr[2 * m], vpair, pk);
+                                    const uint4 whi = run_values4(wr[2 * m + 1], vpair, pk);
 #pragma unroll
-                                for (int nb = 0; nb < NB; nb++) {
-                                    mma_16816_bf16(acc[m][nb], wlo.x, whi.x, wlo.y, whi.y, xv[nb].x, xv[nb].y);
-                                    mma_16816_bf16(acc[m][nb], wlo.z, whi.z, wlo.w, whi.w, xv[nb].z, xv[nb].w);
+                                    for (int nb = 0; nb < NB; nb++) {
+                                        mma_16816_bf16(acc[m][nb], wlo.x, whi.x, wlo.y, whi.y, xv[nb].x, xv[nb].y);
+                                        mma_16816_bf16(acc[m][nb], wlo.z, whi.z, wlo.w, whi.w, xv[nb].z, xv[nb].w);
+                                    }
+                                }
+                            } else {
+                                const uint32_t sl = runbuf + static_cast<uint32_t>(t) * RB + gid * LB;
+#pragma unroll
+                                for (int m = 0; m < kMT; m++) {
+                                    const uint4 wlo = slot_values<BITS>(sl + 16 * m * LB, vtab, vpair, pk);
+                                    const uint4 whi = slot_values<BITS>(sl + (16 * m + 8) * LB, vtab, vpair, pk);
+#pragma unroll
+                                    for (int nb = 0; nb < NB; nb++) {
+                                        mma_16816_bf16(acc[m][nb], wlo.x, whi.x, wlo.y, whi.y, xv[nb].x, xv[nb].y);
+                                        mma_16816_bf16(acc[m][nb], wlo.z, whi.z, wlo.w, whi.w, xv[nb].z, xv[nb].w);
+                                    }
                                 }
                             }
                         }
