@@ -256,9 +256,14 @@ def test_corrupt_device_data_sets_status_without_hanging(entro):
         0, 256, (info["payload_bytes"],), dtype=torch.uint8, device="cuda", generator=gen)
     torch.cuda.synchronize()
     st = _status()
-    dt.decode_dequant_bf16(status=st)
+    bf = dt.decode_dequant_bf16(status=st)
     torch.cuda.synchronize()
-    assert int(st.item()) in (0, entro.E_OVERRUN, entro.E_CORRUPT)
+    code = int(st.item())
+    assert code in (0, entro.E_OVERRUN, entro.E_CORRUPT)
+    if code == 0:   # decoded without a complaint: then not to the original weights
+        q, s, z, _ = oracle.quantize(w, 4, oracle.MODE_ASYM)
+        got = bf.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
+        assert not np.array_equal(got, oracle.dequant_bf16(q, s, z))
 
 
 def test_decode_is_deterministic(entro):
