@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
     constexpr int kStepsPerCheck = 8;
     constexpr int kUnit = CO ? 4 : LANES;  // chunk sizes are multiples of it
     constexpr bool kQuad = BITS == 4 && LANES == 32 && OUT == OUT_GEMV && NB == 2;  // slot order, see rows_slot
+    constexpr bool kPreX = BITS == 4 && OUT == OUT_GEMV && NB == 1;  // activations loaded before a block's decode
     const int warps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;  // MMA fragment coordinates
     const Pipes pk{a.k_one, a.k_one << 2, a.k_one << 3, a.k_one << 8, a.k_one << 12, a.k_one << 24};
@@ -368,8 +369,19 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
 #pragma unroll
                 for (int nb = 0; nb < NB; nb++)
                     xrow[nb] = OUT == OUT_GEMV ? g.x + min(8 * nb + gid, a.batch - 1) * sh.K + col0 : nullptr;
+                const bool xlive0 = gid < a.batch;
                 for (int tb = 0; tb < runs; tb += kRowsBlock) {
                     const int te = min(tb + kRowsBlock, runs);
+                    // 4-bit GEMV at batch 1-8: the block's activations load while the block decodes
+                    // (8-bit: measured no better)
+                    uint4 xpre[kRowsBlock / 4];
+                    if constexpr (kPreX) {
+#pragma unroll
+                        for (int gq = 0; gq < kRowsBlock / 4; gq++) {
+                            const int tq = tb + 4 * gq + tig;
+                            xpre[gq] = (tq < te && xlive0) ? ldg_nc_v4(xrow[0] + kRun * tq) : make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
                     wide_decode_to<kStepsPerCheck>(ld, pk, slim, soffs, ssyms, te, runs, d.max_len, refill_each,
                                                    a.status);
                     __syncwarp();
@@ -377,13 +389,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                     if (OUT == OUT_GEMV) {
                         // groups of 4 runs = 32 columns: thread (gid, tig) supplies run t0 + tig of
                         // rows gid and gid + 8 of each 16-row tile (A) and of batch row 8 nb + gid (B)
-                        for (int t0 = tb; t0 < te; t0 += 4) {
+                        auto emit = [&](int t0, const uint4 (&xv)[NB]) {
                             const int t = t0 + tig;
-                            uint4 xv[NB];
-#pragma unroll
-                            for (int nb = 0; nb < NB; nb++)
-                                xv[nb] = (t < te && 8 * nb + gid < a.batch) ? ldg_nc_v4(xrow[nb] + kRun * t)
-                                                                            : make_uint4(0u, 0u, 0u, 0u);
                             if (kQuad) {
                                 // the slots of rows gid, gid + 8, gid + 16, gid + 24 at run t
                                 const uint4 w4 = lds128(runbuf + static_cast<uint32_t>(t) * RB + 16u * gid);
@@ -410,6 +417,24 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rows_kernel(const __grid_co
                                         mma_16816_bf16(acc[m][nb], wlo.z, whi.z, wlo.w, whi.w, xv[nb].z, xv[nb].w);
                                     }
                                 }
+                            }
+                        };
+                        if constexpr (kPreX) {
+#pragma unroll
+                            for (int gq = 0; gq < kRowsBlock / 4; gq++) {
+                                if (tb + 4 * gq >= te) break;
+                                const uint4 xv[NB] = {xpre[gq]};
+                                emit(tb + 4 * gq, xv);
+                            }
+                        } else {
+                            for (int t0 = tb; t0 < te; t0 += 4) {
+                                const int t = t0 + tig;
+                                uint4 xv[NB];
+#pragma unroll
+                                for (int nb = 0; nb < NB; nb++)
+                                    xv[nb] = (t < te && 8 * nb + gid < a.batch) ? ldg_nc_v4(xrow[nb] + kRun * t)
+                                                                                : make_uint4(0u, 0u, 0u, 0u);
+                                emit(t0, xv);
                             }
                         }
                     } else {
