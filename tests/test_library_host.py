@@ -174,6 +174,29 @@ def test_blob_bytes_roundtrip_and_validation():
         entro.Blob.from_bytes(data[:-4])
 
 
+def test_consumption_order_blob_validation():
+    """A consumption-order blob round-trips through bytes; a chunk whose word count is not a
+    whole number of 16-byte groups, or smaller than its header and first three rows, is
+    refused before anything reaches a device."""
+    w = workloads.small_tensor("laplace", 64, 1024, seed=4)
+    blob = entro.Blob.encode(w, bits=4, quant_mode=entro.QUANT_ASYM, fmt=entro.FORMAT_ROWS_CO, chunk_symbols=8192)
+    data = blob.to_bytes()
+    again = entro.Blob.from_bytes(data)
+    assert again.to_bytes() == data and again.info()["format"] == entro.FORMAT_ROWS_CO
+    info = blob.info()
+    # max_chunk_words: the staging rows a chunk needs (its words over 32 lanes, rounded up)
+    idx = np.frombuffer(data, np.uint64, 2 * (info["n_chunks"] + 1), 384).reshape(-1, 2)
+    sizes = np.diff(idx[:, 0].astype(np.int64))
+    assert info["max_chunk_words"] == int(-(-sizes.max() // 32))
+    assert (sizes % 4 == 0).all() and (sizes >= 8 + 3 * 32).all()
+    for start1 in (int(idx[1, 0]) + 1, 8 + 3 * 32 - 4):   # 1 word off; chunk 0 below header + three rows
+        bad = bytearray(data)
+        bad[384 + 16: 384 + 24] = np.uint64(start1).tobytes()
+        with pytest.raises(entro.EntroError) as e:
+            entro.Blob.from_bytes(bytes(bad))
+        assert e.value.code == entro.E_FORMAT
+
+
 def test_device_bytes_layout():
     w = workloads.small_tensor("t4", 64, 256, seed=2)
     blob = entro.Blob.encode(w, bits=8, chunk_symbols=2048)
